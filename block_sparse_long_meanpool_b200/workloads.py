@@ -1,0 +1,227 @@
+"""Seeded synthetic workloads for the MoBA prefill forward.
+
+This module only makes inputs: shapes, seeds and the value structure of the
+five workloads (block-offset keys, planted needle blocks, packed varlen
+sequences).  It holds none of the method's arithmetic (no block means, gate
+scores, selection or attention), so both the CUDA path and the float64 oracle
+can be fed from it.  It also holds the algorithmic FLOP count used to report
+throughput, which is a measurement formula, not part of the forward.
+
+Every tensor is drawn from a ``torch.Generator`` seeded per workload, in
+float32, then rounded to bf16 (round to nearest even).  The same call on the
+same device gives the same bits.
+"""
+
+from dataclasses import dataclass, field
+from typing import List, Optional
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    seqlens: List[int]
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    chunk_size: int
+    topk: int
+    structure: str  # "qk_offsets" | "k_offsets" | "needles"
+    seed: int
+    description: str = ""
+
+    @property
+    def total_tokens(self) -> int:
+        return int(sum(self.seqlens))
+
+    @property
+    def cu_seqlens(self) -> List[int]:
+        cu = [0]
+        for n in self.seqlens:
+            cu.append(cu[-1] + int(n))
+        return cu
+
+    @property
+    def max_seqlen(self) -> int:
+        return int(max(self.seqlens)) if self.seqlens else 0
+
+
+# The five workloads.  Shapes follow the analysis page's training/eval
+# settings (8K/512/top-3, 32K/512/top-3, 1M/4096/top-12) and a varlen GQA mix.
+WORKLOADS = {
+    "tiny_2k": Workload(
+        "tiny_2k", [2048], 4, 4, 64, 256, 3, "qk_offsets", 1001,
+        "1 x 2048 tokens, 4 heads MHA, d=64, chunk 256 (8 blocks), top-3"),
+    "scaling_8k": Workload(
+        "scaling_8k", [8192, 8192], 16, 16, 128, 512, 3, "k_offsets", 1002,
+        "2 x 8192 tokens, 16 heads MHA, d=128, chunk 512 (16 blocks), top-3"),
+    "long_32k": Workload(
+        "long_32k", [32768], 32, 32, 128, 512, 3, "needles", 1003,
+        "1 x 32768 tokens, 32 heads MHA, d=128, chunk 512 (64 blocks), top-3, 8 needle blocks"),
+    "varlen_gqa": Workload(
+        "varlen_gqa", [1000, 5000, 17000, 40000], 32, 8, 128, 1024, 4, "k_offsets", 1004,
+        "4 packed sequences {1000,5000,17000,40000}, 32 q / 8 kv heads, d=128, chunk 1024, top-4"),
+    "prefill_1m": Workload(
+        "prefill_1m", [1048576], 32, 8, 128, 4096, 12, "k_offsets", 1005,
+        "1 x 1,048,576 tokens, 32 q / 8 kv heads, d=128, chunk 4096 (256 blocks), top-12"),
+}
+
+
+def custom(name, seqlens, hq, hkv, d, chunk, topk, structure="k_offsets", seed=7):
+    """A workload of any shape with the same value recipe (for tests and sweeps)."""
+    return Workload(name, [int(x) for x in seqlens], hq, hkv, d, chunk, topk, structure, seed)
+
+
+def _block_layout(seqlens, chunk):
+    """Token -> (sequence, block start offsets) bookkeeping for planting structure."""
+    blocks = []  # (seq, start, end)
+    for i, (s, n) in enumerate(zip(_cum(seqlens), seqlens)):
+        for j in range((n + chunk - 1) // chunk):
+            blocks.append((i, s + j * chunk, min(s + (j + 1) * chunk, s + n)))
+    return blocks
+
+
+def _cum(seqlens):
+    out, acc = [], 0
+    for n in seqlens:
+        out.append(acc)
+        acc += n
+    return out
+
+
+def _token_block_ids(seqlens, chunk, device):
+    lens = [e - s for (_, s, e) in _block_layout(seqlens, chunk)]
+    ids = torch.arange(len(lens), device=device)
+    return torch.repeat_interleave(ids, torch.tensor(lens, device=device))
+
+
+def _randn(gen, shape, device, chunk_rows=1 << 16):
+    """N(0,1) float32, drawn in row chunks so that huge inputs stay bounded."""
+    out = torch.empty(shape, dtype=torch.bfloat16, device=device)
+    for r0 in range(0, shape[0], chunk_rows):
+        r1 = min(r0 + chunk_rows, shape[0])
+        out[r0:r1] = torch.randn((r1 - r0,) + tuple(shape[1:]), generator=gen,
+                                 device=device, dtype=torch.float32).to(torch.bfloat16)
+    return out
+
+
+def make_inputs(w: Workload, device="cpu", seed: Optional[int] = None):
+    """Seeded bf16 ``q [T,Hq,d]``, ``k``/``v [T,Hkv,d]`` and int32 ``cu_seqlens``.
+
+    Value recipe per structure:
+
+    * ``k_offsets``: q, k, v ~ N(0,1); every (block, kv head) draws an offset
+      vector ~ 0.5 N(0, I_d) that is added to each key row of that block.
+    * ``qk_offsets``: as ``k_offsets``; in addition a Bernoulli(0.1) subset of
+      query rows (t, h) gets the offset of a block chosen uniformly among the
+      blocks of its sequence that start at or before t.
+    * ``needles``: q, k, v ~ N(0,1); 8 distinct needle blocks per sequence
+      (uniform in 1..nb-2) each get a random unit direction u per kv head, and
+      2.0 u is added to each key row of the block.  A Bernoulli(0.05) subset of
+      query rows that have a needle block strictly before their own block is
+      replaced by |q| (0.8 u + 0.6 w), w a random unit vector orthogonal to
+      u, for one such needle chosen uniformly: cosine 0.8 with the planted
+      direction.
+    """
+    device = torch.device(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed if seed is None else seed)
+    T, hq, hkv, d, B = w.total_tokens, w.num_q_heads, w.num_kv_heads, w.head_dim, w.chunk_size
+    q = _randn(gen, (T, hq, d), device)
+    k = _randn(gen, (T, hkv, d), device)
+    v = _randn(gen, (T, hkv, d), device)
+    blocks = _block_layout(w.seqlens, B)
+    cu = torch.tensor(w.cu_seqlens, dtype=torch.int32, device=device)
+    if T == 0:
+        return {"q": q, "k": k, "v": v, "cu_seqlens": cu}
+
+    if w.structure in ("k_offsets", "qk_offsets"):
+        off = 0.5 * torch.randn((len(blocks), hkv, d), generator=gen, device=device)
+        bid = _token_block_ids(w.seqlens, B, device)
+        for r0 in range(0, T, 1 << 16):
+            r1 = min(r0 + (1 << 16), T)
+            k[r0:r1] = (k[r0:r1].float() + off[bid[r0:r1]]).to(torch.bfloat16)
+        if w.structure == "qk_offsets":
+            pick = torch.rand((T, hq), generator=gen, device=device) < 0.1
+            u = torch.rand((T, hq), generator=gen, device=device)
+            starts = torch.tensor([b[1] for b in blocks], device=device)
+            seq_first = torch.tensor(_first_block_of_seq(blocks, len(w.seqlens)), device=device)
+            seq_of_tok = torch.repeat_interleave(
+                torch.arange(len(w.seqlens), device=device),
+                torch.tensor(w.seqlens, device=device))
+            t = torch.arange(T, device=device)
+            first = seq_first[seq_of_tok]                                  # first block of t's sequence
+            n_avail = torch.searchsorted(starts, t, right=True) - first   # blocks starting <= t
+            pos = torch.minimum((u * n_avail[:, None]).long(), (n_avail - 1)[:, None])
+            j = first[:, None] + pos
+            grp = hq // hkv
+            heads = torch.arange(hq, device=device) // grp
+            add = off[j, heads[None, :]]                                   # [T, hq, d]
+            qf = q.float()
+            qf = torch.where(pick[..., None], qf + add, qf)
+            q = qf.to(torch.bfloat16)
+    elif w.structure == "needles":
+        grp = hq // hkv
+        qf = q.float()
+        kf = k.float()
+        for i, (s, n) in enumerate(zip(_cum(w.seqlens), w.seqlens)):
+            nb = (n + B - 1) // B
+            if nb < 4:
+                continue
+            cand = torch.randperm(nb - 2, generator=gen, device=device)[:8] + 1
+            needles, _ = torch.sort(cand)
+            dirs = torch.randn((len(needles), hkv, d), generator=gen, device=device)
+            dirs = dirs / dirs.norm(dim=-1, keepdim=True)
+            for a, j in enumerate(needles.tolist()):
+                r0, r1 = s + j * B, min(s + (j + 1) * B, s + n)
+                kf[r0:r1] += 2.0 * dirs[a][None]
+            pick = torch.rand((n, hq), generator=gen, device=device) < 0.05
+            u = torch.rand((n, hq), generator=gen, device=device)
+            wv = torch.randn((n, hq, d), generator=gen, device=device)
+            own = torch.arange(n, device=device) // B                       # own block, local
+            n_before = (needles[None, :] < own[:, None]).sum(dim=1)          # needles strictly before
+            which = torch.minimum((u * n_before[:, None]).long(), (n_before - 1).clamp(min=0)[:, None])
+            ok = pick & (n_before[:, None] > 0)
+            heads = torch.arange(hq, device=device) // grp
+            ud = dirs[which, heads[None, :]]                                 # [n, hq, d]
+            wv = wv - (wv * ud).sum(-1, keepdim=True) * ud
+            wv = wv / wv.norm(dim=-1, keepdim=True)
+            qs = qf[s:s + n]
+            newq = qs.norm(dim=-1, keepdim=True) * (0.8 * ud + 0.6 * wv)
+            qf[s:s + n] = torch.where(ok[..., None], newq, qs)
+        q = qf.to(torch.bfloat16)
+        k = kf.to(torch.bfloat16)
+    else:
+        raise ValueError(f"unknown structure {w.structure}")
+    return {"q": q.contiguous(), "k": k.contiguous(), "v": v.contiguous(), "cu_seqlens": cu}
+
+
+def _first_block_of_seq(blocks, nseq):
+    first = [0] * nseq
+    seen = set()
+    for idx, (i, _, _) in enumerate(blocks):
+        if i not in seen:
+            first[i] = idx
+            seen.add(i)
+    return first
+
+
+def selected_block_flops(seqlens, num_q_heads, head_dim, chunk, topk):
+    """Algorithmic FLOPs of the attention over the selected blocks.
+
+    4 * d * Hq * sum_t [ (t - s - c*B + 1) + B * min(topk - 1, c) ]: QK^T and
+    PV (2 FLOPs per multiply-add each) over the causal prefix of the row's own
+    block plus ``topk - 1`` whole past blocks (fewer for the first blocks).
+    Past candidate blocks are always full, so the count does not depend on
+    which blocks were chosen.
+    """
+    total = 0
+    for n in seqlens:
+        nb = (n + chunk - 1) // chunk
+        for c in range(nb):
+            rows = min(chunk, n - c * chunk)
+            causal = rows * (rows + 1) // 2
+            past = rows * chunk * min(topk - 1, c)
+            total += causal + past
+    return 4 * head_dim * num_q_heads * total

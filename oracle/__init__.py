@@ -1,0 +1,31 @@
+"""Float64 CPU oracle for the MoBA causal prefill forward.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import, call or
+execute this package: only the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` use it.  It shares
+no code, table or constant with the CUDA path under
+``block_sparse_long_meanpool_b200/``.
+
+Every function follows the plain definition of the method as stated on the
+page "《MoBA: Mixture of Block Attention for Long-Context LLMs》深度解读报告"
+(the zako-mio knowledge-base analysis of the MoBA paper), sections 2.1-2.3 and
+3.2, and on the course page "Paper: MoBA (Moonshot)" (module F26).  Where those
+pages are silent the reading taken is stated in the docstring.
+
+Parity pins: every function here is pinned by a ``-m "not gpu"`` test in
+``tests/test_oracle_pins.py`` against something other than itself (a library
+routine it reduces to, brute force, closed forms, the pages' printed sparsity
+figures).  No function is "parity unpinned".
+"""
+
+from .moba_ref import (  # noqa: F401
+    block_table,
+    block_means,
+    gate_scores_row,
+    select_blocks,
+    select_blocks_rows,
+    attend_rows,
+    attention_masked_dense,
+    moba_forward,
+    attended_keys,
+)
