@@ -1,0 +1,17 @@
+"""B200-native MoBA (Mixture of Block Attention) causal prefill forward.
+
+The compute path is the C-ABI library ``libmoba.so`` (CUDA for sm_100a, headers in
+``include/moba.h``); ``moba`` is its thin ctypes binding and ``workloads`` makes seeded
+synthetic inputs.  Build the library with ``python -m block_sparse_long_meanpool_b200.build``.
+"""
+
+from .moba import (  # noqa: F401
+    MobaError,
+    attn_fwd,
+    gate_topk,
+    load_library,
+    meanpool,
+    num_blocks,
+    workspace_size,
+    make_params,
+)

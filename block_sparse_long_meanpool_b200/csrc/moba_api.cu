@@ -1,0 +1,329 @@
+// Host side of the C ABI declared in include/moba.h: argument checks, workspace layout,
+// and the launch sequence of the MoBA prefill forward.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "moba.h"
+#include "moba_internal.cuh"
+
+using namespace moba;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+moba_status fail(moba_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+moba_status fail(moba_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+moba_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(MOBA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Shape checks common to every entry point.
+moba_status check_params(const moba_params* p) {
+    if (!p) return fail(MOBA_ERR_INVALID_ARG, "params is NULL");
+    if (p->batch < 1) return fail(MOBA_ERR_INVALID_ARG, "batch must be >= 1 (got %d)", p->batch);
+    if (p->total_tokens < 0)
+        return fail(MOBA_ERR_INVALID_ARG, "total_tokens must be >= 0 (got %d)", p->total_tokens);
+    if (p->num_q_heads < 1 || p->num_kv_heads < 1)
+        return fail(MOBA_ERR_INVALID_ARG, "head counts must be >= 1");
+    if (p->num_q_heads % p->num_kv_heads)
+        return fail(MOBA_ERR_INVALID_ARG, "num_q_heads (%d) %% num_kv_heads (%d) != 0",
+                    p->num_q_heads, p->num_kv_heads);
+    if (p->topk < 1) return fail(MOBA_ERR_INVALID_ARG, "topk must be >= 1 (got %d)", p->topk);
+    if (p->chunk_size < 1)
+        return fail(MOBA_ERR_INVALID_ARG, "chunk_size must be >= 1 (got %d)", p->chunk_size);
+    if (p->head_dim < 1) return fail(MOBA_ERR_INVALID_ARG, "head_dim must be >= 1");
+    if (p->wave_tokens < 0) return fail(MOBA_ERR_INVALID_ARG, "wave_tokens must be >= 0");
+    if (!(p->softmax_scale == p->softmax_scale) || std::isinf(p->softmax_scale))
+        return fail(MOBA_ERR_INVALID_ARG, "softmax_scale must be finite");
+    if (p->head_dim != 64 && p->head_dim != 128)
+        return fail(MOBA_ERR_UNSUPPORTED, "head_dim %d unsupported (64 or 128)", p->head_dim);
+    if (p->chunk_size % kTileM)
+        return fail(MOBA_ERR_UNSUPPORTED, "chunk_size %d unsupported (multiple of %d)",
+                    p->chunk_size, kTileM);
+    if (p->topk > 32) return fail(MOBA_ERR_UNSUPPORTED, "topk %d unsupported (<= 32)", p->topk);
+    if (p->wave_tokens % kTileM)
+        return fail(MOBA_ERR_UNSUPPORTED, "wave_tokens %d must be a multiple of %d",
+                    p->wave_tokens, kTileM);
+    if ((long long)p->num_q_heads * p->topk > (1 << 20))
+        return fail(MOBA_ERR_UNSUPPORTED, "num_q_heads * topk too large");
+    return MOBA_OK;
+}
+
+long long blocks_bound(const moba_params& p) {
+    if (p.total_tokens == 0) return 0;
+    long long nb = (p.total_tokens + (long long)p.chunk_size - 1) / p.chunk_size + p.batch - 1;
+    return nb < p.total_tokens ? nb : p.total_tokens;
+}
+
+struct Layout {
+    size_t hdr, cu_blocks, blk_start, blk_len, blk_seq, blk_local, means, sel, counts, offsets,
+        cursor, entries, items, part_o, part_lse, total;
+    int wave;
+    long long nb_cap, max_items;
+};
+
+Layout make_layout(const moba_params& p) {
+    Layout L{};
+    const long long T = p.total_tokens;
+    L.nb_cap = blocks_bound(p);
+    L.wave = (p.wave_tokens > 0 && p.wave_tokens < T) ? p.wave_tokens : (int)T;
+    const long long W = L.wave;
+    const long long lists = (long long)p.num_kv_heads * L.nb_cap;
+    const long long routed = W * p.num_q_heads * (p.topk - 1);
+    const long long past_items = routed / kTileM + (lists < routed ? lists : routed) + 1;
+    const long long blk_in_wave = L.nb_cap < W ? L.nb_cap : W;
+    const long long diag_items = (long long)p.num_q_heads * (W / kTileM + blk_in_wave + 4);
+    L.max_items = past_items + diag_items;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o = align_up(o + bytes);
+        return at;
+    };
+    L.hdr = take(sizeof(WsHeader));
+    L.cu_blocks = take(4ull * (p.batch + 1));
+    L.blk_start = take(4ull * L.nb_cap);
+    L.blk_len = take(4ull * L.nb_cap);
+    L.blk_seq = take(4ull * L.nb_cap);
+    L.blk_local = take(4ull * L.nb_cap);
+    L.means = take(4ull * L.nb_cap * p.num_kv_heads * p.head_dim);
+    L.sel = take(4ull * p.num_q_heads * T * p.topk);
+    L.counts = take(4ull * lists);
+    L.offsets = take(4ull * (lists + 1));
+    L.cursor = take(4ull * lists);
+    L.entries = take(4ull * routed);
+    L.items = take(sizeof(WorkItem) * L.max_items);
+    L.part_o = take(4ull * W * p.num_q_heads * p.topk * p.head_dim);
+    L.part_lse = take(4ull * W * p.num_q_heads * p.topk);
+    L.total = o;
+    return L;
+}
+
+Problem make_problem(const moba_params& p, long long nb_cap) {
+    Problem P;
+    P.batch = p.batch;
+    P.T = p.total_tokens;
+    P.hq = p.num_q_heads;
+    P.hkv = p.num_kv_heads;
+    P.d = p.head_dim;
+    P.chunk = p.chunk_size;
+    P.topk = p.topk;
+    P.group = p.num_q_heads / p.num_kv_heads;
+    P.nb_cap = (int)nb_cap;
+    P.scale = p.softmax_scale > 0.f ? p.softmax_scale : 1.0f / sqrtf((float)p.head_dim);
+    P.scale_log2 = P.scale * 1.4426950408889634f;
+    return P;
+}
+
+int device_sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return 148;
+    return n;
+}
+
+// Index-range limits of the 32-bit indices used on the device.
+moba_status check_ranges(const moba_params& p, const Layout& L) {
+    const long long lim = 0x7fffffffLL;
+    if ((long long)L.wave * p.num_q_heads * p.topk > lim)
+        return fail(MOBA_ERR_UNSUPPORTED,
+                    "wave_tokens * num_q_heads * topk exceeds 2^31; set a smaller wave_tokens");
+    if (L.max_items > lim || (long long)p.num_kv_heads * L.nb_cap > lim)
+        return fail(MOBA_ERR_UNSUPPORTED, "too many blocks for 32-bit work indices");
+    return MOBA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moba_num_blocks_bound(const moba_params* p) {
+    if (check_params(p) != MOBA_OK) return -1;
+    return (int)blocks_bound(*p);
+}
+
+size_t moba_workspace_size(const moba_params* p) {
+    if (check_params(p) != MOBA_OK) return 0;
+    return make_layout(*p).total;
+}
+
+moba_status moba_meanpool(const moba_params* p, const void* k, const int* cu_seqlens,
+                          float* k_mean, void* stream) {
+    moba_status s = check_params(p);
+    if (s != MOBA_OK) return s;
+    if (p->total_tokens == 0) return MOBA_OK;
+    if (!k || !cu_seqlens || !k_mean) return fail(MOBA_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned16(k) || !aligned16(k_mean))
+        return fail(MOBA_ERR_INVALID_ARG, "k and k_mean must be 16-byte aligned");
+    const Problem P = make_problem(*p, blocks_bound(*p));
+    cudaError_t e = launch_meanpool(P, static_cast<const __nv_bfloat16*>(k), cu_seqlens, k_mean,
+                                    static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "meanpool launch");
+    return MOBA_OK;
+}
+
+moba_status moba_gate_topk(const moba_params* p, const void* q, const float* k_mean,
+                           const int* cu_seqlens, int* sel, void* stream) {
+    moba_status s = check_params(p);
+    if (s != MOBA_OK) return s;
+    if (p->total_tokens == 0) return MOBA_OK;
+    if (!q || !k_mean || !cu_seqlens || !sel)
+        return fail(MOBA_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned16(q) || !aligned16(k_mean))
+        return fail(MOBA_ERR_INVALID_ARG, "q and k_mean must be 16-byte aligned");
+    const Problem P = make_problem(*p, blocks_bound(*p));
+    cudaError_t e = launch_gate(P, static_cast<const __nv_bfloat16*>(q), k_mean, cu_seqlens, sel,
+                                static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "gate launch");
+    return MOBA_OK;
+}
+
+moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, const void* v,
+                          const int* cu_seqlens, const int* sel_in, int* sel_out,
+                          void* workspace, size_t workspace_bytes, void* out, float* lse,
+                          moba_run_info* info, void* stream) {
+    moba_status s = check_params(p);
+    if (s != MOBA_OK) return s;
+    if (info) {
+        info->launches = 0;
+        info->waves = 0;
+    }
+    if (p->total_tokens == 0) return MOBA_OK;
+    if (!q || !k || !v || !cu_seqlens || !out || !lse)
+        return fail(MOBA_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return fail(MOBA_ERR_INVALID_ARG, "q, k, v and out must be 16-byte aligned");
+    const Layout L = make_layout(*p);
+    s = check_ranges(*p, L);
+    if (s != MOBA_OK) return s;
+    if (!workspace || workspace_bytes < L.total)
+        return fail(MOBA_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", L.total,
+                    workspace ? workspace_bytes : (size_t)0);
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+        return fail(MOBA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const Problem P = make_problem(*p, L.nb_cap);
+    char* base = static_cast<char*>(workspace);
+    Workspace ws;
+    ws.hdr = reinterpret_cast<WsHeader*>(base + L.hdr);
+    ws.cu_blocks = reinterpret_cast<int*>(base + L.cu_blocks);
+    ws.blk_start = reinterpret_cast<int*>(base + L.blk_start);
+    ws.blk_len = reinterpret_cast<int*>(base + L.blk_len);
+    ws.blk_seq = reinterpret_cast<int*>(base + L.blk_seq);
+    ws.blk_local = reinterpret_cast<int*>(base + L.blk_local);
+    ws.means = reinterpret_cast<float*>(base + L.means);
+    ws.sel = reinterpret_cast<int*>(base + L.sel);
+    ws.counts = reinterpret_cast<int*>(base + L.counts);
+    ws.offsets = reinterpret_cast<int*>(base + L.offsets);
+    ws.cursor = reinterpret_cast<int*>(base + L.cursor);
+    ws.entries = reinterpret_cast<int*>(base + L.entries);
+    ws.items = reinterpret_cast<WorkItem*>(base + L.items);
+    ws.part_o = reinterpret_cast<float*>(base + L.part_o);
+    ws.part_lse = reinterpret_cast<float*>(base + L.part_lse);
+
+    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
+    const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
+    const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(v);
+    int launches = 0;
+    auto record = [&](int idx) -> cudaError_t {
+        if (info && info->events && idx < info->n_events && info->events[idx])
+            return cudaEventRecord(static_cast<cudaEvent_t>(info->events[idx]), st);
+        return cudaSuccess;
+    };
+    cudaError_t e;
+#define MOBA_TRY(expr, what)                      \
+    do {                                          \
+        e = (expr);                               \
+        if (e != cudaSuccess) return cuda_fail(e, what); \
+    } while (0)
+
+    MOBA_TRY(record(MOBA_EV_BEGIN), "event record");
+    MOBA_TRY(launch_plan_blocks(P, cu_seqlens, ws, st), "block table launch");
+    MOBA_TRY(launch_meanpool(P, kb, cu_seqlens, ws.means, st), "meanpool launch");
+    launches += 2;
+    MOBA_TRY(record(MOBA_EV_MEANS_DONE), "event record");
+    const int* sel_use = sel_in;
+    if (!sel_use) {
+        int* dst = sel_out ? sel_out : ws.sel;
+        MOBA_TRY(launch_gate(P, qb, ws.means, cu_seqlens, dst, st), "gate launch");
+        ++launches;
+        sel_use = dst;
+    }
+    MOBA_TRY(record(MOBA_EV_GATE_DONE), "event record");
+
+    const int num_sms = device_sm_count();
+    const int T = p->total_tokens;
+    int w = 0;
+    for (int t0 = 0; t0 < T; t0 += L.wave, ++w) {
+        const int t1 = (T - t0 > L.wave) ? t0 + L.wave : T;
+        const int ev = MOBA_EV_WAVE0 + 4 * w;
+        MOBA_TRY(record(ev), "event record");
+        MOBA_TRY(cudaMemsetAsync(ws.counts, 0, 4ull * P.hkv * L.nb_cap, st), "memset");
+        MOBA_TRY(launch_route_count(P, cu_seqlens, sel_use, ws, t0, t1, st), "route count launch");
+        MOBA_TRY(launch_route_plan(P, ws, t0, t1, st), "route plan launch");
+        MOBA_TRY(launch_route_scatter(P, cu_seqlens, sel_use, ws, t0, t1, st), "route scatter launch");
+        MOBA_TRY(record(ev + 1), "event record");
+        MOBA_TRY(launch_attention(P, qb, kb, vb, ws, t0, t1, num_sms, st), "attention launch");
+        MOBA_TRY(record(ev + 2), "event record");
+        MOBA_TRY(launch_merge(P, cu_seqlens, sel_use, ws, t0, t1,
+                              static_cast<__nv_bfloat16*>(out), lse, st),
+                 "merge launch");
+        MOBA_TRY(record(ev + 3), "event record");
+        launches += 5;
+    }
+#undef MOBA_TRY
+    if (info) {
+        info->launches = launches;
+        info->waves = w;
+    }
+    return MOBA_OK;
+}
+
+moba_status moba_device_status(const moba_params* p, const void* workspace, void* stream) {
+    moba_status s = check_params(p);
+    if (s != MOBA_OK) return s;
+    if (!workspace) return fail(MOBA_ERR_WORKSPACE, "workspace is NULL");
+    int word = 0;
+    const WsHeader* hdr = static_cast<const WsHeader*>(workspace);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(&word, &hdr->status, sizeof(int), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "status read");
+    if (word == 0) return MOBA_OK;
+    return fail((moba_status)word, "device status word %d", word);
+}
+
+const char* moba_status_string(moba_status s) {
+    switch (s) {
+        case MOBA_OK: return "MOBA_OK";
+        case MOBA_ERR_INVALID_ARG: return "MOBA_ERR_INVALID_ARG";
+        case MOBA_ERR_UNSUPPORTED: return "MOBA_ERR_UNSUPPORTED";
+        case MOBA_ERR_WORKSPACE: return "MOBA_ERR_WORKSPACE";
+        case MOBA_ERR_CUDA: return "MOBA_ERR_CUDA";
+        case MOBA_ERR_DEVICE_TIMEOUT: return "MOBA_ERR_DEVICE_TIMEOUT";
+    }
+    return "MOBA_ERR_UNKNOWN";
+}
+
+const char* moba_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

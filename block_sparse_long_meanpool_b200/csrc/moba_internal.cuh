@@ -1,0 +1,160 @@
+// Internal declarations shared by the MoBA CUDA sources (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace moba {
+
+// Rows of a routed tile / query tile of the current block.
+constexpr int kTileM = 128;
+
+// Device-side header at the start of the workspace.
+struct WsHeader {
+    int nb_total;           // number of blocks (sum over sequences of ceil(L / B))
+    int status;             // 0 or a moba_status code written by a kernel
+    unsigned work_counter;  // persistent-kernel work cursor (zeroed per wave)
+    int n_items;            // work items of the current wave
+    int n_past_items;       // of which routed history tiles (the rest are current-block tiles)
+    int pad[11];
+};
+
+// One unit of attention work.
+//   kind 0 (history tile): a = list id (g * nb_cap + block), b = first entry, c = rows
+//   kind 1 (current-block tile): a = block, b = query head, c = query tile index
+struct WorkItem {
+    int a, b, c, kind;
+};
+
+// Problem description passed by value to kernels.
+struct Problem {
+    int batch, T, hq, hkv, d, chunk, topk;
+    int group;       // hq / hkv
+    int nb_cap;      // capacity of per-block arrays (upper bound of the block count)
+    float scale;     // softmax scale (natural units)
+    float scale_log2;  // scale * log2(e)
+};
+
+// Views into the workspace of one moba_attn_fwd call.
+struct Workspace {
+    WsHeader* hdr;
+    int* cu_blocks;   // [batch + 1]
+    int* blk_start;   // [nb_cap]
+    int* blk_len;     // [nb_cap]
+    int* blk_seq;     // [nb_cap]
+    int* blk_local;   // [nb_cap]
+    float* means;     // [nb_cap, hkv, d]
+    int* sel;         // [hq, T, topk]
+    int* counts;      // [hkv * nb_cap]
+    int* offsets;     // [hkv * nb_cap + 1]
+    int* cursor;      // [hkv * nb_cap]
+    int* entries;     // [wave * hq * (topk - 1)]
+    WorkItem* items;  // [max_items]
+    float* part_o;    // [wave * hq * topk, d]
+    float* part_lse;  // [wave * hq * topk]
+};
+
+// ---------------------------------------------------------------------------------------
+// Device helpers
+
+// Index of the sequence holding token t: the last i with cu[i] <= t (empty sequences skipped).
+__device__ __forceinline__ int seq_of_token(const int* __restrict__ cu, int batch, int t) {
+    int lo = 0, hi = batch;  // answer in [0, batch)
+    while (hi - lo > 1) {
+        int mid = (lo + hi) >> 1;
+        if (__ldg(cu + mid) <= t) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
+// Selection rule shared by routing and merge: entry i of a row is a routed history block iff
+// 0 <= j < c, it is not a repeat of an earlier routed entry, and fewer than topk-1 entries
+// have been routed before it.  Returns the number of routed entries and, for each routed
+// entry, calls f(slot, j) with slot = 1 + its rank among the routed entries.
+template <typename F>
+__device__ __forceinline__ int for_each_routed(const int* __restrict__ row, int topk, int c, F f) {
+    int n = 0;
+    for (int i = 0; i < topk; ++i) {
+        int j = row[i];
+        if (j < 0 || j >= c || n >= topk - 1) continue;
+        bool dup = false;
+        for (int i2 = 0; i2 < i; ++i2) dup |= (row[i2] == j);
+        if (dup) continue;
+        f(n + 1, j);
+        ++n;
+    }
+    return n;
+}
+
+// ---------------------------------------------------------------------------------------
+// Launchers (defined in the .cu files).  Each returns cudaGetLastError() of its launch.
+
+cudaError_t launch_plan_blocks(const Problem& P, const int* cu_seqlens, const Workspace& ws,
+                               cudaStream_t st);
+cudaError_t launch_meanpool(const Problem& P, const __nv_bfloat16* k, const int* cu_seqlens,
+                            float* means, cudaStream_t st);
+cudaError_t launch_gate(const Problem& P, const __nv_bfloat16* q, const float* means,
+                        const int* cu_seqlens, int* sel, cudaStream_t st);
+cudaError_t launch_route_count(const Problem& P, const int* cu_seqlens, const int* sel,
+                               const Workspace& ws, int t0, int t1, cudaStream_t st);
+cudaError_t launch_route_plan(const Problem& P, const Workspace& ws, int t0, int t1,
+                              cudaStream_t st);
+cudaError_t launch_route_scatter(const Problem& P, const int* cu_seqlens, const int* sel,
+                                 const Workspace& ws, int t0, int t1, cudaStream_t st);
+cudaError_t launch_attention(const Problem& P, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                             const __nv_bfloat16* v, const Workspace& ws, int t0, int t1,
+                             int num_sms, cudaStream_t st);
+cudaError_t launch_merge(const Problem& P, const int* cu_seqlens, const int* sel,
+                         const Workspace& ws, int t0, int t1, __nv_bfloat16* out, float* lse,
+                         cudaStream_t st);
+
+}  // namespace moba
+
+namespace moba {
+
+// Locates global block b without a precomputed block table: a warp scans the per-sequence
+// block counts ceil(L_i / chunk) over cu_seqlens.  Must be called by all 32 lanes of a warp;
+// every lane gets the same answer.  Returns false when b is past the last block.
+struct BlockRef {
+    int seq, local, start, len, first;  // first = global index of the sequence's block 0
+};
+
+__device__ __forceinline__ bool find_block(const int* __restrict__ cu, int batch, int chunk,
+                                           int b, BlockRef& r) {
+    const unsigned full = 0xffffffffu;
+    const int lane = threadIdx.x & 31;
+    int base = 0;
+    for (int i0 = 0; i0 < batch; i0 += 32) {
+        const int i = i0 + lane;
+        int s = 0, e = 0, n = 0;
+        if (i < batch) {
+            s = __ldg(cu + i);
+            e = __ldg(cu + i + 1);
+            n = (e - s + chunk - 1) / chunk;
+        }
+        int incl = n;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            int y = __shfl_up_sync(full, incl, off);
+            if (lane >= off) incl += y;
+        }
+        const int excl = incl - n;
+        const bool hit = (i < batch) && (b >= base + excl) && (b < base + incl);
+        const unsigned m = __ballot_sync(full, hit);
+        if (m) {
+            const int src = __ffs(m) - 1;
+            r.seq = __shfl_sync(full, i, src);
+            r.first = base + __shfl_sync(full, excl, src);
+            r.local = b - r.first;
+            r.start = __shfl_sync(full, s, src) + r.local * chunk;
+            const int e_src = __shfl_sync(full, e, src);
+            r.len = min(chunk, e_src - r.start);
+            return true;
+        }
+        base += __shfl_sync(full, incl, 31);
+    }
+    return false;
+}
+
+}  // namespace moba

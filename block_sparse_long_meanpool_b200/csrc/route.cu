@@ -1,0 +1,241 @@
+// Block table and the MoE-style dispatch of query rows to (KV head, block) lists.
+//
+// The analysis page of the MoBA paper (§3.2) computes the history blocks by regrouping the
+// queries per selected KV block, as in mixture-of-experts dispatch, and computes the
+// current block separately with a causal mask.  Here, per wave of query tokens [t0, t1):
+//
+//   route_count    histogram of routed rows per (KV head g, global block b)
+//   route_plan     exclusive scan -> list offsets; work items: the history tiles (<= 128 rows
+//                  of one list each), then the current-block tiles, largest first
+//   route_scatter  writes each routed row's partial-output index into its list
+//
+// A routed entry is the row's partial-output index ((t - t0) * Hq + h) * topk + slot, where
+// slot 0 is the own block and slots 1.. are the routed history blocks in row order.
+#include "moba_internal.cuh"
+
+namespace moba {
+
+namespace {
+
+constexpr int kPlanThreads = 1024;
+
+// Block-wide exclusive scan of one value per thread (kPlanThreads threads).  Returns the
+// exclusive prefix; *total receives the sum over the block.
+__device__ int block_exclusive_scan(int v, int* s_warp, int* total) {
+    const unsigned full = 0xffffffffu;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(full, incl, off);
+        if (lane >= off) incl += y;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = (lane < kPlanThreads / 32) ? s_warp[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(full, wi, off);
+            if (lane >= off) wi += y;
+        }
+        if (lane < kPlanThreads / 32) s_warp[lane] = wi - w;
+        if (lane == 31) s_warp[32] = wi;
+    }
+    __syncthreads();
+    const int res = s_warp[warp] + incl - v;
+    *total = s_warp[32];
+    __syncthreads();
+    return res;
+}
+
+__global__ void __launch_bounds__(kPlanThreads)
+plan_blocks_kernel(const int* __restrict__ cu, Problem P, Workspace ws) {
+    __shared__ int s_total;
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int i = 0; i < P.batch; ++i) {
+            ws.cu_blocks[i] = run;
+            const int n = cu[i + 1] - cu[i];
+            run += (n + P.chunk - 1) / P.chunk;
+        }
+        ws.cu_blocks[P.batch] = run;
+        ws.hdr->nb_total = run;
+        ws.hdr->status = 0;
+        s_total = run;
+    }
+    __syncthreads();
+    const int nb = s_total;
+    for (int b = threadIdx.x; b < nb; b += blockDim.x) {
+        int lo = 0, hi = P.batch;  // last sequence i with cu_blocks[i] <= b
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (ws.cu_blocks[mid] <= b) lo = mid; else hi = mid;
+        }
+        const int i = lo;
+        const int local = b - ws.cu_blocks[i];
+        const int start = cu[i] + local * P.chunk;
+        ws.blk_start[b] = start;
+        ws.blk_len[b] = min(P.chunk, cu[i + 1] - start);
+        ws.blk_seq[b] = i;
+        ws.blk_local[b] = local;
+    }
+}
+
+// One thread per query row (t, h) of the wave.  kScatter = false counts, true scatters.
+template <bool kScatter>
+__global__ void route_rows_kernel(const int* __restrict__ cu, const int* __restrict__ sel,
+                                  Problem P, Workspace ws, int t0, int t1) {
+    const long long n = (long long)(t1 - t0) * P.hq;
+    for (long long r = blockIdx.x * (long long)blockDim.x + threadIdx.x; r < n;
+         r += (long long)gridDim.x * blockDim.x) {
+        const int t = t0 + (int)(r / P.hq);
+        const int h = (int)(r % P.hq);
+        const int i = seq_of_token(cu, P.batch, t);
+        const int c = (t - __ldg(cu + i)) / P.chunk;
+        const int first = ws.cu_blocks[i];
+        const int g = h / P.group;
+        const int* row = sel + ((size_t)h * P.T + t) * P.topk;
+        int* lists = ws.counts + (size_t)g * P.nb_cap + first;
+        const int pbase = (int)(r * P.topk);
+        for_each_routed(row, P.topk, c, [&](int slot, int j) {
+            if (kScatter) {
+                const int pos = atomicAdd(ws.cursor + (size_t)g * P.nb_cap + first + j, 1);
+                ws.entries[pos] = pbase + slot;
+            } else {
+                atomicAdd(lists + j, 1);
+            }
+        });
+    }
+}
+
+__global__ void __launch_bounds__(kPlanThreads)
+route_plan_kernel(Problem P, Workspace ws, int t0, int t1) {
+    __shared__ int s_warp[33];
+    const int n_lists = P.hkv * P.nb_cap;
+    // 1. list offsets
+    int carry = 0;
+    for (int base = 0; base < n_lists; base += kPlanThreads) {
+        const int L = base + threadIdx.x;
+        const int cnt = (L < n_lists) ? ws.counts[L] : 0;
+        int tot;
+        const int ex = block_exclusive_scan(cnt, s_warp, &tot);
+        if (L < n_lists) {
+            ws.offsets[L] = carry + ex;
+            ws.cursor[L] = carry + ex;
+        }
+        carry += tot;
+    }
+    if (threadIdx.x == 0) ws.offsets[n_lists] = carry;
+    // 2. history tiles, list by list
+    int tcarry = 0;
+    for (int base = 0; base < n_lists; base += kPlanThreads) {
+        const int L = base + threadIdx.x;
+        const int cnt = (L < n_lists) ? ws.counts[L] : 0;
+        const int nt = (cnt + kTileM - 1) / kTileM;
+        int tot;
+        const int ex = block_exclusive_scan(nt, s_warp, &tot);
+        if (L < n_lists && nt > 0) {
+            const int off = ws.offsets[L];
+            for (int i = 0; i < nt; ++i) {
+                WorkItem it;
+                it.a = L;
+                it.b = off + i * kTileM;
+                it.c = min(kTileM, cnt - i * kTileM);
+                it.kind = 0;
+                ws.items[tcarry + ex + i] = it;
+            }
+        }
+        tcarry += tot;
+    }
+    const int n_past = tcarry;
+    // 3. current-block tiles of the blocks overlapping [t0, t1), by decreasing tile index
+    //    (tile q has q + 1 key tiles of work)
+    const int nb = ws.hdr->nb_total;
+    int lo = 0, hi = nb;  // first block whose end is > t0
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (ws.blk_start[mid] + ws.blk_len[mid] <= t0) lo = mid + 1; else hi = mid;
+    }
+    const int b_lo = lo;
+    lo = b_lo;
+    hi = nb;  // first block whose start is >= t1
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (ws.blk_start[mid] < t1) lo = mid + 1; else hi = mid;
+    }
+    const int b_hi = lo;
+    const int levels = (P.chunk + kTileM - 1) / kTileM;
+    int dcarry = n_past;
+    for (int qt = levels - 1; qt >= 0; --qt) {
+        for (int base = b_lo; base < b_hi; base += kPlanThreads) {
+            const int b = base + threadIdx.x;
+            int has = 0;
+            if (b < b_hi) {
+                const int r0 = qt * kTileM;
+                const int len = ws.blk_len[b];
+                if (r0 < len) {
+                    const int a = ws.blk_start[b] + r0;
+                    const int e = ws.blk_start[b] + min(r0 + kTileM, len);
+                    has = (a < t1 && e > t0) ? 1 : 0;
+                }
+            }
+            int tot;
+            const int ex = block_exclusive_scan(has, s_warp, &tot);
+            if (has) {
+                for (int h = 0; h < P.hq; ++h) {
+                    WorkItem it;
+                    it.a = b;
+                    it.b = h;
+                    it.c = qt;
+                    it.kind = 1;
+                    ws.items[dcarry + ex * P.hq + h] = it;
+                }
+            }
+            dcarry += tot * P.hq;
+        }
+    }
+    if (threadIdx.x == 0) {
+        ws.hdr->n_items = dcarry;
+        ws.hdr->n_past_items = n_past;
+        ws.hdr->work_counter = 0u;
+    }
+}
+
+int rows_grid(long long n) {
+    long long g = (n + 255) / 256;
+    if (g > 65536) g = 65536;
+    if (g < 1) g = 1;
+    return (int)g;
+}
+
+}  // namespace
+
+cudaError_t launch_plan_blocks(const Problem& P, const int* cu_seqlens, const Workspace& ws,
+                               cudaStream_t st) {
+    plan_blocks_kernel<<<1, kPlanThreads, 0, st>>>(cu_seqlens, P, ws);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_route_count(const Problem& P, const int* cu_seqlens, const int* sel,
+                               const Workspace& ws, int t0, int t1, cudaStream_t st) {
+    const long long n = (long long)(t1 - t0) * P.hq;
+    route_rows_kernel<false><<<rows_grid(n), 256, 0, st>>>(cu_seqlens, sel, P, ws, t0, t1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_route_plan(const Problem& P, const Workspace& ws, int t0, int t1,
+                              cudaStream_t st) {
+    route_plan_kernel<<<1, kPlanThreads, 0, st>>>(P, ws, t0, t1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_route_scatter(const Problem& P, const int* cu_seqlens, const int* sel,
+                                 const Workspace& ws, int t0, int t1, cudaStream_t st) {
+    const long long n = (long long)(t1 - t0) * P.hq;
+    route_rows_kernel<true><<<rows_grid(n), 256, 0, st>>>(cu_seqlens, sel, P, ws, t0, t1);
+    return cudaGetLastError();
+}
+
+}  // namespace moba

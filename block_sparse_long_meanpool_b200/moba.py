@@ -1,0 +1,259 @@
+"""Thin ctypes binding of libmoba.so (include/moba.h).
+
+Argument marshalling only: every step of the forward runs in the library's CUDA kernels.
+PyTorch provides device memory, the current stream and events.  There is no fallback: if
+the library is missing or the tensors are not on a CUDA device, the calls raise.
+"""
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoba.so")
+
+# Every symbol the C ABI exports (checked by the CPU test suite).
+EXPORTS = (
+    "moba_num_blocks_bound",
+    "moba_workspace_size",
+    "moba_meanpool",
+    "moba_gate_topk",
+    "moba_attn_fwd",
+    "moba_device_status",
+    "moba_status_string",
+    "moba_last_error",
+)
+
+# moba_status codes
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT = range(6)
+
+# moba_run_info event slots
+EV_BEGIN, EV_MEANS_DONE, EV_GATE_DONE, EV_WAVE0 = 0, 1, 2, 3
+
+
+class MobaParams(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int),
+        ("total_tokens", ctypes.c_int),
+        ("num_q_heads", ctypes.c_int),
+        ("num_kv_heads", ctypes.c_int),
+        ("head_dim", ctypes.c_int),
+        ("chunk_size", ctypes.c_int),
+        ("topk", ctypes.c_int),
+        ("softmax_scale", ctypes.c_float),
+        ("wave_tokens", ctypes.c_int),
+    ]
+
+
+class MobaRunInfo(ctypes.Structure):
+    _fields_ = [
+        ("events", ctypes.POINTER(ctypes.c_void_p)),
+        ("n_events", ctypes.c_int),
+        ("launches", ctypes.c_int),
+        ("waves", ctypes.c_int),
+    ]
+
+
+class MobaError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(message)
+        self.status = status
+
+
+_lib = None
+
+
+def load_library(path=LIB_PATH):
+    """Loads libmoba.so and declares its signatures.  Raises if it has not been built."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m block_sparse_long_meanpool_b200.build`")
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER(MobaParams)
+    vp = ctypes.c_void_p
+    lib.moba_num_blocks_bound.argtypes = [P]
+    lib.moba_num_blocks_bound.restype = ctypes.c_int
+    lib.moba_workspace_size.argtypes = [P]
+    lib.moba_workspace_size.restype = ctypes.c_size_t
+    lib.moba_meanpool.argtypes = [P, vp, vp, vp, vp]
+    lib.moba_meanpool.restype = ctypes.c_int
+    lib.moba_gate_topk.argtypes = [P, vp, vp, vp, vp, vp]
+    lib.moba_gate_topk.restype = ctypes.c_int
+    lib.moba_attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp,
+                                  ctypes.POINTER(MobaRunInfo), vp]
+    lib.moba_attn_fwd.restype = ctypes.c_int
+    lib.moba_device_status.argtypes = [P, vp, vp]
+    lib.moba_device_status.restype = ctypes.c_int
+    lib.moba_status_string.argtypes = [ctypes.c_int]
+    lib.moba_status_string.restype = ctypes.c_char_p
+    lib.moba_last_error.argtypes = []
+    lib.moba_last_error.restype = ctypes.c_char_p
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def _check(status):
+    if status != OK:
+        lib = load_library()
+        name = lib.moba_status_string(status).decode()
+        msg = lib.moba_last_error().decode()
+        raise MobaError(status, f"{name}: {msg}")
+
+
+def make_params(batch, total_tokens, num_q_heads, num_kv_heads, head_dim, chunk_size, topk,
+                softmax_scale=None, wave_tokens=0):
+    return MobaParams(int(batch), int(total_tokens), int(num_q_heads), int(num_kv_heads),
+                      int(head_dim), int(chunk_size), int(topk),
+                      float(softmax_scale) if softmax_scale else 0.0, int(wave_tokens))
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _require(cond, msg):
+    if not cond:
+        raise ValueError(msg)
+
+
+def _check_qkv(q, k, v=None):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t is None:
+            continue
+        _require(t.is_cuda, f"{name} must be a CUDA tensor")
+        _require(t.dtype == torch.bfloat16, f"{name} must be bf16")
+        _require(t.dim() == 3 and t.is_contiguous(), f"{name} must be contiguous [T, H, d]")
+
+
+def num_blocks(seqlens, chunk_size):
+    """Exact block count sum(ceil(L_i / chunk)) from host-side sequence lengths."""
+    return int(sum((int(n) + chunk_size - 1) // chunk_size for n in seqlens))
+
+
+def num_blocks_bound(params):
+    n = load_library().moba_num_blocks_bound(ctypes.byref(params))
+    if n < 0:
+        raise MobaError(ERR_INVALID_ARG, load_library().moba_last_error().decode())
+    return n
+
+
+def workspace_size(params):
+    n = load_library().moba_workspace_size(ctypes.byref(params))
+    if n == 0 and params.total_tokens > 0:
+        raise MobaError(ERR_INVALID_ARG, load_library().moba_last_error().decode())
+    return n
+
+
+def meanpool(k, cu_seqlens, chunk_size, num_blocks_out=None):
+    """Block means fp32 [NB, Hkv, d] of k bf16 [T, Hkv, d] (moba_meanpool)."""
+    _check_qkv(None, k)
+    batch = cu_seqlens.numel() - 1
+    T, hkv, d = k.shape
+    p = make_params(batch, T, hkv, hkv, d, chunk_size, 1)
+    nb = num_blocks_out if num_blocks_out is not None else max(load_library().moba_num_blocks_bound(ctypes.byref(p)), 0)
+    out = torch.empty((max(nb, 1), hkv, d), dtype=torch.float32, device=k.device)
+    _check(load_library().moba_meanpool(ctypes.byref(p), _ptr(k), _ptr(cu_seqlens), _ptr(out),
+                                        _stream(k.device)))
+    return out[:nb]
+
+
+def gate_topk(q, k_mean, cu_seqlens, chunk_size, topk, num_kv_heads=None):
+    """Selections int32 [Hq, T, topk] (moba_gate_topk)."""
+    _check_qkv(q, None)
+    _require(k_mean.dtype == torch.float32 and k_mean.is_contiguous(), "k_mean must be fp32")
+    batch = cu_seqlens.numel() - 1
+    T, hq, d = q.shape
+    hkv = num_kv_heads or k_mean.shape[1]
+    p = make_params(batch, T, hq, hkv, d, chunk_size, topk)
+    sel = torch.empty((hq, T, topk), dtype=torch.int32, device=q.device)
+    _check(load_library().moba_gate_topk(ctypes.byref(p), _ptr(q), _ptr(k_mean), _ptr(cu_seqlens),
+                                         _ptr(sel), _stream(q.device)))
+    return sel
+
+
+def choose_wave_tokens(T, hq, hkv, d, chunk_size, topk, batch, budget_bytes):
+    """Largest multiple of 128 query tokens per wave whose workspace fits in budget_bytes."""
+    lib = load_library()
+    full = make_params(batch, T, hq, hkv, d, chunk_size, topk, None, 0)
+    if lib.moba_workspace_size(ctypes.byref(full)) <= budget_bytes and T * hq * topk < 2 ** 31:
+        return 0
+    one = make_params(batch, T, hq, hkv, d, chunk_size, topk, None, 128)
+    base = lib.moba_workspace_size(ctypes.byref(one))
+    two = make_params(batch, T, hq, hkv, d, chunk_size, topk, None, 256)
+    per128 = max(lib.moba_workspace_size(ctypes.byref(two)) - base, 1)
+    n = max(1, int((budget_bytes - base) // per128) + 1)
+    n = min(n, (2 ** 31 - 1) // (hq * topk * 128))
+    w = 128 * max(n, 1)
+    return 0 if w >= T else w
+
+
+def attn_fwd(q, k, v, cu_seqlens, chunk_size, topk, softmax_scale=None, sel=None,
+             return_sel=False, wave_tokens=None, workspace=None, events=None,
+             workspace_budget=None, out=None, lse=None):
+    """MoBA causal prefill forward (moba_attn_fwd).
+
+    q bf16 [T, Hq, d], k/v bf16 [T, Hkv, d], cu_seqlens int32 [batch + 1] on the device.
+    sel: optional int32 [Hq, T, topk] selection to use instead of the gate.
+    Returns (out bf16 [T, Hq, d], lse fp32 [Hq, T]) and, with return_sel, the gate's
+    selection.  ``events`` may be a list of torch.cuda.Event recorded at the library's stage
+    boundaries; the call's moba_run_info is returned in ``attn_fwd.last_info``.
+    """
+    _check_qkv(q, k, v)
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    _require(k.shape == v.shape and k.shape[0] == T and k.shape[2] == d, "k/v shape mismatch")
+    _require(cu_seqlens.dtype == torch.int32 and cu_seqlens.is_cuda, "cu_seqlens int32 CUDA")
+    batch = cu_seqlens.numel() - 1
+    dev = q.device
+    if wave_tokens is None:
+        if workspace_budget is None:
+            free, _ = torch.cuda.mem_get_info(dev)
+            workspace_budget = min(int(free * 0.45), 48 << 30)
+        wave_tokens = choose_wave_tokens(T, hq, hkv, d, chunk_size, topk, batch, workspace_budget)
+    p = make_params(batch, T, hq, hkv, d, chunk_size, topk, softmax_scale, wave_tokens)
+    need = workspace_size(p)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    if out is None:
+        out = torch.empty((T, hq, d), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((hq, T), dtype=torch.float32, device=dev)
+    sel_out = None
+    if sel is not None:
+        _require(sel.dtype == torch.int32 and sel.is_contiguous() and tuple(sel.shape) == (hq, T, topk),
+                 "sel must be int32 [Hq, T, topk]")
+    elif return_sel:
+        sel_out = torch.empty((hq, T, topk), dtype=torch.int32, device=dev)
+    info = MobaRunInfo()
+    ev_arr = None
+    if events:
+        stream = torch.cuda.current_stream(dev)
+        for e in events:
+            if not e.cuda_event:
+                e.record(stream)
+        ev_arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+        info.events = ctypes.cast(ev_arr, ctypes.POINTER(ctypes.c_void_p))
+        info.n_events = len(events)
+    status = load_library().moba_attn_fwd(
+        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), _ptr(sel), _ptr(sel_out),
+        _ptr(workspace), ctypes.c_size_t(workspace.numel()), _ptr(out), _ptr(lse),
+        ctypes.byref(info), _stream(dev))
+    _check(status)
+    attn_fwd.last_info = {"launches": info.launches, "waves": info.waves,
+                          "wave_tokens": wave_tokens, "workspace_bytes": need}
+    if return_sel and sel is None:
+        return out, lse, sel_out
+    return out, lse
+
+
+attn_fwd.last_info = None

@@ -1,0 +1,154 @@
+/*
+ * moba.h - C ABI of the B200 MoBA (Mixture of Block Attention) causal prefill forward.
+ *
+ * The operation is the one defined on the page "《MoBA: Mixture of Block Attention for
+ * Long-Context LLMs》深度解读报告" (an analysis of the MoBA paper), sections 2.1-2.3 and 3.2:
+ *
+ *   1. every packed sequence is cut into blocks of `chunk_size` tokens (§2.1);
+ *   2. each block is summarised per KV head by the mean of its keys (§2.2);
+ *   3. each query row (token t, query head h) scores every block j of its sequence by
+ *      s_j = <q, mean_j> (§2.2);
+ *   4. blocks after the row's own block c are masked to -inf, block c is always taken
+ *      and the best `topk - 1` blocks j < c are routed (§2.3, hard top-k of §2.2);
+ *   5. the row attends, softmax-normalised, over the union of its selected blocks, with a
+ *      causal mask inside block c (§2.2-§2.3); the history blocks and the current block are
+ *      computed separately and merged by their log-sum-exp (§3.2).
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are packed varlen ("THD"): q is bf16 [T, Hq, d], k and v are bf16 [T, Hkv, d],
+ *     row-major, rows of all sequences back to back.  cu_seqlens is int32 [batch + 1],
+ *     cu_seqlens[0] = 0, non-decreasing, cu_seqlens[batch] = T.  The caller guarantees
+ *     cu_seqlens matches `total_tokens`; it is read on the device only.
+ *   - GQA: query head h reads KV head h / (Hq / Hkv).
+ *   - Blocks are numbered globally, sequence by sequence: the blocks of sequence i are
+ *     cu_blocks[i] .. cu_blocks[i+1]-1 with cu_blocks[i+1]-cu_blocks[i] = ceil(L_i / chunk).
+ *     A final partial block is allowed; its mean is over its valid tokens.
+ *   - Selections are int32 [Hq, T, topk]: block indices local to the row's sequence,
+ *     ascending, padded with -1.  `topk` counts the forced current block.
+ *   - All device pointers are owned by the caller, must be 16-byte aligned and stay valid
+ *     until the work on `stream` finishes.  The library allocates no device memory and keeps
+ *     no state between calls.  `stream` is a cudaStream_t (NULL = legacy default stream).
+ *   - Every call checks its arguments on the host and returns a status before launching
+ *     anything; on success all work is queued asynchronously on `stream`.  A launch failure
+ *     returns MOBA_ERR_CUDA.  moba_last_error() describes the most recent failure of the
+ *     calling host thread.
+ *   - GPU path limits: head_dim in {64, 128}; chunk_size a positive multiple of 128;
+ *     1 <= topk <= 32; Hq % Hkv == 0.  Other values return MOBA_ERR_UNSUPPORTED
+ *     (or MOBA_ERR_INVALID_ARG when they are meaningless, e.g. topk < 1).
+ */
+#ifndef MOBA_H_
+#define MOBA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOBA_OK = 0,
+    MOBA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, Hq % Hkv != 0, topk < 1 ... */
+    MOBA_ERR_UNSUPPORTED = 2,   /* valid but outside the GPU path limits above */
+    MOBA_ERR_WORKSPACE = 3,     /* workspace pointer NULL or smaller than moba_workspace_size */
+    MOBA_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+    MOBA_ERR_DEVICE_TIMEOUT = 5 /* a bounded device-side wait gave up (see moba_device_status) */
+} moba_status;
+
+typedef struct {
+    int batch;            /* number of packed sequences, >= 1 */
+    int total_tokens;     /* T = cu_seqlens[batch], >= 0 */
+    int num_q_heads;      /* Hq >= 1 */
+    int num_kv_heads;     /* Hkv >= 1, Hq % Hkv == 0 */
+    int head_dim;         /* d */
+    int chunk_size;       /* B, tokens per block */
+    int topk;             /* blocks per query row, counting its own block */
+    float softmax_scale;  /* logit scale of the attention softmax; <= 0 means 1/sqrt(d) */
+    int wave_tokens;      /* moba_attn_fwd only: query tokens per wave, 0 = all tokens in one
+                             wave; otherwise a positive multiple of 128.  Bounds the workspace
+                             (per-wave partial outputs), see moba_workspace_size. */
+} moba_params;
+
+/* Optional instrumentation for moba_attn_fwd.  All fields may be left zero. */
+typedef struct {
+    void** events;   /* in: cudaEvent_t array or NULL.  When non-NULL the call records
+                        events[MOBA_EV_*] (and, per wave w, events[MOBA_EV_WAVE0 + 4*w + i])
+                        on `stream` at the stage boundaries listed below, as long as the
+                        index is < n_events. */
+    int n_events;
+    int launches;    /* out: number of kernel launches the call queued */
+    int waves;       /* out: number of query waves */
+} moba_run_info;
+
+enum {
+    MOBA_EV_BEGIN = 0,      /* before the first launch */
+    MOBA_EV_MEANS_DONE = 1, /* after the mean-pool kernel */
+    MOBA_EV_GATE_DONE = 2,  /* after the gate kernel (same point as 1 when sel_in is given) */
+    MOBA_EV_WAVE0 = 3       /* per wave w: +4w route start, +4w+1 attention start,
+                               +4w+2 attention end, +4w+3 merge end */
+};
+
+/* Upper bound of the total number of blocks, ceil(T / B) + batch - 1 (0 when T = 0).
+ * Size k_mean buffers with it when the exact count is not known on the host.
+ * Returns -1 when params are invalid. */
+int moba_num_blocks_bound(const moba_params* p);
+
+/* Bytes of device workspace moba_attn_fwd needs for these params (wave size included).
+ * Returns 0 when params are invalid. */
+size_t moba_workspace_size(const moba_params* p);
+
+/* Step 2 (analysis §2.2): k_mean[b, g, :] = mean over the valid tokens of block b of
+ * k[t, g, :], fp32 accumulation, fp32 out.
+ *   k        bf16 [T, Hkv, d] device
+ *   cu_seqlens int32 [batch + 1] device
+ *   k_mean   fp32 [NB, Hkv, d] device, NB >= the true block count (moba_num_blocks_bound
+ *            is always enough); rows past the true count are left untouched.
+ * Uses no workspace. */
+moba_status moba_meanpool(const moba_params* p, const void* k, const int* cu_seqlens,
+                          float* k_mean, void* stream);
+
+/* Steps 3-4 (analysis §2.2-§2.3): per query row, gate scores against the means of the past
+ * blocks of its sequence (fp32), future blocks excluded, the own block forced, the best
+ * topk-1 past blocks kept (ties to the lower block index).
+ *   q       bf16 [T, Hq, d] device
+ *   k_mean  fp32 [NB, Hkv, d] device, as written by moba_meanpool
+ *   sel     int32 [Hq, T, topk] device, written in full (ascending, -1 padded).
+ * Uses no workspace. */
+moba_status moba_gate_topk(const moba_params* p, const void* q, const float* k_mean,
+                           const int* cu_seqlens, int* sel, void* stream);
+
+/* The whole forward (steps 1-5): mean-pool, gate (unless sel_in is given), routing of rows
+ * to (KV head, block) lists, block attention on the tensor cores, log-sum-exp merge.
+ *   q, k, v     bf16 device, see conventions
+ *   sel_in      int32 [Hq, T, topk] device or NULL.  NULL: the gate runs.  Otherwise the
+ *               selection is taken from it (e.g. the oracle's): per row, entries in [0, c)
+ *               are routed past blocks (the first topk-1 such entries, in row order), the
+ *               own block c is always attended whether listed or not, anything else is
+ *               ignored.
+ *   sel_out     int32 [Hq, T, topk] device or NULL: receives the gate's selection (ignored
+ *               when sel_in is given).
+ *   workspace   device, >= moba_workspace_size(p) bytes, 256-byte aligned
+ *   out         bf16 [T, Hq, d] device (fp32 merge rounded to nearest even)
+ *   lse         fp32 [Hq, T] device: natural-log log-sum-exp of the scaled logits
+ *   info        optional instrumentation, may be NULL
+ * Workspace contents are undefined after the call. */
+moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, const void* v,
+                          const int* cu_seqlens, const int* sel_in, int* sel_out,
+                          void* workspace, size_t workspace_bytes, void* out, float* lse,
+                          moba_run_info* info, void* stream);
+
+/* Reads (synchronously, on `stream`) the device status word a previous moba_attn_fwd left in
+ * `workspace`: MOBA_OK, or MOBA_ERR_DEVICE_TIMEOUT when a bounded device-side wait gave up.
+ * Waits for the stream. */
+moba_status moba_device_status(const moba_params* p, const void* workspace, void* stream);
+
+/* Static description of a status code. */
+const char* moba_status_string(moba_status s);
+
+/* Description of the last failure on the calling host thread ("" if none). */
+const char* moba_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOBA_H_ */

@@ -165,7 +165,6 @@ def select_blocks_rows(q, means, cu_seqlens, chunk, topk, rows):
     sampled rows of inputs too large to select in full.  Returns
     ``[len(rows), topk]`` int64.
     """
-    q = np.asarray(q)
     means = np.asarray(means)
     Hq, Hkv = q.shape[1], means.shape[1]
     group = Hq // Hkv

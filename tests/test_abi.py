@@ -1,0 +1,139 @@
+"""Host-only checks of the C ABI: the library loads, exports every declared symbol, and
+rejects bad arguments with the documented status before touching the GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from block_sparse_long_meanpool_b200 import build, moba
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moba.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return moba.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moba_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(moba.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def params(**kw):
+    base = dict(batch=1, total_tokens=2048, num_q_heads=4, num_kv_heads=4, head_dim=64,
+                chunk_size=256, topk=3, softmax_scale=None, wave_tokens=0)
+    base.update(kw)
+    return moba.make_params(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(batch=0), moba.ERR_INVALID_ARG),
+    (dict(total_tokens=-1), moba.ERR_INVALID_ARG),
+    (dict(num_kv_heads=3), moba.ERR_INVALID_ARG),
+    (dict(topk=0), moba.ERR_INVALID_ARG),
+    (dict(chunk_size=0), moba.ERR_INVALID_ARG),
+    (dict(wave_tokens=-128), moba.ERR_INVALID_ARG),
+    (dict(head_dim=96), moba.ERR_UNSUPPORTED),
+    (dict(chunk_size=100), moba.ERR_UNSUPPORTED),
+    (dict(topk=33), moba.ERR_UNSUPPORTED),
+    (dict(wave_tokens=100), moba.ERR_UNSUPPORTED),
+])
+def test_invalid_params_are_rejected(lib, kw, status):
+    p = params(**kw)
+    assert lib.moba_workspace_size(ctypes.byref(p)) == 0
+    assert lib.moba_num_blocks_bound(ctypes.byref(p)) == -1
+    rc = lib.moba_attn_fwd(ctypes.byref(p), None, None, None, None, None, None, None, 0, None,
+                           None, None, None)
+    assert rc == status, lib.moba_last_error()
+    assert lib.moba_last_error()
+    assert lib.moba_meanpool(ctypes.byref(p), None, None, None, None) == status
+    assert lib.moba_gate_topk(ctypes.byref(p), None, None, None, None, None) == status
+
+
+def test_null_params_and_null_pointers(lib):
+    assert lib.moba_attn_fwd(None, None, None, None, None, None, None, None, 0, None, None,
+                             None, None) == moba.ERR_INVALID_ARG
+    p = params()
+    assert lib.moba_attn_fwd(ctypes.byref(p), None, None, None, None, None, None, None, 0, None,
+                             None, None, None) == moba.ERR_INVALID_ARG
+    assert b"NULL" in lib.moba_last_error()
+    assert lib.moba_device_status(ctypes.byref(p), None, None) == moba.ERR_WORKSPACE
+
+
+def test_empty_input_is_a_no_op(lib):
+    p = params(total_tokens=0)
+    assert lib.moba_workspace_size(ctypes.byref(p)) > 0
+    assert lib.moba_num_blocks_bound(ctypes.byref(p)) == 0
+    info = moba.MobaRunInfo()
+    rc = lib.moba_attn_fwd(ctypes.byref(p), None, None, None, None, None, None, None, 0, None,
+                           None, ctypes.byref(info), None)
+    assert rc == moba.OK and info.launches == 0
+    assert lib.moba_meanpool(ctypes.byref(p), None, None, None, None) == moba.OK
+
+
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="hands fake device addresses to the library: host-only check")
+def test_workspace_and_alignment_checks_precede_any_launch(lib):
+    p = params()
+    fake = ctypes.c_void_p(1 << 20)
+    need = lib.moba_workspace_size(ctypes.byref(p))
+    rc = lib.moba_attn_fwd(ctypes.byref(p), fake, fake, fake, fake, None, None, fake, need - 1,
+                           fake, fake, None, None)
+    assert rc == moba.ERR_WORKSPACE
+    assert str(need).encode() in lib.moba_last_error()
+    rc = lib.moba_attn_fwd(ctypes.byref(p), fake, fake, fake, fake, None, None, None, need,
+                           fake, fake, None, None)
+    assert rc == moba.ERR_WORKSPACE
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    rc = lib.moba_attn_fwd(ctypes.byref(p), odd, fake, fake, fake, None, None, fake, need,
+                           fake, fake, None, None)
+    assert rc == moba.ERR_INVALID_ARG
+    rc = lib.moba_attn_fwd(ctypes.byref(p), fake, fake, fake, fake, None, None,
+                           ctypes.c_void_p((1 << 20) + 128), need, fake, fake, None, None)
+    assert rc == moba.ERR_WORKSPACE
+    # 32-bit partial-output indices: one wave of 1M tokens x 64 heads x top-32 is refused
+    big = params(total_tokens=1 << 20, num_q_heads=64, num_kv_heads=8, head_dim=128,
+                 chunk_size=4096, topk=32, wave_tokens=0)
+    need_big = lib.moba_workspace_size(ctypes.byref(big))
+    assert need_big > 0
+    rc = lib.moba_attn_fwd(ctypes.byref(big), fake, fake, fake, fake, None, None, fake,
+                           need_big, fake, fake, None, None)
+    assert rc == moba.ERR_UNSUPPORTED
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert lib.moba_status_string(code).startswith(b"MOBA_")
+    assert lib.moba_status_string(99) == b"MOBA_ERR_UNKNOWN"
+
+
+def test_workspace_grows_with_the_wave_and_block_bound(lib):
+    sizes = [lib.moba_workspace_size(ctypes.byref(params(total_tokens=8192, wave_tokens=w)))
+             for w in (128, 1024, 4096, 0)]
+    assert sizes == sorted(sizes) and sizes[0] < sizes[-1]
+    p = params(batch=3, total_tokens=1000, chunk_size=256)
+    assert lib.moba_num_blocks_bound(ctypes.byref(p)) == 4 + 2
+
+
+def test_wave_choice_respects_budget(lib):
+    w = moba.choose_wave_tokens(1 << 20, 32, 8, 128, 4096, 12, 1, 8 << 30)
+    assert w > 0 and w % 128 == 0
+    p = moba.make_params(1, 1 << 20, 32, 8, 128, 4096, 12, None, w)
+    assert lib.moba_workspace_size(ctypes.byref(p)) <= 8 << 30
+    assert moba.choose_wave_tokens(2048, 4, 4, 64, 256, 3, 1, 1 << 30) == 0
