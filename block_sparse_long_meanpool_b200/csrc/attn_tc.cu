@@ -1,0 +1,682 @@
+// Step 5 of the forward on the 5th-generation tensor cores (tcgen05 + TMEM + TMA), sm_100a.
+//
+// The analysis page of the MoBA paper (§3.2): history blocks are attended without a causal
+// mask (rule 1 of §2.3 already excluded every future block), the own block with a causal
+// mask, and the partial softmax results are merged afterwards by their log-sum-exp.
+//
+// Work items (from the routing pass) are 128 query rows against one KV range: a history tile
+// is up to 128 routed rows (any query heads of one KV head) against one whole block, a
+// current-block tile is 128 consecutive tokens of one query head against the causal prefix
+// of their block.  A persistent CTA per SM takes items from an atomic cursor.
+//
+// Warp roles (224 threads):
+//   warps 0-3  softmax + epilogue, thread r owns query row r (TMEM lane r)
+//   warp 4     K/V producer: TMA (SWIZZLE_128B, no multicast) into a 4-stage ring
+//   warp 5     item fetch + Q gather: routed rows by cp.async into a swizzled K-major tile
+//   warp 6     TMEM owner and single-thread MMA issuer
+// Per 128-key chunk n: S_n = Q K_n^T (SS MMA, fp32 in TMEM, double-buffered), softmax in
+// registers after tcgen05.ld, P_n (bf16) written back over S_n with tcgen05.st, then
+// O += P_n V_n (TS MMA: A from TMEM, V from shared memory, MN-major).  The MMA warp issues
+// QK_{n+1} before PV_n so the tensor core works while the softmax of chunk n runs.  The
+// running max is only raised (and O rescaled) when it grows by more than 2^8, so O is
+// rarely touched.  P has its own TMEM columns (never aliasing S), so QK^T of chunk n+2 can
+// run while PV of chunk n still reads P_n.
+//
+// Every mbarrier wait is bounded: on expiry the kernel records MOBA_ERR_DEVICE_TIMEOUT in
+// the workspace status word, all roles leave their loops, in-flight copies and MMAs are
+// drained (bounded), TMEM is freed and the CTA returns.
+#include <cuda.h>
+
+#include <climits>
+
+#include "moba_internal.cuh"
+
+namespace moba {
+
+namespace {
+
+constexpr int kBN = 128;       // keys per chunk
+constexpr int kStages = 4;     // K/V ring depth
+constexpr int kThreads = 224;  // 7 warps
+constexpr int kWarpKV = 4, kWarpQ = 5, kWarpMMA = 6;
+constexpr uint32_t kSpinLimit = 1u << 22;  // try_wait polls before a wait is declared stuck
+constexpr int kTimeoutStatus = 5;          // MOBA_ERR_DEVICE_TIMEOUT
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled when max grows > 2^8
+
+struct ItemSlot {
+    int kind;  // -1 = no more work
+    int g, key_start, key_end, nchunks;
+    int pidx[kTileM];
+    int tlim[kTileM];
+};
+
+template <int D>
+struct SmemLayout {
+    static constexpr int kTileBytes = kTileM * D * 2;  // 128 rows of bf16 (Q tile, K or V chunk)
+    static constexpr int kQ = 0;                       // 2 Q buffers
+    static constexpr int kKV = 2 * kTileBytes;         // kStages K/V buffers
+    static constexpr int kSlots = kKV + kStages * kTileBytes;
+    static constexpr int kBars = kSlots + 2 * (int)sizeof(ItemSlot);
+    static constexpr int kNumBars = 2 + 2 + 2 + kStages + kStages + 2 + 2 + 1 + 2 + 1;
+    static constexpr int kMisc = kBars + kNumBars * 8;
+    static constexpr int kBytes = kMisc + 16 + 1024;  // + slack for 1024-byte alignment
+};
+
+// ---------------------------------------------------------------------------------------
+// PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, int count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint32_t bar, int c0,
+                                            int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+    const int sz = valid ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(sz)
+                 : "memory");
+}
+
+// Shared-memory matrix descriptor, SWIZZLE_128B, sm_100 version bits.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// Instruction descriptor kind::f16: bf16 x bf16 -> fp32, M = 128.
+__host__ __device__ constexpr uint32_t idesc_bf16(int n, bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+           ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                       uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+        : "memory");
+}
+
+// 32 consecutive TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+        "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31]));
+}
+__device__ __forceinline__ void tmem_st_wait() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Bounded wait, called by all 32 lanes of a warp; the result is warp-uniform.  Returns false
+// when the CTA is aborting (this wait expired or another role's did).
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         int* status) {
+    bool ok = false;
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        if (mbar_try_wait(bar, parity)) {
+            ok = true;
+            break;
+        }
+        if ((i & 63u) == 63u && *abort_flag) break;
+    }
+    if (!ok && !*abort_flag) {
+        *abort_flag = 1;
+        atomicExch(status, kTimeoutStatus);
+    }
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Bounded wait that ignores the abort flag (used to drain in-flight work on the way out).
+__device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kSpinLimit; ++i)
+        if (mbar_try_wait(bar, parity)) return;
+}
+
+// ---------------------------------------------------------------------------------------
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+               const __nv_bfloat16* __restrict__ q, Problem P, Workspace ws, int t0, int t1) {
+    using L = SmemLayout<D>;
+    constexpr int kHalves = D / 64;          // 128-byte swizzle atoms along d
+    constexpr int kHalfBytes = kTileM * 128;  // one [128 rows x 64 bf16] swizzled half
+    constexpr uint32_t kChunkBytes = kTileM * D * 2;
+    constexpr int kKSteps = D / 16;           // QK^T k-steps (16 bf16 each)
+    constexpr uint32_t kIdescQK = idesc_bf16(kBN, false);
+    constexpr uint32_t kIdescPV = idesc_bf16(D, true);
+    // TMEM columns: S0, S1 (fp32, 128 each), P0, P1 (bf16 pairs, 64 each), O (D)
+    constexpr uint32_t kColS0 = 0, kColP0 = 2 * kBN, kColO = 3 * kBN;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    ItemSlot* slots = reinterpret_cast<ItemSlot*>(smem + L::kSlots);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+
+    const uint32_t sm_base = smem_u32(smem);
+    const uint32_t bar0 = smem_u32(bars);
+    // barrier indices
+    auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+    const int B_INFO = 0, B_QFULL = 2, B_ITEM_EMPTY = 4, B_KV_FULL = 6, B_KV_EMPTY = 6 + kStages,
+              B_S_FULL = 6 + 2 * kStages, B_P_FULL = B_S_FULL + 2, B_PV_DONE = B_P_FULL + 2,
+              B_O_EMPTY = B_PV_DONE + 2, B_FINAL = B_O_EMPTY + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int* status = &ws.hdr->status;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(BAR(B_INFO + i), 32);
+            mbar_init(BAR(B_QFULL + i), 32);
+            mbar_init(BAR(B_ITEM_EMPTY + i), 128);
+            mbar_init(BAR(B_S_FULL + i), 1);
+            mbar_init(BAR(B_P_FULL + i), 128);
+        }
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(BAR(B_KV_FULL + i), 1);
+            mbar_init(BAR(B_KV_EMPTY + i), 1);
+        }
+        mbar_init(BAR(B_PV_DONE), 1);
+        mbar_init(BAR(B_PV_DONE + 1), 1);
+        mbar_init(BAR(B_O_EMPTY), 128);
+        mbar_init(BAR(B_FINAL), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == kWarpMMA) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                         smem_u32(tmem_slot)));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == kWarpQ) {
+        // ---------------- item fetch + Q gather ----------------
+        const int n_items = ws.hdr->n_items;
+        constexpr int CK = D / 8;  // 16-byte chunks per row
+        for (int it = 0;; ++it) {
+            const int s = it & 1;
+            const uint32_t ph = (uint32_t)(it >> 1) & 1u;
+            if (it >= 2 && !wait_bar(BAR(B_ITEM_EMPTY + s), ph ^ 1u, abort_flag, status)) break;
+            int idx = 0;
+            if (lane == 0) idx = (int)atomicAdd(&ws.hdr->work_counter, 1u);
+            idx = __shfl_sync(0xffffffffu, idx, 0);
+            ItemSlot& sl = slots[s];
+            if (idx >= n_items) {
+                if (lane == 0) sl.kind = -1;
+                __syncwarp();
+                mbar_arrive(BAR(B_INFO + s));
+                break;
+            }
+            const WorkItem w = ws.items[idx];
+            int g, key_start, key_end;
+            long long qoff[kTileM / 32];
+            if (w.kind == 0) {
+                g = w.a / P.nb_cap;
+                const int b = w.a - g * P.nb_cap;
+                key_start = ws.blk_start[b];
+                key_end = key_start + ws.blk_len[b];
+#pragma unroll
+                for (int i = 0; i < kTileM / 32; ++i) {
+                    const int r = lane + 32 * i;
+                    int pidx = -1;
+                    long long off = -1;
+                    if (r < w.c) {
+                        pidx = ws.entries[w.b + r];
+                        const int rid = pidx / P.topk;
+                        const int t = t0 + rid / P.hq;
+                        const int h = rid - (rid / P.hq) * P.hq;
+                        off = ((long long)t * P.hq + h) * D;
+                    }
+                    sl.pidx[r] = pidx;
+                    sl.tlim[r] = INT_MAX;
+                    qoff[i] = off;
+                }
+            } else {
+                const int b = w.a, h = w.b, qt = w.c;
+                g = h / P.group;
+                key_start = ws.blk_start[b];
+                const int len = ws.blk_len[b];
+                key_end = key_start + min((qt + 1) * kTileM, len);
+#pragma unroll
+                for (int i = 0; i < kTileM / 32; ++i) {
+                    const int r = lane + 32 * i;
+                    const int rr = qt * kTileM + r;
+                    const int t = key_start + rr;
+                    const bool ok = rr < len && t >= t0 && t < t1;
+                    sl.pidx[r] = ok ? ((t - t0) * P.hq + h) * P.topk : -1;
+                    sl.tlim[r] = ok ? t : INT_MAX;
+                    qoff[i] = ok ? ((long long)t * P.hq + h) * D : -1;
+                }
+            }
+            if (lane == 0) {
+                sl.kind = w.kind;
+                sl.g = g;
+                sl.key_start = key_start;
+                sl.key_end = key_end;
+                sl.nchunks = (key_end - key_start + kBN - 1) / kBN;
+            }
+            __syncwarp();
+            mbar_arrive(BAR(B_INFO + s));
+            // gather the 128 rows: lane handles rows lane + 32 i, all 16-byte chunks
+            const uint32_t qbuf = sm_base + L::kQ + (uint32_t)s * L::kTileBytes;
+#pragma unroll
+            for (int i = 0; i < kTileM / 32; ++i) {
+                const int r = lane + 32 * i;
+                const long long off = qoff[i];
+                const __nv_bfloat16* src = off >= 0 ? q + off : q;
+#pragma unroll
+                for (int c = 0; c < CK; ++c) {
+                    const uint32_t dst = qbuf + (uint32_t)(c >> 3) * kHalfBytes + (uint32_t)r * 128u +
+                                         (uint32_t)(((c & 7) ^ (r & 7)) << 4);
+                    cp_async16(dst, src + (off >= 0 ? c * 8 : 0), off >= 0);
+                }
+            }
+            asm volatile("cp.async.commit_group;" ::: "memory");
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+            fence_proxy_async();
+            mbar_arrive(BAR(B_QFULL + s));
+        }
+    } else if (warp == kWarpKV) {
+        // ---------------- K/V producer (TMA) ----------------
+        uint32_t c = 0;  // ring position
+        for (int it = 0;; ++it) {
+            const int s = it & 1;
+            if (!wait_bar(BAR(B_INFO + s), (uint32_t)(it >> 1) & 1u, abort_flag, status)) break;
+            const ItemSlot& sl = slots[s];
+            if (sl.kind < 0) break;
+            const int g = sl.g, key_start = sl.key_start, N = sl.nchunks;
+            // consumption order of the MMA warp: K0, then per n: K_{n+1} (if any), V_n
+            auto load = [&](bool is_v, int chunk) -> bool {
+                const uint32_t st = c % kStages;
+                if (c >= kStages &&
+                    !wait_bar(BAR(B_KV_EMPTY + st), ((c / kStages) - 1u) & 1u, abort_flag, status))
+                    return false;
+                if (lane == 0) {
+                    const uint32_t dst = sm_base + L::kKV + st * L::kTileBytes;
+                    mbar_arrive_tx(BAR(B_KV_FULL + st), kChunkBytes);
+                    const void* tm = is_v ? (const void*)&tmap_v : (const void*)&tmap_k;
+#pragma unroll
+                    for (int hh = 0; hh < kHalves; ++hh)
+                        tma_load_3d(dst + hh * kHalfBytes, tm, BAR(B_KV_FULL + st), hh * 64, g,
+                                    key_start + chunk * kBN);
+                }
+                __syncwarp();
+                ++c;
+                return true;
+            };
+            bool ok = load(false, 0);
+            for (int n = 0; n < N && ok; ++n) {
+                if (n + 1 < N) ok = load(false, n + 1);
+                if (ok) ok = load(true, n);
+            }
+            if (!ok) break;
+        }
+        // drain: every issued load must land before the CTA exits
+        const uint32_t issued = c;
+        for (uint32_t k = (issued > kStages ? issued - kStages : 0); k < issued; ++k)
+            drain_bar(BAR(B_KV_FULL + k % kStages), (k / kStages) & 1u);
+    } else if (warp == kWarpMMA) {
+        // ---------------- MMA issuer ----------------
+        uint32_t c = 0;     // ring position
+        uint32_t glob = 0;  // global chunk counter (S buffers, pv_done phases)
+        bool ok = true;
+        for (int it = 0; ok; ++it) {
+            const int s = it & 1;
+            const uint32_t ph = (uint32_t)(it >> 1) & 1u;
+            if (!wait_bar(BAR(B_INFO + s), ph, abort_flag, status)) break;
+            const ItemSlot& sl = slots[s];
+            if (sl.kind < 0) break;
+            const int N = sl.nchunks;
+            if (!wait_bar(BAR(B_QFULL + s), ph, abort_flag, status)) break;
+            tc_fence_after();
+            const uint32_t qbuf = sm_base + L::kQ + (uint32_t)s * L::kTileBytes;
+            const uint32_t o_tmem = tmem + kColO;
+            auto issue_qk = [&](uint32_t chunk_g) -> bool {
+                const uint32_t st = c % kStages;
+                if (!wait_bar(BAR(B_KV_FULL + st), (c / kStages) & 1u, abort_flag, status))
+                    return false;
+                tc_fence_after();
+                const uint32_t kbuf = sm_base + L::kKV + st * L::kTileBytes;
+                const uint32_t s_tmem = tmem + kColS0 + (chunk_g & 1u) * kBN;
+                if (lane == 0) {
+#pragma unroll
+                    for (int kk = 0; kk < kKSteps; ++kk) {
+                        const uint32_t koff = (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32u;
+                        mma_ss(s_tmem, smem_desc(qbuf + koff, 16, 1024), smem_desc(kbuf + koff, 16, 1024),
+                               kIdescQK, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(BAR(B_KV_EMPTY + st));
+                    mma_commit(BAR(B_S_FULL + (chunk_g & 1u)));
+                }
+                __syncwarp();
+                ++c;
+                return true;
+            };
+            if (!issue_qk(glob)) break;
+            for (int n = 0; n < N; ++n) {
+                if (n + 1 < N && !issue_qk(glob + n + 1)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t cg = glob + (uint32_t)n;
+                // O is single-buffered: the previous item's epilogue must have read it
+                if (n == 0 && it >= 1 &&
+                    !wait_bar(BAR(B_O_EMPTY), (uint32_t)(it - 1) & 1u, abort_flag, status)) {
+                    ok = false;
+                    break;
+                }
+                if (!wait_bar(BAR(B_P_FULL + (cg & 1u)), (cg >> 1) & 1u, abort_flag, status)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t st = c % kStages;
+                if (!wait_bar(BAR(B_KV_FULL + st), (c / kStages) & 1u, abort_flag, status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t vbuf = sm_base + L::kKV + st * L::kTileBytes;
+                const uint32_t p_tmem = tmem + kColP0 + (cg & 1u) * (kBN / 2);
+                if (lane == 0) {
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk) {
+                        // A = P: 16 keys = 8 packed columns; B = V rows kk*16.., MN-major
+                        mma_ts(o_tmem, p_tmem + (uint32_t)kk * 8u,
+                               smem_desc(vbuf + (uint32_t)kk * 2048u, (uint32_t)kHalfBytes, 1024),
+                               kIdescPV, (n > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(BAR(B_KV_EMPTY + st));
+                    mma_commit(BAR(B_PV_DONE + (cg & 1u)));
+                }
+                __syncwarp();
+                ++c;
+            }
+            glob += (uint32_t)N;
+        }
+        // drain the tensor pipe before TMEM is freed
+        if (lane == 0) mma_commit(BAR(B_FINAL));
+        __syncwarp();
+        drain_bar(BAR(B_FINAL), 0);
+    } else {
+        // ---------------- softmax + epilogue (warps 0-3) ----------------
+        const int row = warp * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        uint32_t glob = 0;
+        const float ln2 = 0.69314718055994531f;
+        bool ok = true;
+        for (int it = 0; ok; ++it) {
+            const int s = it & 1;
+            if (!wait_bar(BAR(B_INFO + s), (uint32_t)(it >> 1) & 1u, abort_flag, status)) break;
+            const ItemSlot& sl = slots[s];
+            if (sl.kind < 0) break;
+            const int N = sl.nchunks, key_start = sl.key_start, key_end = sl.key_end;
+            const int pidx = sl.pidx[row];
+            const int tl = sl.tlim[row];
+            const uint32_t o_tmem = tmem + lane_off + kColO;
+            float m = -INFINITY, l = 0.f;
+            for (int n = 0; n < N; ++n) {
+                const uint32_t cg = glob + (uint32_t)n;
+                const uint32_t b = cg & 1u;
+                if (!wait_bar(BAR(B_S_FULL + b), (cg >> 1) & 1u, abort_flag, status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t s_tmem = tmem + lane_off + kColS0 + b * kBN;
+                const uint32_t p_tmem = tmem + lane_off + kColP0 + b * (kBN / 2);
+                float x[kBN];
+#pragma unroll
+                for (int j = 0; j < kBN / 32; ++j) {
+                    float v[32];
+                    tmem_ld32(s_tmem + 32u * j, v);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) x[32 * j + e] = v[e];
+                }
+                tmem_ld_wait();
+                const int key0 = key_start + n * kBN;
+                const int lim = min(key_end - 1, tl) - key0;  // last valid key offset
+                float mloc = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < kBN; ++j) {
+                    const float y = (j <= lim) ? x[j] * P.scale_log2 : -INFINITY;
+                    x[j] = y;
+                    mloc = fmaxf(mloc, y);
+                }
+                if (n == 0) {
+                    m = mloc;
+                } else {
+                    const bool need = mloc > m + kRescaleThreshold;
+                    if (__any_sync(0xffffffffu, need)) {
+                        // O must hold every earlier PV before it is rescaled
+                        const uint32_t pg = cg - 1u;
+                        if (!wait_bar(BAR(B_PV_DONE + (pg & 1u)), (pg >> 1) & 1u, abort_flag, status)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const float mn = fmaxf(m, mloc);
+                        const float alpha = exp2f(m - mn);
+#pragma unroll
+                        for (int j = 0; j < D / 32; ++j) {
+                            float v[32];
+                            tmem_ld32(o_tmem + 32u * j, v);
+                            tmem_ld_wait();
+                            uint32_t w[32];
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(v[e] * alpha);
+                            tmem_st32(o_tmem + 32u * j, w);
+                        }
+                        tmem_st_wait();
+                        l *= alpha;
+                        m = mn;
+                    }
+                }
+                float rs = 0.f;
+#pragma unroll
+                for (int j = 0; j < kBN; ++j) {
+                    const float p = exp2f(x[j] - m);
+                    x[j] = p;
+                    rs += p;
+                }
+                l += rs;
+#pragma unroll
+                for (int j = 0; j < kBN / 64; ++j) {
+                    uint32_t w[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) w[e] = pack_bf16(x[64 * j + 2 * e], x[64 * j + 2 * e + 1]);
+                    tmem_st32(p_tmem + 32u * j, w);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(BAR(B_P_FULL + b));
+            }
+            if (!ok) break;
+            // epilogue: O of the last chunk, normalise, write the partial (o, lse)
+            const uint32_t lastg = glob + (uint32_t)N - 1u;
+            if (!wait_bar(BAR(B_PV_DONE + (lastg & 1u)), (lastg >> 1) & 1u, abort_flag, status)) break;
+            tc_fence_after();
+            const float inv = 1.f / l;
+            float* dst = ws.part_o + (size_t)(pidx < 0 ? 0 : pidx) * D;
+#pragma unroll
+            for (int j = 0; j < D / 32; ++j) {
+                float v[32];
+                tmem_ld32(o_tmem + 32u * j, v);
+                tmem_ld_wait();
+                if (pidx >= 0) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4*>(dst + 32 * j + e) =
+                            make_float4(v[e] * inv, v[e + 1] * inv, v[e + 2] * inv, v[e + 3] * inv);
+                }
+            }
+            if (pidx >= 0) ws.part_lse[pidx] = m * ln2 + logf(l);
+            tc_fence_before();
+            mbar_arrive(BAR(B_O_EMPTY));
+            mbar_arrive(BAR(B_ITEM_EMPTY + s));
+            glob += (uint32_t)N;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kWarpMMA) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Host side: tensor maps through the driver entry point (no libcuda link dependency)
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// [T, Hkv, d] bf16 as a 3-D tensor (d, Hkv, T); box (64, 1, 128) with 128-byte swizzle.
+cudaError_t make_kv_map(CUtensorMap* m, const void* base, const Problem& P) {
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    cuuint64_t dims[3] = {(cuuint64_t)P.d, (cuuint64_t)P.hkv, (cuuint64_t)P.T};
+    cuuint64_t strides[2] = {(cuuint64_t)P.d * 2, (cuuint64_t)P.hkv * P.d * 2};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)kTileM};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int D>
+cudaError_t launch_tc_d(const Problem& P, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                        const __nv_bfloat16* v, const Workspace& ws, int t0, int t1, int num_sms,
+                        cudaStream_t st) {
+    CUtensorMap mk, mv;
+    cudaError_t e = make_kv_map(&mk, k, P);
+    if (e != cudaSuccess) return e;
+    e = make_kv_map(&mv, v, P);
+    if (e != cudaSuccess) return e;
+    const int smem = SmemLayout<D>::kBytes;
+    e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attn_tc_kernel<D><<<num_sms, kThreads, smem, st>>>(mk, mv, q, P, ws, t0, t1);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const Problem& P, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                             const __nv_bfloat16* v, const Workspace& ws, int t0, int t1,
+                             int num_sms, cudaStream_t st) {
+    if (P.d == 64) return launch_tc_d<64>(P, q, k, v, ws, t0, t1, num_sms, st);
+    return launch_tc_d<128>(P, q, k, v, ws, t0, t1, num_sms, st);
+}
+
+}  // namespace moba
