@@ -153,6 +153,11 @@ moba_status check_ranges(const moba_params& p, const Layout& L) {
 
 }  // namespace
 
+namespace moba {
+// Lets other translation units of the library report a failure through moba_last_error().
+void set_error_message(const char* msg) { g_last_error = msg; }
+}  // namespace moba
+
 extern "C" {
 
 int moba_num_blocks_bound(const moba_params* p) {

@@ -21,6 +21,7 @@ EXPORTS = (
     "moba_meanpool",
     "moba_gate_topk",
     "moba_attn_fwd",
+    "moba_attn_fwd_noalloc",
     "moba_device_status",
     "moba_status_string",
     "moba_last_error",
@@ -87,6 +88,8 @@ def load_library(path=LIB_PATH):
     lib.moba_attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp,
                                   ctypes.POINTER(MobaRunInfo), vp]
     lib.moba_attn_fwd.restype = ctypes.c_int
+    lib.moba_attn_fwd_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
+    lib.moba_attn_fwd_noalloc.restype = ctypes.c_int
     lib.moba_device_status.argtypes = [P, vp, vp]
     lib.moba_device_status.restype = ctypes.c_int
     lib.moba_status_string.argtypes = [ctypes.c_int]

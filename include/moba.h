@@ -27,7 +27,9 @@
  *     ascending, padded with -1.  `topk` counts the forced current block.
  *   - All device pointers are owned by the caller, must be 16-byte aligned and stay valid
  *     until the work on `stream` finishes.  The library allocates no device memory and keeps
- *     no state between calls.  `stream` is a cudaStream_t (NULL = legacy default stream).
+ *     no state between calls, apart from the static scratch array behind
+ *     moba_attn_fwd_noalloc (see below).  `stream` is a cudaStream_t (NULL = legacy default
+ *     stream).
  *   - Every call checks its arguments on the host and returns a status before launching
  *     anything; on success all work is queued asynchronously on `stream`.  A launch failure
  *     returns MOBA_ERR_CUDA.  moba_last_error() describes the most recent failure of the
@@ -140,6 +142,32 @@ moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, co
  * `workspace`: MOBA_OK, or MOBA_ERR_DEVICE_TIMEOUT when a bounded device-side wait gave up.
  * Waits for the stream. */
 moba_status moba_device_status(const moba_params* p, const void* workspace, void* stream);
+
+/* ---- Allocation-free forward (no counterpart in the paper) -----------------------------
+ *
+ * Some callers cannot allocate device memory or hand over a workspace: plugin hosts that own
+ * every device allocation, or services that forbid allocation once they are running.  For
+ * them moba_attn_fwd_noalloc computes exactly what moba_attn_fwd computes with
+ * sel_in = sel_out = NULL and info = NULL, and allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library call).  Its scratch is one array of MOBA_NOALLOC_SCRATCH_BYTES in
+ * static device memory inside the library, held on every GPU that loads the library until
+ * the process exits.
+ *   - p->wave_tokens is ignored: the call picks the largest query wave (a multiple of 128
+ *     tokens) whose workspace fits the array.  A problem that does not fit even with
+ *     128-token waves returns MOBA_ERR_UNSUPPORTED before any launch; moba_last_error() gives
+ *     the bytes it would need.  Other arguments are checked as in moba_attn_fwd.
+ *   - The caller still owns and passes q, k, v, cu_seqlens, out and lse (same layouts).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call before any
+ *     stream capture.
+ *   - All calls on a device share the array and it keeps the previous call's contents; the
+ *     forward re-initialises everything it reads.  Calls whose GPU work overlaps (other
+ *     streams or host threads on the same device) race on the array and must be serialised
+ *     by the caller. */
+#define MOBA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+moba_status moba_attn_fwd_noalloc(const moba_params* p, const void* q, const void* k,
+                                  const void* v, const int* cu_seqlens, void* out, float* lse,
+                                  void* stream);
 
 /* Static description of a status code. */
 const char* moba_status_string(moba_status s);
