@@ -99,28 +99,34 @@ class ClockSampler:
                 "samples_under_load": len(load), "power_w_max": max(pw) if pw else None}
 
 
-def dist_setup(args):
+def dist_setup():
+    """One process per GPU: NCCL process group when WORLD_SIZE > 1 (gloo without CUDA)."""
     import torch
     import torch.distributed as dist
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
+    if world > 1 and not dist.is_initialized():
         from datetime import timedelta
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=timedelta(seconds=300))
     return world, rank, local
 
 
-def max_over_ranks(x, world, device):
+def max_over_ranks(x, world):
+    """Max of a host float over all ranks (the job's time is its slowest rank's)."""
     import torch
     import torch.distributed as dist
 
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -130,6 +136,16 @@ def barrier(world):
 
     if world > 1:
         dist.barrier()
+
+
+def rank_seed(w, rank):
+    """Weak scaling: every rank draws its own independent problem."""
+    return w.seed + 7919 * rank
+
+
+def job_value(tokens_per_rank, world, ms_max):
+    """Whole-job throughput: all ranks' tokens over the slowest rank's time."""
+    return world * tokens_per_rank / (ms_max * 1e-3)
 
 
 def cpu_oracle_sample(w, budget_s, seed=0, inputs=None):
@@ -245,7 +261,7 @@ def run_ours(args, w, world, rank, local):
     del lib
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    x = W.make_inputs(w, device=dev, seed=w.seed + rank)
+    x = W.make_inputs(w, device=dev, seed=rank_seed(w, rank))
     q, k, v, cu = x["q"], x["k"], x["v"], x["cu_seqlens"]
     T, hq, d = q.shape
     hkv = k.shape[1]
@@ -287,7 +303,7 @@ def run_ours(args, w, world, rank, local):
     clocks = sampler.stop()
     barrier(world)
     ms_local = start.elapsed_time(end) / args.steps
-    ms = max_over_ranks(ms_local, world, dev)
+    ms = max_over_ranks(ms_local, world)
     launches = moba.attn_fwd.last_info["launches"]
 
     # per-stage device times (ms per step, mean over steps)
@@ -311,7 +327,7 @@ def run_ours(args, w, world, rank, local):
     long_step = ms > 200.0
     peak = peaks["bf16_tflops_sustained"] if long_step else peaks["bf16_tflops"]
     traffic = _read_traffic(w.name)
-    value = world * T / (ms * 1e-3)
+    value = job_value(T, world, ms)
 
     # end to end through the public API: pinned host inputs -> H2D -> forward -> D2H
     e2e = None
@@ -345,8 +361,8 @@ def run_ours(args, w, world, rank, local):
             e2e_step()
         b.record()
         torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, world, dev)
-        e2e = {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s",
+        e2e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, world)
+        e2e = {"value": job_value(T, world, e2e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                "steps": n_e2e}
 
@@ -454,7 +470,7 @@ def main():
         rank = int(os.environ.get("RANK", "0"))
         run_reference(args, w, world, rank)
         return
-    world, rank, local = dist_setup(args)
+    world, rank, local = dist_setup()
     try:
         run_ours(args, w, world, rank, local)
     finally:
