@@ -9,11 +9,12 @@
 // current-block tile is 128 consecutive tokens of one query head against the causal prefix
 // of their block.  A persistent CTA per SM takes items from an atomic cursor.
 //
-// Warp roles (224 threads):
-//   warps 0-3  softmax + epilogue, thread r owns query row r (TMEM lane r)
-//   warp 4     K/V producer: TMA (SWIZZLE_128B, no multicast) into a 4-stage ring
-//   warp 5     item fetch + Q gather: routed rows by cp.async into a swizzled K-major tile
-//   warp 6     TMEM owner and single-thread MMA issuer
+// Warp roles (352 threads):
+//   warps 0-7  softmax + epilogue: two threads per query row (TMEM lane), 64 key columns
+//              each; the halves agree on the row maximum through a shared exchange
+//   warp 8     K/V producer: TMA (SWIZZLE_128B, no multicast) into a 4-stage ring
+//   warp 9     item fetch + Q gather: routed rows by cp.async into a swizzled K-major tile
+//   warp 10    TMEM owner and single-thread MMA issuer
 // Per 128-key chunk n: S_n = Q K_n^T (SS MMA, fp32 in TMEM, double-buffered), softmax in
 // registers after tcgen05.ld, P_n (bf16) written back over S_n with tcgen05.st, then
 // O += P_n V_n (TS MMA: A from TMEM, V from shared memory, MN-major).  The MMA warp issues
@@ -37,8 +38,9 @@ namespace {
 
 constexpr int kBN = 128;       // keys per chunk
 constexpr int kStages = 4;     // K/V ring depth
-constexpr int kThreads = 224;  // 7 warps
-constexpr int kWarpKV = 4, kWarpQ = 5, kWarpMMA = 6;
+constexpr int kThreads = 352;  // 11 warps
+constexpr int kWarpKV = 8, kWarpQ = 9, kWarpMMA = 10;
+constexpr int kSoftmaxThreads = 256;  // warps 0-7
 constexpr uint32_t kSpinLimit = 1u << 22;  // try_wait polls before a wait is declared stuck
 constexpr int kTimeoutStatus = 5;          // MOBA_ERR_DEVICE_TIMEOUT
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled when max grows > 2^8
@@ -57,8 +59,9 @@ struct SmemLayout {
     static constexpr int kKV = 2 * kTileBytes;         // kStages K/V buffers
     static constexpr int kSlots = kKV + kStages * kTileBytes;
     static constexpr int kBars = kSlots + 2 * (int)sizeof(ItemSlot);
-    static constexpr int kNumBars = 2 + 2 + 2 + kStages + kStages + 2 + 2 + 1 + 2 + 1;
-    static constexpr int kMisc = kBars + kNumBars * 8;
+    static constexpr int kNumBars = 2 + 2 + 2 + kStages + kStages + 2 + 2 + 2 + 1 + 1 + 4;
+    static constexpr int kXchg = kBars + kNumBars * 8;  // row exchange: float [2][2][128]
+    static constexpr int kMisc = kXchg + 2 * 2 * kTileM * 4;
     static constexpr int kBytes = kMisc + 16 + 1024;  // + slack for 1024-byte alignment
 };
 
@@ -171,6 +174,26 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
+// 64 consecutive TMEM columns of this thread's lane (one instruction, waited).
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+    uint32_t r[64];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 2^x on the SFU (PTX ex2.approx.ftz.f32): relative error about 2^-22, -inf -> +0.
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -249,7 +272,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
     auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
     const int B_INFO = 0, B_QFULL = 2, B_ITEM_EMPTY = 4, B_KV_FULL = 6, B_KV_EMPTY = 6 + kStages,
               B_S_FULL = 6 + 2 * kStages, B_P_FULL = B_S_FULL + 2, B_PV_DONE = B_P_FULL + 2,
-              B_O_EMPTY = B_PV_DONE + 2, B_FINAL = B_O_EMPTY + 1;
+              B_O_EMPTY = B_PV_DONE + 2, B_FINAL = B_O_EMPTY + 1, B_PAIR = B_FINAL + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int* status = &ws.hdr->status;
@@ -258,9 +281,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
         for (int i = 0; i < 2; ++i) {
             mbar_init(BAR(B_INFO + i), 32);
             mbar_init(BAR(B_QFULL + i), 32);
-            mbar_init(BAR(B_ITEM_EMPTY + i), 128);
+            mbar_init(BAR(B_ITEM_EMPTY + i), kSoftmaxThreads);
             mbar_init(BAR(B_S_FULL + i), 1);
-            mbar_init(BAR(B_P_FULL + i), 128);
+            mbar_init(BAR(B_P_FULL + i), kSoftmaxThreads);
         }
         for (int i = 0; i < kStages; ++i) {
             mbar_init(BAR(B_KV_FULL + i), 1);
@@ -268,7 +291,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
         }
         mbar_init(BAR(B_PV_DONE), 1);
         mbar_init(BAR(B_PV_DONE + 1), 1);
-        mbar_init(BAR(B_O_EMPTY), 128);
+        mbar_init(BAR(B_O_EMPTY), kSoftmaxThreads);
+        for (int i = 0; i < 4; ++i) mbar_init(BAR(B_PAIR + i), 64);
         mbar_init(BAR(B_FINAL), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -492,11 +516,30 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
         __syncwarp();
         drain_bar(BAR(B_FINAL), 0);
     } else {
-        // ---------------- softmax + epilogue (warps 0-3) ----------------
-        const int row = warp * 32 + lane;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        // ---------------- softmax + epilogue (warps 0-7) ----------------
+        // Warps w and w+4 share TMEM lane quadrant w&3, i.e. query rows 32(w&3) .. +31.  Warp
+        // w < 4 owns key columns 0-63 of every chunk (and O columns 0 .. D/2-1), warp w+4 the
+        // other half.  The two halves of a row agree on the row maximum (and at the end on
+        // the row sum) through a small shared exchange guarded by a per-pair mbarrier.
+        const int quad = warp & 3, hf = warp >> 2;
+        const int row = quad * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        float* xchg = reinterpret_cast<float*>(smem + L::kXchg);  // [parity][half][row]
+        const uint32_t pair_bar = BAR(B_PAIR + quad);
+        uint32_t xph = 0;  // exchanges done by this pair
+        auto exchange = [&](float mine, float& other) -> bool {
+            float* slot = xchg + (xph & 1u) * 2 * kTileM;
+            slot[hf * kTileM + row] = mine;
+            mbar_arrive(pair_bar);
+            const bool r = wait_bar(pair_bar, xph & 1u, abort_flag, status);
+            other = slot[(1 - hf) * kTileM + row];
+            ++xph;
+            return r;
+        };
+        constexpr int kOHalf = D / 2;  // O columns per half
         uint32_t glob = 0;
         const float ln2 = 0.69314718055994531f;
+        const float sl2 = P.scale_log2;
         bool ok = true;
         for (int it = 0; ok; ++it) {
             const int s = it & 1;
@@ -506,8 +549,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
             const int N = sl.nchunks, key_start = sl.key_start, key_end = sl.key_end;
             const int pidx = sl.pidx[row];
             const int tl = sl.tlim[row];
-            const uint32_t o_tmem = tmem + lane_off + kColO;
-            float m = -INFINITY, l = 0.f;
+            const uint32_t o_tmem = tmem + lane_off + kColO + (uint32_t)(hf * kOHalf);
+            float m = -INFINITY;  // running row maximum, log2 units (identical in both halves)
+            float l = 0.f;        // running sum over this half's columns
             for (int n = 0; n < N; ++n) {
                 const uint32_t cg = glob + (uint32_t)n;
                 const uint32_t b = cg & 1u;
@@ -516,26 +560,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                     break;
                 }
                 tc_fence_after();
-                const uint32_t s_tmem = tmem + lane_off + kColS0 + b * kBN;
-                const uint32_t p_tmem = tmem + lane_off + kColP0 + b * (kBN / 2);
-                float x[kBN];
+                float x[64];
+                tmem_ld64(tmem + lane_off + kColS0 + b * kBN + (uint32_t)(hf * 64), x);
+                // keys past the block / after the row (current-block tiles only)
+                const int lim = min(key_end - 1, tl) - (key_start + n * kBN + hf * 64);
+                if (__any_sync(0xffffffffu, lim < 63)) {
 #pragma unroll
-                for (int j = 0; j < kBN / 32; ++j) {
-                    float v[32];
-                    tmem_ld32(s_tmem + 32u * j, v);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) x[32 * j + e] = v[e];
+                    for (int j = 0; j < 64; ++j) x[j] = (j <= lim) ? x[j] : -INFINITY;
                 }
-                tmem_ld_wait();
-                const int key0 = key_start + n * kBN;
-                const int lim = min(key_end - 1, tl) - key0;  // last valid key offset
-                float mloc = -INFINITY;
+                float mx[8];
 #pragma unroll
-                for (int j = 0; j < kBN; ++j) {
-                    const float y = (j <= lim) ? x[j] * P.scale_log2 : -INFINITY;
-                    x[j] = y;
-                    mloc = fmaxf(mloc, y);
+                for (int j = 0; j < 8; ++j) mx[j] = x[j];
+#pragma unroll
+                for (int j = 8; j < 64; ++j) mx[j & 7] = fmaxf(mx[j & 7], x[j]);
+                float mh = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                float mo;
+                if (!exchange(mh, mo)) {
+                    ok = false;
+                    break;
                 }
+                const float mloc = fmaxf(mh, mo) * sl2;
                 if (n == 0) {
                     m = mloc;
                 } else {
@@ -549,12 +594,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                         }
                         tc_fence_after();
                         const float mn = fmaxf(m, mloc);
-                        const float alpha = exp2f(m - mn);
+                        const float alpha = ex2(m - mn);
 #pragma unroll
-                        for (int j = 0; j < D / 32; ++j) {
+                        for (int j = 0; j < kOHalf / 32; ++j) {
                             float v[32];
                             tmem_ld32(o_tmem + 32u * j, v);
-                            tmem_ld_wait();
                             uint32_t w[32];
 #pragma unroll
                             for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(v[e] * alpha);
@@ -565,37 +609,38 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                         m = mn;
                     }
                 }
-                float rs = 0.f;
+                // p = 2^(s * scale * log2(e) - m), packed to bf16 pairs into P
+                const float negm = -m;
+                uint32_t w[32];
+                float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
-                for (int j = 0; j < kBN; ++j) {
-                    const float p = exp2f(x[j] - m);
-                    x[j] = p;
-                    rs += p;
+                for (int e = 0; e < 32; ++e) {
+                    const float p0 = ex2(fmaf(x[2 * e], sl2, negm));
+                    const float p1 = ex2(fmaf(x[2 * e + 1], sl2, negm));
+                    rs0 += p0;
+                    rs1 += p1;
+                    w[e] = pack_bf16(p0, p1);
                 }
-                l += rs;
-#pragma unroll
-                for (int j = 0; j < kBN / 64; ++j) {
-                    uint32_t w[32];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) w[e] = pack_bf16(x[64 * j + 2 * e], x[64 * j + 2 * e + 1]);
-                    tmem_st32(p_tmem + 32u * j, w);
-                }
+                l += rs0 + rs1;
+                tmem_st32(tmem + lane_off + kColP0 + b * (kBN / 2) + (uint32_t)(hf * 32), w);
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(BAR(B_P_FULL + b));
             }
             if (!ok) break;
-            // epilogue: O of the last chunk, normalise, write the partial (o, lse)
+            // epilogue: O of the last chunk, normalise, write this half of the partial (o, lse)
             const uint32_t lastg = glob + (uint32_t)N - 1u;
             if (!wait_bar(BAR(B_PV_DONE + (lastg & 1u)), (lastg >> 1) & 1u, abort_flag, status)) break;
             tc_fence_after();
-            const float inv = 1.f / l;
-            float* dst = ws.part_o + (size_t)(pidx < 0 ? 0 : pidx) * D;
+            float lo;
+            if (!exchange(l, lo)) break;
+            const float ltot = l + lo;
+            const float inv = 1.f / ltot;
+            float* dst = ws.part_o + (size_t)(pidx < 0 ? 0 : pidx) * D + hf * kOHalf;
 #pragma unroll
-            for (int j = 0; j < D / 32; ++j) {
+            for (int j = 0; j < kOHalf / 32; ++j) {
                 float v[32];
                 tmem_ld32(o_tmem + 32u * j, v);
-                tmem_ld_wait();
                 if (pidx >= 0) {
 #pragma unroll
                     for (int e = 0; e < 32; e += 4)
@@ -603,7 +648,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                             make_float4(v[e] * inv, v[e + 1] * inv, v[e + 2] * inv, v[e + 3] * inv);
                 }
             }
-            if (pidx >= 0) ws.part_lse[pidx] = m * ln2 + logf(l);
+            if (pidx >= 0 && hf == 0) ws.part_lse[pidx] = m * ln2 + logf(ltot);
             tc_fence_before();
             mbar_arrive(BAR(B_O_EMPTY));
             mbar_arrive(BAR(B_ITEM_EMPTY + s));
