@@ -5,8 +5,10 @@
 // online-softmax rule.  For partials (o_i, lse_i), i = 0 .. n-1 (slot 0 = own block):
 //   m = max_i lse_i,  w_i = exp(lse_i - m),  o = sum_i w_i o_i / sum_i w_i,
 //   lse = m + log(sum_i w_i).
-// One warp per query row; each lane owns d/32 consecutive channels (vectorised fp32 loads),
-// the output is rounded once to bf16 (nearest even).  HBM-bound.
+// One warp per query row: lane s reads slot s's lse, the maximum and the weights come from
+// warp reductions, then each lane accumulates d/32 consecutive channels with several partial
+// rows in flight (streaming loads).  The output is rounded once to bf16 (nearest even).
+// HBM-bound.
 #include "moba_internal.cuh"
 
 namespace moba {
@@ -20,37 +22,51 @@ __global__ void __launch_bounds__(kWarps * 32)
 merge_kernel(const int* __restrict__ cu, const int* __restrict__ sel, Problem P, Workspace ws,
              int t0, int t1, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
     constexpr int V = D / 32;
+    constexpr int kUnroll = 4;  // partial rows in flight per warp
+    const unsigned full = 0xffffffffu;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long n = (long long)(t1 - t0) * P.hq;
     for (long long r = (long long)blockIdx.x * kWarps + warp; r < n;
          r += (long long)gridDim.x * kWarps) {
         const int t = t0 + (int)(r / P.hq);
         const int h = (int)(r % P.hq);
-        const int i = seq_of_token(cu, P.batch, t);
-        const int c = (t - __ldg(cu + i)) / P.chunk;
-        const int* row = sel + ((size_t)h * P.T + t) * P.topk;
-        const int ns = 1 + for_each_routed(row, P.topk, c, [](int, int) {});
+        const int ns = ws.nslots[r];  // own block + routed history blocks (routing pass)
         const size_t pbase = (size_t)r * P.topk;
-        float mx = -INFINITY;
-        for (int s = 0; s < ns; ++s) mx = fmaxf(mx, ws.part_lse[pbase + s]);
+        // lane s holds slot s: max and weights by warp reductions
+        const float lv = (lane < ns) ? __ldcs(ws.part_lse + pbase + lane) : -INFINITY;
+        float mx = lv;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(full, mx, off));
+        const float wv = (lane < ns) ? expf(lv - mx) : 0.f;
+        float L = wv;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(full, L, off);
         float acc[V];
 #pragma unroll
         for (int u = 0; u < V; ++u) acc[u] = 0.f;
-        float L = 0.f;
-        for (int s = 0; s < ns; ++s) {
-            const float w = expf(ws.part_lse[pbase + s] - mx);
-            L += w;
-            const float* src = ws.part_o + (pbase + s) * D + lane * V;
-            if constexpr (V == 4) {
-                const float4 x = *reinterpret_cast<const float4*>(src);
-                acc[0] = fmaf(w, x.x, acc[0]);
-                acc[1] = fmaf(w, x.y, acc[1]);
-                acc[2] = fmaf(w, x.z, acc[2]);
-                acc[3] = fmaf(w, x.w, acc[3]);
-            } else {
-                const float2 x = *reinterpret_cast<const float2*>(src);
-                acc[0] = fmaf(w, x.x, acc[0]);
-                acc[1] = fmaf(w, x.y, acc[1]);
+        const float* base = ws.part_o + pbase * D + lane * V;
+        for (int s0 = 0; s0 < ns; s0 += kUnroll) {
+            float x[kUnroll][V];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                if (s0 + u < ns) {
+                    if constexpr (V == 4) {
+                        const float4 y = __ldcs(reinterpret_cast<const float4*>(base + (size_t)(s0 + u) * D));
+                        x[u][0] = y.x; x[u][1] = y.y; x[u][2] = y.z; x[u][3] = y.w;
+                    } else {
+                        const float2 y = __ldcs(reinterpret_cast<const float2*>(base + (size_t)(s0 + u) * D));
+                        x[u][0] = y.x; x[u][1] = y.y;
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < V; ++e) x[u][e] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const float w = __shfl_sync(full, wv, (s0 + u) & 31);
+#pragma unroll
+                for (int e = 0; e < V; ++e) acc[e] = fmaf(w, x[u][e], acc[e]);
             }
         }
         const float inv = 1.f / L;

@@ -74,7 +74,7 @@ long long blocks_bound(const moba_params& p) {
 
 struct Layout {
     size_t hdr, cu_blocks, blk_start, blk_len, blk_seq, blk_local, means, sel, counts, offsets,
-        cursor, entries, items, part_o, part_lse, total;
+        cursor, entries, items, part_o, part_lse, nslots, total;
     int wave;
     long long nb_cap, max_items;
 };
@@ -112,6 +112,7 @@ Layout make_layout(const moba_params& p) {
     L.items = take(sizeof(WorkItem) * L.max_items);
     L.part_o = take(4ull * W * p.num_q_heads * p.topk * p.head_dim);
     L.part_lse = take(4ull * W * p.num_q_heads * p.topk);
+    L.nslots = take(1ull * W * p.num_q_heads);
     L.total = o;
     return L;
 }
@@ -195,8 +196,8 @@ moba_status moba_gate_topk(const moba_params* p, const void* q, const float* k_m
     if (!aligned16(q) || !aligned16(k_mean))
         return fail(MOBA_ERR_INVALID_ARG, "q and k_mean must be 16-byte aligned");
     const Problem P = make_problem(*p, blocks_bound(*p));
-    cudaError_t e = launch_gate(P, static_cast<const __nv_bfloat16*>(q), k_mean, cu_seqlens, sel,
-                                static_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_gate_best(P, static_cast<const __nv_bfloat16*>(q), k_mean, cu_seqlens,
+                                     sel, nullptr, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "gate launch");
     return MOBA_OK;
 }
@@ -244,6 +245,7 @@ moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, co
     ws.items = reinterpret_cast<WorkItem*>(base + L.items);
     ws.part_o = reinterpret_cast<float*>(base + L.part_o);
     ws.part_lse = reinterpret_cast<float*>(base + L.part_lse);
+    ws.nslots = reinterpret_cast<unsigned char*>(base + L.nslots);
 
     const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
     const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
@@ -269,7 +271,8 @@ moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, co
     const int* sel_use = sel_in;
     if (!sel_use) {
         int* dst = sel_out ? sel_out : ws.sel;
-        MOBA_TRY(launch_gate(P, qb, ws.means, cu_seqlens, dst, st), "gate launch");
+        MOBA_TRY(launch_gate_best(P, qb, ws.means, cu_seqlens, dst, &ws.hdr->status, st),
+                 "gate launch");
         ++launches;
         sel_use = dst;
     }

@@ -53,6 +53,7 @@ struct Workspace {
     WorkItem* items;  // [max_items]
     float* part_o;    // [wave * hq * topk, d]
     float* part_lse;  // [wave * hq * topk]
+    unsigned char* nslots;  // [wave * hq]: 1 + routed history blocks of each row
 };
 
 // ---------------------------------------------------------------------------------------
@@ -68,21 +69,27 @@ __device__ __forceinline__ int seq_of_token(const int* __restrict__ cu, int batc
     return lo;
 }
 
-// Selection rule shared by routing and merge: entry i of a row is a routed history block iff
+// Selection rule of the routing pass: entry i of a row is a routed history block iff
 // 0 <= j < c, it is not a repeat of an earlier routed entry, and fewer than topk-1 entries
-// have been routed before it.  Returns the number of routed entries and, for each routed
-// entry, calls f(slot, j) with slot = 1 + its rank among the routed entries.
-template <typename F>
+// have been routed before it.  The row (topk <= K entries) is read into registers once.
+// Returns the number of routed entries and, for each routed entry, calls f(slot, j) with
+// slot = 1 + its rank among the routed entries.
+template <int K, typename F>
 __device__ __forceinline__ int for_each_routed(const int* __restrict__ row, int topk, int c, F f) {
+    int v[K];
+#pragma unroll
+    for (int i = 0; i < K; ++i) v[i] = (i < topk) ? __ldg(row + i) : -1;
     int n = 0;
-    for (int i = 0; i < topk; ++i) {
-        int j = row[i];
-        if (j < 0 || j >= c || n >= topk - 1) continue;
-        bool dup = false;
-        for (int i2 = 0; i2 < i; ++i2) dup |= (row[i2] == j);
-        if (dup) continue;
-        f(n + 1, j);
-        ++n;
+#pragma unroll
+    for (int i = 0; i < K; ++i) {
+        const int j = v[i];
+        bool take = j >= 0 && j < c && n < topk - 1;
+#pragma unroll
+        for (int i2 = 0; i2 < i; ++i2) take = take && v[i2] != j;
+        if (take) {
+            f(n + 1, j);
+            ++n;
+        }
     }
     return n;
 }
@@ -96,6 +103,8 @@ cudaError_t launch_meanpool(const Problem& P, const __nv_bfloat16* k, const int*
                             float* means, cudaStream_t st);
 cudaError_t launch_gate(const Problem& P, const __nv_bfloat16* q, const float* means,
                         const int* cu_seqlens, int* sel, cudaStream_t st);
+cudaError_t launch_gate_best(const Problem& P, const __nv_bfloat16* q, const float* means,
+                             const int* cu_seqlens, int* sel, int* status, cudaStream_t st);
 cudaError_t launch_route_count(const Problem& P, const int* cu_seqlens, const int* sel,
                                const Workspace& ws, int t0, int t1, cudaStream_t st);
 cudaError_t launch_route_plan(const Problem& P, const Workspace& ws, int t0, int t1,

@@ -83,29 +83,98 @@ plan_blocks_kernel(const int* __restrict__ cu, Problem P, Workspace ws) {
     }
 }
 
-// One thread per query row (t, h) of the wave.  kScatter = false counts, true scatters.
-template <bool kScatter>
-__global__ void route_rows_kernel(const int* __restrict__ cu, const int* __restrict__ sel,
-                                  Problem P, Workspace ws, int t0, int t1) {
+// Rows of the wave are processed in CTA-sized ranges of consecutive (t, h) rows.  All the
+// lists a range can touch are (g, b) with b in [first block of the range's first sequence,
+// own block of its last row), so a CTA counts its entries in a shared-memory histogram over
+// that span and touches each global list counter once (kScatter = false), or reserves one
+// contiguous range per list with one global atomic and hands out positions from shared
+// memory (kScatter = true).  Spans too wide for shared memory fall back to one global atomic
+// per entry.  Positions inside a list depend on timing, results do not: every row's partial
+// output index travels with it.
+constexpr int kRouteThreads = 256;
+constexpr int kRouteRows = 4096;        // query rows per CTA
+constexpr int kRouteSmemLists = 12288;  // shared-memory histogram capacity (48 KB)
+
+struct RowRef {
+    int t, h, g, c, first;
+    const int* row;
+};
+
+__device__ __forceinline__ RowRef row_ref(const int* __restrict__ cu, const int* __restrict__ sel,
+                                          const Problem& P, const Workspace& ws, int t0,
+                                          long long r) {
+    RowRef x;
+    x.t = t0 + (int)(r / P.hq);
+    x.h = (int)(r % P.hq);
+    const int i = seq_of_token(cu, P.batch, x.t);
+    x.c = (x.t - __ldg(cu + i)) / P.chunk;
+    x.first = ws.cu_blocks[i];
+    x.g = x.h / P.group;
+    x.row = sel + ((size_t)x.h * P.T + x.t) * P.topk;
+    return x;
+}
+
+template <bool kScatter, int K>
+__global__ void __launch_bounds__(kRouteThreads)
+route_rows_kernel(const int* __restrict__ cu, const int* __restrict__ sel, Problem P,
+                  Workspace ws, int t0, int t1) {
+    __shared__ int hist[kRouteSmemLists];
     const long long n = (long long)(t1 - t0) * P.hq;
-    for (long long r = blockIdx.x * (long long)blockDim.x + threadIdx.x; r < n;
-         r += (long long)gridDim.x * blockDim.x) {
-        const int t = t0 + (int)(r / P.hq);
-        const int h = (int)(r % P.hq);
-        const int i = seq_of_token(cu, P.batch, t);
-        const int c = (t - __ldg(cu + i)) / P.chunk;
-        const int first = ws.cu_blocks[i];
-        const int g = h / P.group;
-        const int* row = sel + ((size_t)h * P.T + t) * P.topk;
-        int* lists = ws.counts + (size_t)g * P.nb_cap + first;
+    const long long r0 = (long long)blockIdx.x * kRouteRows;
+    if (r0 >= n) return;
+    const long long r1 = min(n, r0 + kRouteRows);
+    // block span of the lists this range can touch
+    const RowRef a = row_ref(cu, sel, P, ws, t0, r0);
+    const RowRef z = row_ref(cu, sel, P, ws, t0, r1 - 1);
+    const int b_lo = a.first;
+    const int b_hi = z.first + z.c;  // exclusive: history blocks are strictly before c
+    const int span = b_hi - b_lo;
+    if (span <= 0) {  // no row of the range routes anything: one slot (the own block) each
+        if (!kScatter)
+            for (long long r = r0 + threadIdx.x; r < r1; r += kRouteThreads) ws.nslots[r] = 1;
+        return;
+    }
+    const bool in_smem = (long long)P.hkv * span <= kRouteSmemLists;
+    if (!in_smem) {
+        for (long long r = r0 + threadIdx.x; r < r1; r += kRouteThreads) {
+            const RowRef x = row_ref(cu, sel, P, ws, t0, r);
+            const int pbase = (int)(r * P.topk);
+            const int nr = for_each_routed<K>(x.row, P.topk, x.c, [&](int slot, int j) {
+                int* ctr = (kScatter ? ws.cursor : ws.counts) + (size_t)x.g * P.nb_cap + x.first + j;
+                const int pos = atomicAdd(ctr, 1);
+                if (kScatter) ws.entries[pos] = pbase + slot;
+            });
+            if (!kScatter) ws.nslots[r] = (unsigned char)(1 + nr);
+        }
+        return;
+    }
+    const int nl = P.hkv * span;
+    for (int i = threadIdx.x; i < nl; i += kRouteThreads) hist[i] = 0;
+    __syncthreads();
+    for (long long r = r0 + threadIdx.x; r < r1; r += kRouteThreads) {
+        const RowRef x = row_ref(cu, sel, P, ws, t0, r);
+        const int nr = for_each_routed<K>(x.row, P.topk, x.c, [&](int, int j) {
+            atomicAdd(&hist[x.g * span + (x.first + j - b_lo)], 1);
+        });
+        if (!kScatter) ws.nslots[r] = (unsigned char)(1 + nr);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < nl; i += kRouteThreads) {
+        const int cnt = hist[i];
+        if (cnt == 0) continue;
+        const int g = i / span, bb = i - g * span;
+        int* ctr = (kScatter ? ws.cursor : ws.counts) + (size_t)g * P.nb_cap + b_lo + bb;
+        const int base = atomicAdd(ctr, cnt);
+        if (kScatter) hist[i] = base;
+    }
+    if (!kScatter) return;
+    __syncthreads();
+    for (long long r = r0 + threadIdx.x; r < r1; r += kRouteThreads) {
+        const RowRef x = row_ref(cu, sel, P, ws, t0, r);
         const int pbase = (int)(r * P.topk);
-        for_each_routed(row, P.topk, c, [&](int slot, int j) {
-            if (kScatter) {
-                const int pos = atomicAdd(ws.cursor + (size_t)g * P.nb_cap + first + j, 1);
-                ws.entries[pos] = pbase + slot;
-            } else {
-                atomicAdd(lists + j, 1);
-            }
+        for_each_routed<K>(x.row, P.topk, x.c, [&](int slot, int j) {
+            const int pos = atomicAdd(&hist[x.g * span + (x.first + j - b_lo)], 1);
+            ws.entries[pos] = pbase + slot;
         });
     }
 }
@@ -203,11 +272,22 @@ route_plan_kernel(Problem P, Workspace ws, int t0, int t1) {
     }
 }
 
+template <bool kScatter>
+void launch_rows(const Problem& P, const int* cu, const int* sel, const Workspace& ws, int t0,
+                 int t1, int grid, cudaStream_t st) {
+    if (P.topk <= 4)
+        route_rows_kernel<kScatter, 4><<<grid, kRouteThreads, 0, st>>>(cu, sel, P, ws, t0, t1);
+    else if (P.topk <= 8)
+        route_rows_kernel<kScatter, 8><<<grid, kRouteThreads, 0, st>>>(cu, sel, P, ws, t0, t1);
+    else if (P.topk <= 16)
+        route_rows_kernel<kScatter, 16><<<grid, kRouteThreads, 0, st>>>(cu, sel, P, ws, t0, t1);
+    else
+        route_rows_kernel<kScatter, 32><<<grid, kRouteThreads, 0, st>>>(cu, sel, P, ws, t0, t1);
+}
+
 int rows_grid(long long n) {
-    long long g = (n + 255) / 256;
-    if (g > 65536) g = 65536;
-    if (g < 1) g = 1;
-    return (int)g;
+    long long g = (n + kRouteRows - 1) / kRouteRows;
+    return (int)(g < 1 ? 1 : g);
 }
 
 }  // namespace
@@ -221,7 +301,7 @@ cudaError_t launch_plan_blocks(const Problem& P, const int* cu_seqlens, const Wo
 cudaError_t launch_route_count(const Problem& P, const int* cu_seqlens, const int* sel,
                                const Workspace& ws, int t0, int t1, cudaStream_t st) {
     const long long n = (long long)(t1 - t0) * P.hq;
-    route_rows_kernel<false><<<rows_grid(n), 256, 0, st>>>(cu_seqlens, sel, P, ws, t0, t1);
+    launch_rows<false>(P, cu_seqlens, sel, ws, t0, t1, rows_grid(n), st);
     return cudaGetLastError();
 }
 
@@ -234,7 +314,7 @@ cudaError_t launch_route_plan(const Problem& P, const Workspace& ws, int t0, int
 cudaError_t launch_route_scatter(const Problem& P, const int* cu_seqlens, const int* sel,
                                  const Workspace& ws, int t0, int t1, cudaStream_t st) {
     const long long n = (long long)(t1 - t0) * P.hq;
-    route_rows_kernel<true><<<rows_grid(n), 256, 0, st>>>(cu_seqlens, sel, P, ws, t0, t1);
+    launch_rows<true>(P, cu_seqlens, sel, ws, t0, t1, rows_grid(n), st);
     return cudaGetLastError();
 }
 
