@@ -7,21 +7,22 @@
 // Work items (from the routing pass) are 128 query rows against one KV range: a history tile
 // is up to 128 routed rows (any query heads of one KV head) against one whole block, a
 // current-block tile is 128 consecutive tokens of one query head against the causal prefix
-// of their block.  A persistent CTA per SM takes items from an atomic cursor.
+// of their block.  Two persistent CTAs per SM take items from an atomic cursor; each is a
+// single-tile pipeline, and the two run out of phase so that one CTA's softmax overlaps the
+// other's matrix products on the SM's tensor core.
 //
-// Warp roles (352 threads):
-//   warps 0-7  softmax + epilogue: two threads per query row (TMEM lane), 64 key columns
-//              each; the halves agree on the row maximum through a shared exchange
-//   warp 8     K/V producer: TMA (SWIZZLE_128B, no multicast) into a 4-stage ring
-//   warp 9     item fetch + Q gather: routed rows by cp.async into a swizzled K-major tile
-//   warp 10    TMEM owner and single-thread MMA issuer
-// Per 128-key chunk n: S_n = Q K_n^T (SS MMA, fp32 in TMEM, double-buffered), softmax in
-// registers after tcgen05.ld, P_n (bf16) written back over S_n with tcgen05.st, then
-// O += P_n V_n (TS MMA: A from TMEM, V from shared memory, MN-major).  The MMA warp issues
-// QK_{n+1} before PV_n so the tensor core works while the softmax of chunk n runs.  The
-// running max is only raised (and O rescaled) when it grows by more than 2^8, so O is
-// rarely touched.  P has its own TMEM columns (never aliasing S), so QK^T of chunk n+2 can
-// run while PV of chunk n still reads P_n.
+// Warp roles per CTA (224 threads):
+//   warps 0-3  softmax + epilogue, thread r owns query row r (TMEM lane r)
+//   warp 4     K/V producer: TMA (SWIZZLE_128B, no multicast) into a 2-stage ring
+//   warp 5     item fetch + Q gather: routed rows by cp.async into a swizzled K-major tile
+//   warp 6     TMEM owner and single-thread MMA issuer
+// Per 128-key chunk n: S_n = Q K_n^T (SS MMA, fp32 in TMEM); the softmax reads S_n twice with
+// tcgen05.ld (row maximum, then p = 2^(s*scale*log2e - m)) and writes P_n as bf16 pairs over
+// the S columns it has already read; then O += P_n V_n (TS MMA: A = P from TMEM, B = V
+// MN-major from shared memory).  The MMA warp issues PV_{n-1} before QK_n, so the barrier
+// that announces S_n also guarantees that O holds every earlier PV: the softmax may rescale
+// O right away.  The running max is only raised (and O rescaled) when it grows by more than
+// 2^8, so O is rarely touched.  TMEM per CTA: S/P 128 columns + O d columns (256 allocated).
 //
 // Every mbarrier wait is bounded: on expiry the kernel records MOBA_ERR_DEVICE_TIMEOUT in
 // the workspace status word, all roles leave their loops, in-flight copies and MMAs are
@@ -40,10 +41,10 @@ namespace {
 using namespace ptx;
 
 constexpr int kBN = 128;       // keys per chunk
-constexpr int kStages = 4;     // K/V ring depth
-constexpr int kThreads = 352;  // 11 warps
-constexpr int kWarpKV = 8, kWarpQ = 9, kWarpMMA = 10;
-constexpr int kSoftmaxThreads = 256;  // warps 0-7
+constexpr int kStages = 2;     // K/V ring depth
+constexpr int kThreads = 224;  // 7 warps
+constexpr int kWarpKV = 4, kWarpQ = 5, kWarpMMA = 6;
+constexpr int kCtasPerSm = 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled when max grows > 2^8
 
 struct ItemSlot {
@@ -56,47 +57,42 @@ struct ItemSlot {
 template <int D>
 struct SmemLayout {
     static constexpr int kTileBytes = kTileM * D * 2;  // 128 rows of bf16 (Q tile, K or V chunk)
-    static constexpr int kQ = 0;                       // 2 Q buffers
-    static constexpr int kKV = 2 * kTileBytes;         // kStages K/V buffers
+    static constexpr int kQ = 0;                       // one Q buffer
+    static constexpr int kKV = kTileBytes;             // kStages K/V buffers
     static constexpr int kSlots = kKV + kStages * kTileBytes;
     static constexpr int kBars = kSlots + 2 * (int)sizeof(ItemSlot);
-    static constexpr int kNumBars = 2 + 2 + 2 + kStages + kStages + 2 + 2 + 2 + 1 + 1 + 4;
-    static constexpr int kXchg = kBars + kNumBars * 8;  // row exchange: float [2][2][128]
-    static constexpr int kMisc = kXchg + 2 * 2 * kTileM * 4;
+    static constexpr int kNumBars = 16;
+    static constexpr int kMisc = kBars + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16 + 1024;  // + slack for 1024-byte alignment
 };
 
-// ---------------------------------------------------------------------------------------
-
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                const __nv_bfloat16* __restrict__ q, Problem P, Workspace ws, int t0, int t1) {
     using L = SmemLayout<D>;
-    constexpr int kHalves = D / 64;          // 128-byte swizzle atoms along d
+    constexpr int kHalves = D / 64;           // 128-byte swizzle atoms along d
     constexpr int kHalfBytes = kTileM * 128;  // one [128 rows x 64 bf16] swizzled half
     constexpr uint32_t kChunkBytes = kTileM * D * 2;
     constexpr int kKSteps = D / 16;           // QK^T k-steps (16 bf16 each)
     constexpr uint32_t kIdescQK = idesc_bf16(kBN, false);
     constexpr uint32_t kIdescPV = idesc_bf16(D, true);
-    // TMEM columns: S0, S1 (fp32, 128 each), P0, P1 (bf16 pairs, 64 each), O (D)
-    constexpr uint32_t kColS0 = 0, kColP0 = 2 * kBN, kColO = 3 * kBN;
+    constexpr uint32_t kColS = 0, kColO = kBN;  // TMEM: S (P over its first 64 columns), O
+    constexpr uint32_t kTmemCols = 256;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     ItemSlot* slots = reinterpret_cast<ItemSlot*>(smem + L::kSlots);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
     const uint32_t sm_base = smem_u32(smem);
-    const uint32_t bar0 = smem_u32(bars);
-    // barrier indices
+    const uint32_t bar0 = sm_base + L::kBars;
     auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-    const int B_INFO = 0, B_QFULL = 2, B_ITEM_EMPTY = 4, B_KV_FULL = 6, B_KV_EMPTY = 6 + kStages,
-              B_S_FULL = 6 + 2 * kStages, B_P_FULL = B_S_FULL + 2, B_PV_DONE = B_P_FULL + 2,
-              B_O_EMPTY = B_PV_DONE + 2, B_FINAL = B_O_EMPTY + 1, B_PAIR = B_FINAL + 1;
+    const int B_INFO = 0, B_ITEM_EMPTY = 2, B_QFULL = 4, B_QEMPTY = 5, B_KV_FULL = 6,
+              B_KV_EMPTY = 6 + kStages, B_SFULL = 6 + 2 * kStages, B_PFULL = B_SFULL + 1,
+              B_OFULL = B_PFULL + 1, B_OEMPTY = B_OFULL + 1, B_FINAL = B_OEMPTY + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int* status = &ws.hdr->status;
@@ -104,26 +100,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(BAR(B_INFO + i), 32);
-            mbar_init(BAR(B_QFULL + i), 32);
-            mbar_init(BAR(B_ITEM_EMPTY + i), kSoftmaxThreads);
-            mbar_init(BAR(B_S_FULL + i), 1);
-            mbar_init(BAR(B_P_FULL + i), kSoftmaxThreads);
+            mbar_init(BAR(B_ITEM_EMPTY + i), 128);
         }
         for (int i = 0; i < kStages; ++i) {
             mbar_init(BAR(B_KV_FULL + i), 1);
             mbar_init(BAR(B_KV_EMPTY + i), 1);
         }
-        mbar_init(BAR(B_PV_DONE), 1);
-        mbar_init(BAR(B_PV_DONE + 1), 1);
-        mbar_init(BAR(B_O_EMPTY), kSoftmaxThreads);
-        for (int i = 0; i < 4; ++i) mbar_init(BAR(B_PAIR + i), 64);
+        mbar_init(BAR(B_QFULL), 32);
+        mbar_init(BAR(B_QEMPTY), 1);
+        mbar_init(BAR(B_SFULL), 1);
+        mbar_init(BAR(B_PFULL), 128);
+        mbar_init(BAR(B_OFULL), 1);
+        mbar_init(BAR(B_OEMPTY), 128);
         mbar_init(BAR(B_FINAL), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == kWarpMMA) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
-                         smem_u32(tmem_slot)));
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)), "r"(kTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     tc_fence_before();
@@ -199,8 +194,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
             }
             __syncwarp();
             mbar_arrive(BAR(B_INFO + s));
-            // gather the 128 rows: lane handles rows lane + 32 i, all 16-byte chunks
-            const uint32_t qbuf = sm_base + L::kQ + (uint32_t)s * L::kTileBytes;
+            // the single Q buffer is free once every QK^T of the previous item has completed
+            if (it >= 1 && !wait_bar(BAR(B_QEMPTY), (uint32_t)(it - 1) & 1u, abort_flag, status)) break;
+            const uint32_t qbuf = sm_base + L::kQ;
 #pragma unroll
             for (int i = 0; i < kTileM / 32; ++i) {
                 const int r = lane + 32 * i;
@@ -216,10 +212,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
             asm volatile("cp.async.commit_group;" ::: "memory");
             asm volatile("cp.async.wait_group 0;" ::: "memory");
             fence_proxy_async();
-            mbar_arrive(BAR(B_QFULL + s));
+            mbar_arrive(BAR(B_QFULL));
         }
     } else if (warp == kWarpKV) {
-        // ---------------- K/V producer (TMA) ----------------
+        // ---------------- K/V producer (TMA), in MMA consumption order K0 V0 K1 V1 ... ----------
         uint32_t c = 0;  // ring position
         for (int it = 0;; ++it) {
             const int s = it & 1;
@@ -227,12 +223,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
             const ItemSlot& sl = slots[s];
             if (sl.kind < 0) break;
             const int g = sl.g, key_start = sl.key_start, N = sl.nchunks;
-            // consumption order of the MMA warp: K0, then per n: K_{n+1} (if any), V_n
-            auto load = [&](bool is_v, int chunk) -> bool {
+            bool ok = true;
+            for (int j = 0; j < 2 * N && ok; ++j) {
+                const bool is_v = (j & 1) != 0;
+                const int chunk = j >> 1;
                 const uint32_t st = c % kStages;
                 if (c >= kStages &&
-                    !wait_bar(BAR(B_KV_EMPTY + st), ((c / kStages) - 1u) & 1u, abort_flag, status))
-                    return false;
+                    !wait_bar(BAR(B_KV_EMPTY + st), ((c / kStages) - 1u) & 1u, abort_flag, status)) {
+                    ok = false;
+                    break;
+                }
                 if (lane == 0) {
                     const uint32_t dst = sm_base + L::kKV + st * L::kTileBytes;
                     mbar_arrive_tx(BAR(B_KV_FULL + st), kChunkBytes);
@@ -244,12 +244,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                 }
                 __syncwarp();
                 ++c;
-                return true;
-            };
-            bool ok = load(false, 0);
-            for (int n = 0; n < N && ok; ++n) {
-                if (n + 1 < N) ok = load(false, n + 1);
-                if (ok) ok = load(true, n);
             }
             if (!ok) break;
         }
@@ -258,80 +252,70 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
         for (uint32_t k = (issued > kStages ? issued - kStages : 0); k < issued; ++k)
             drain_bar(BAR(B_KV_FULL + k % kStages), (k / kStages) & 1u);
     } else if (warp == kWarpMMA) {
-        // ---------------- MMA issuer ----------------
+        // ---------------- MMA issuer: QK0, then per n >= 1: PV_{n-1}, QK_n; finally PV_{N-1} ----
         uint32_t c = 0;     // ring position
-        uint32_t glob = 0;  // global chunk counter (S buffers, pv_done phases)
+        uint32_t glob = 0;  // global chunk counter (S / P barrier phases)
         bool ok = true;
+        const uint32_t s_tmem = tmem + kColS, o_tmem = tmem + kColO;
+        auto wait_stage = [&]() -> uint32_t {
+            const uint32_t st = c % kStages;
+            if (!wait_bar(BAR(B_KV_FULL + st), (c / kStages) & 1u, abort_flag, status)) return ~0u;
+            tc_fence_after();
+            return st;
+        };
         for (int it = 0; ok; ++it) {
             const int s = it & 1;
-            const uint32_t ph = (uint32_t)(it >> 1) & 1u;
-            if (!wait_bar(BAR(B_INFO + s), ph, abort_flag, status)) break;
+            if (!wait_bar(BAR(B_INFO + s), (uint32_t)(it >> 1) & 1u, abort_flag, status)) break;
             const ItemSlot& sl = slots[s];
             if (sl.kind < 0) break;
             const int N = sl.nchunks;
-            if (!wait_bar(BAR(B_QFULL + s), ph, abort_flag, status)) break;
+            if (!wait_bar(BAR(B_QFULL), (uint32_t)it & 1u, abort_flag, status)) break;
             tc_fence_after();
-            const uint32_t qbuf = sm_base + L::kQ + (uint32_t)s * L::kTileBytes;
-            const uint32_t o_tmem = tmem + kColO;
-            auto issue_qk = [&](uint32_t chunk_g) -> bool {
-                const uint32_t st = c % kStages;
-                if (!wait_bar(BAR(B_KV_FULL + st), (c / kStages) & 1u, abort_flag, status))
-                    return false;
-                tc_fence_after();
-                const uint32_t kbuf = sm_base + L::kKV + st * L::kTileBytes;
-                const uint32_t s_tmem = tmem + kColS0 + (chunk_g & 1u) * kBN;
-                if (lane == 0) {
-#pragma unroll
-                    for (int kk = 0; kk < kKSteps; ++kk) {
-                        const uint32_t koff = (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32u;
-                        mma_ss(s_tmem, smem_desc(qbuf + koff, 16, 1024), smem_desc(kbuf + koff, 16, 1024),
-                               kIdescQK, kk > 0 ? 1u : 0u);
+            const uint32_t qbuf = sm_base + L::kQ;
+            for (int n = 0; n <= N && ok; ++n) {
+                if (n > 0) {
+                    // PV_{n-1}: P from TMEM (16 keys = 8 packed columns per step), V MN-major
+                    const uint32_t pg = glob + (uint32_t)(n - 1);
+                    if (!wait_bar(BAR(B_PFULL), pg & 1u, abort_flag, status)) { ok = false; break; }
+                    if (n == 1 && it >= 1 &&
+                        !wait_bar(BAR(B_OEMPTY), (uint32_t)(it - 1) & 1u, abort_flag, status)) {
+                        ok = false;
+                        break;
                     }
-                    mma_commit(BAR(B_KV_EMPTY + st));
-                    mma_commit(BAR(B_S_FULL + (chunk_g & 1u)));
-                }
-                __syncwarp();
-                ++c;
-                return true;
-            };
-            if (!issue_qk(glob)) break;
-            for (int n = 0; n < N; ++n) {
-                if (n + 1 < N && !issue_qk(glob + n + 1)) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t cg = glob + (uint32_t)n;
-                // O is single-buffered: the previous item's epilogue must have read it
-                if (n == 0 && it >= 1 &&
-                    !wait_bar(BAR(B_O_EMPTY), (uint32_t)(it - 1) & 1u, abort_flag, status)) {
-                    ok = false;
-                    break;
-                }
-                if (!wait_bar(BAR(B_P_FULL + (cg & 1u)), (cg >> 1) & 1u, abort_flag, status)) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t st = c % kStages;
-                if (!wait_bar(BAR(B_KV_FULL + st), (c / kStages) & 1u, abort_flag, status)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t vbuf = sm_base + L::kKV + st * L::kTileBytes;
-                const uint32_t p_tmem = tmem + kColP0 + (cg & 1u) * (kBN / 2);
-                if (lane == 0) {
+                    const uint32_t st = wait_stage();
+                    if (st == ~0u) { ok = false; break; }
+                    const uint32_t vbuf = sm_base + L::kKV + st * L::kTileBytes;
+                    if (lane == 0) {
 #pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk) {
-                        // A = P: 16 keys = 8 packed columns; B = V rows kk*16.., MN-major
-                        mma_ts(o_tmem, p_tmem + (uint32_t)kk * 8u,
-                               smem_desc(vbuf + (uint32_t)kk * 2048u, (uint32_t)kHalfBytes, 1024),
-                               kIdescPV, (n > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < kBN / 16; ++kk)
+                            mma_ts(o_tmem, s_tmem + (uint32_t)kk * 8u,
+                                   smem_desc(vbuf + (uint32_t)kk * 2048u, (uint32_t)kHalfBytes, 1024),
+                                   kIdescPV, (n > 1 || kk > 0) ? 1u : 0u);
+                        mma_commit(BAR(B_KV_EMPTY + st));
+                        if (n == N) mma_commit(BAR(B_OFULL));
                     }
-                    mma_commit(BAR(B_KV_EMPTY + st));
-                    mma_commit(BAR(B_PV_DONE + (cg & 1u)));
+                    __syncwarp();
+                    ++c;
                 }
-                __syncwarp();
-                ++c;
+                if (n < N) {
+                    // QK_n into S (after PV_{n-1} in issue order, so P_{n-1} has been read)
+                    const uint32_t st = wait_stage();
+                    if (st == ~0u) { ok = false; break; }
+                    const uint32_t kbuf = sm_base + L::kKV + st * L::kTileBytes;
+                    if (lane == 0) {
+#pragma unroll
+                        for (int kk = 0; kk < kKSteps; ++kk) {
+                            const uint32_t koff = (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32u;
+                            mma_ss(s_tmem, smem_desc(qbuf + koff, 16, 1024),
+                                   smem_desc(kbuf + koff, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+                        }
+                        mma_commit(BAR(B_KV_EMPTY + st));
+                        mma_commit(BAR(B_SFULL));
+                        if (n == N - 1) mma_commit(BAR(B_QEMPTY));
+                    }
+                    __syncwarp();
+                    ++c;
+                }
             }
             glob += (uint32_t)N;
         }
@@ -340,27 +324,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
         __syncwarp();
         drain_bar(BAR(B_FINAL), 0);
     } else {
-        // ---------------- softmax + epilogue (warps 0-7) ----------------
-        // Warps w and w+4 share TMEM lane quadrant w&3, i.e. query rows 32(w&3) .. +31.  Warp
-        // w < 4 owns key columns 0-63 of every chunk (and O columns 0 .. D/2-1), warp w+4 the
-        // other half.  The two halves of a row agree on the row maximum (and at the end on
-        // the row sum) through a small shared exchange guarded by a per-pair mbarrier.
-        const int quad = warp & 3, hf = warp >> 2;
-        const int row = quad * 32 + lane;
-        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        float* xchg = reinterpret_cast<float*>(smem + L::kXchg);  // [parity][half][row]
-        const uint32_t pair_bar = BAR(B_PAIR + quad);
-        uint32_t xph = 0;  // exchanges done by this pair
-        auto exchange = [&](float mine, float& other) -> bool {
-            float* slot = xchg + (xph & 1u) * 2 * kTileM;
-            slot[hf * kTileM + row] = mine;
-            mbar_arrive(pair_bar);
-            const bool r = wait_bar(pair_bar, xph & 1u, abort_flag, status);
-            other = slot[(1 - hf) * kTileM + row];
-            ++xph;
-            return r;
-        };
-        constexpr int kOHalf = D / 2;  // O columns per half
+        // ---------------- softmax + epilogue (warps 0-3), thread = query row ----------------
+        const int row = warp * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t s_tmem = tmem + lane_off + kColS, o_tmem = tmem + lane_off + kColO;
         uint32_t glob = 0;
         const float ln2 = 0.69314718055994531f;
         const float sl2 = P.scale_log2;
@@ -373,96 +340,91 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
             const int N = sl.nchunks, key_start = sl.key_start, key_end = sl.key_end;
             const int pidx = sl.pidx[row];
             const int tl = sl.tlim[row];
-            const uint32_t o_tmem = tmem + lane_off + kColO + (uint32_t)(hf * kOHalf);
-            float m = -INFINITY;  // running row maximum, log2 units (identical in both halves)
-            float l = 0.f;        // running sum over this half's columns
+            float m = -INFINITY;  // running row maximum, log2 units
+            float l = 0.f;        // running row sum of p
             for (int n = 0; n < N; ++n) {
                 const uint32_t cg = glob + (uint32_t)n;
-                const uint32_t b = cg & 1u;
-                if (!wait_bar(BAR(B_S_FULL + b), (cg >> 1) & 1u, abort_flag, status)) {
+                if (!wait_bar(BAR(B_SFULL), cg & 1u, abort_flag, status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                float x[64];
-                tmem_ld64(tmem + lane_off + kColS0 + b * kBN + (uint32_t)(hf * 64), x);
                 // keys past the block / after the row (current-block tiles only)
-                const int lim = min(key_end - 1, tl) - (key_start + n * kBN + hf * 64);
-                if (__any_sync(0xffffffffu, lim < 63)) {
+                const int lim = min(key_end - 1, tl) - (key_start + n * kBN);
+                const bool masked = __any_sync(0xffffffffu, lim < kBN - 1);
+                // pass 1: row maximum of the raw scores
+                float mh = -INFINITY;
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) x[j] = (j <= lim) ? x[j] : -INFINITY;
+                for (int hh = 0; hh < 2; ++hh) {
+                    float x[64];
+                    tmem_ld64(s_tmem + 64u * hh, x);
+                    if (masked) {
+#pragma unroll
+                        for (int j = 0; j < 64; ++j) x[j] = (64 * hh + j <= lim) ? x[j] : -INFINITY;
+                    }
+                    float mx[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) mx[j] = x[j];
+#pragma unroll
+                    for (int j = 8; j < 64; ++j) mx[j & 7] = fmaxf(mx[j & 7], x[j]);
+                    mh = fmaxf(mh, fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))));
                 }
-                float mx[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) mx[j] = x[j];
-#pragma unroll
-                for (int j = 8; j < 64; ++j) mx[j & 7] = fmaxf(mx[j & 7], x[j]);
-                float mh = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-                float mo;
-                if (!exchange(mh, mo)) {
-                    ok = false;
-                    break;
-                }
-                const float mloc = fmaxf(mh, mo) * sl2;
+                const float mloc = mh * sl2;
                 if (n == 0) {
                     m = mloc;
-                } else {
-                    const bool need = mloc > m + kRescaleThreshold;
-                    if (__any_sync(0xffffffffu, need)) {
-                        // O must hold every earlier PV before it is rescaled
-                        const uint32_t pg = cg - 1u;
-                        if (!wait_bar(BAR(B_PV_DONE + (pg & 1u)), (pg >> 1) & 1u, abort_flag, status)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const float mn = fmaxf(m, mloc);
-                        const float alpha = ex2(m - mn);
+                } else if (__any_sync(0xffffffffu, mloc > m + kRescaleThreshold)) {
+                    // S_n was committed after PV_{n-1}: O already holds every earlier PV
+                    const float mn = fmaxf(m, mloc);
+                    const float alpha = ex2(m - mn);
 #pragma unroll
-                        for (int j = 0; j < kOHalf / 32; ++j) {
-                            float v[32];
-                            tmem_ld32(o_tmem + 32u * j, v);
-                            uint32_t w[32];
+                    for (int j = 0; j < D / 32; ++j) {
+                        float v[32];
+                        tmem_ld32(o_tmem + 32u * j, v);
+                        uint32_t w[32];
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(v[e] * alpha);
-                            tmem_st32(o_tmem + 32u * j, w);
-                        }
-                        tmem_st_wait();
-                        l *= alpha;
-                        m = mn;
+                        for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(v[e] * alpha);
+                        tmem_st32(o_tmem + 32u * j, w);
                     }
+                    tmem_st_wait();
+                    l *= alpha;
+                    m = mn;
                 }
-                // p = 2^(s * scale * log2(e) - m), packed to bf16 pairs into P
+                // pass 2: p = 2^(s * scale * log2(e) - m) as bf16 pairs over the read S columns
                 const float negm = -m;
-                uint32_t w[32];
                 float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const float p0 = ex2(fmaf(x[2 * e], sl2, negm));
-                    const float p1 = ex2(fmaf(x[2 * e + 1], sl2, negm));
-                    rs0 += p0;
-                    rs1 += p1;
-                    w[e] = pack_bf16(p0, p1);
+                for (int hh = 0; hh < 2; ++hh) {
+                    float x[64];
+                    tmem_ld64(s_tmem + 64u * hh, x);
+                    if (masked) {
+#pragma unroll
+                        for (int j = 0; j < 64; ++j) x[j] = (64 * hh + j <= lim) ? x[j] : -INFINITY;
+                    }
+                    uint32_t w[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const float p0 = ex2(fmaf(x[2 * e], sl2, negm));
+                        const float p1 = ex2(fmaf(x[2 * e + 1], sl2, negm));
+                        rs0 += p0;
+                        rs1 += p1;
+                        w[e] = pack_bf16(p0, p1);
+                    }
+                    tmem_st32(s_tmem + 32u * hh, w);
                 }
                 l += rs0 + rs1;
-                tmem_st32(tmem + lane_off + kColP0 + b * (kBN / 2) + (uint32_t)(hf * 32), w);
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(BAR(B_P_FULL + b));
+                mbar_arrive(BAR(B_PFULL));
             }
             if (!ok) break;
-            // epilogue: O of the last chunk, normalise, write this half of the partial (o, lse)
-            const uint32_t lastg = glob + (uint32_t)N - 1u;
-            if (!wait_bar(BAR(B_PV_DONE + (lastg & 1u)), (lastg >> 1) & 1u, abort_flag, status)) break;
+            // epilogue: O after the last PV, normalise, write the partial (o, lse)
+            if (!wait_bar(BAR(B_OFULL), (uint32_t)it & 1u, abort_flag, status)) break;
             tc_fence_after();
-            float lo;
-            if (!exchange(l, lo)) break;
-            const float ltot = l + lo;
-            const float inv = 1.f / ltot;
-            float* dst = ws.part_o + (size_t)(pidx < 0 ? 0 : pidx) * D + hf * kOHalf;
+            const float inv = 1.f / l;
+            float* dst = ws.part_o + (size_t)(pidx < 0 ? 0 : pidx) * D;
 #pragma unroll
-            for (int j = 0; j < kOHalf / 32; ++j) {
+            for (int j = 0; j < D / 32; ++j) {
                 float v[32];
                 tmem_ld32(o_tmem + 32u * j, v);
                 if (pidx >= 0) {
@@ -472,9 +434,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                             make_float4(v[e] * inv, v[e + 1] * inv, v[e + 2] * inv, v[e + 3] * inv);
                 }
             }
-            if (pidx >= 0 && hf == 0) ws.part_lse[pidx] = m * ln2 + logf(ltot);
+            if (pidx >= 0) ws.part_lse[pidx] = m * ln2 + logf(l);
             tc_fence_before();
-            mbar_arrive(BAR(B_O_EMPTY));
+            mbar_arrive(BAR(B_OEMPTY));
             mbar_arrive(BAR(B_ITEM_EMPTY + s));
             glob += (uint32_t)N;
         }
@@ -484,7 +446,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
     __syncthreads();
     tc_fence_after();
     if (warp == kWarpMMA) {
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
     }
 }
 
@@ -535,7 +497,7 @@ cudaError_t launch_tc_d(const Problem& P, const __nv_bfloat16* q, const __nv_bfl
     const int smem = SmemLayout<D>::kBytes;
     e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_tc_kernel<D><<<num_sms, kThreads, smem, st>>>(mk, mv, q, P, ws, t0, t1);
+    attn_tc_kernel<D><<<num_sms * kCtasPerSm, kThreads, smem, st>>>(mk, mv, q, P, ws, t0, t1);
     return cudaGetLastError();
 }
 
