@@ -66,6 +66,25 @@ struct SmemLayout {
     static constexpr int kBytes = kMisc + 16 + 1024;  // + slack for 1024-byte alignment
 };
 
+// One butterfly stage of an 8x8 transpose of float4 elements across the 8 lanes of a lane
+// group: lanes i and i^DIST exchange the element pairs whose index bit DIST differs from
+// their lane bit.  After stages 4, 2, 1, lane i holds a[j] = original a[i] of lane j.
+template <int DIST>
+__device__ __forceinline__ void transpose8x8(float4 (&a)[8], int lane) {
+    const bool up = (lane & DIST) != 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        if (j & DIST) continue;
+        const float4 send = up ? a[j] : a[j | DIST];
+        float4 recv;
+        recv.x = __shfl_xor_sync(0xffffffffu, send.x, DIST);
+        recv.y = __shfl_xor_sync(0xffffffffu, send.y, DIST);
+        recv.z = __shfl_xor_sync(0xffffffffu, send.z, DIST);
+        recv.w = __shfl_xor_sync(0xffffffffu, send.w, DIST);
+        if (up) a[j] = recv; else a[j | DIST] = recv;
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
@@ -422,17 +441,30 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
             if (!wait_bar(BAR(B_OFULL), (uint32_t)it & 1u, abort_flag, status)) break;
             tc_fence_after();
             const float inv = 1.f / l;
-            float* dst = ws.part_o + (size_t)(pidx < 0 ? 0 : pidx) * D;
+            // Rows are 512-byte partial-output records at scattered addresses.  A thread owns a
+            // row, so storing straight from registers would touch 32 cache lines per warp
+            // store.  Instead each group of 8 lanes transposes 8x8 blocks of float4 by shuffles
+            // and every store instruction writes 128 contiguous bytes of 4 rows.
+            int prow[8];
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) prow[jj] = __shfl_sync(0xffffffffu, pidx, (lane & ~7) + jj);
+            const int seg = lane & 7;
 #pragma unroll
             for (int j = 0; j < D / 32; ++j) {
                 float v[32];
                 tmem_ld32(o_tmem + 32u * j, v);
-                if (pidx >= 0) {
+                float4 a[8];
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        *reinterpret_cast<float4*>(dst + 32 * j + e) =
-                            make_float4(v[e] * inv, v[e + 1] * inv, v[e + 2] * inv, v[e + 3] * inv);
-                }
+                for (int e = 0; e < 8; ++e)
+                    a[e] = make_float4(v[4 * e] * inv, v[4 * e + 1] * inv, v[4 * e + 2] * inv,
+                                       v[4 * e + 3] * inv);
+                transpose8x8<4>(a, lane);
+                transpose8x8<2>(a, lane);
+                transpose8x8<1>(a, lane);
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj)
+                    if (prow[jj] >= 0)
+                        *reinterpret_cast<float4*>(ws.part_o + (size_t)prow[jj] * D + 32 * j + 4 * seg) = a[jj];
             }
             if (pidx >= 0) ws.part_lse[pidx] = m * ln2 + logf(l);
             tc_fence_before();
