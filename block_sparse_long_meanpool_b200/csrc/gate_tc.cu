@@ -42,6 +42,26 @@ struct GateSmem {
     static constexpr int kBytes(int n) { return kBars(n) + 8 * 8 + 16 + 1024; }
 };
 
+// Inserts (x, id) into a descending list of K (score, index) pairs when it beats the last
+// entry; an equal score never displaces an entry already in the list.
+template <int K>
+__device__ __forceinline__ void insert_desc(float (&val)[K], int (&idx)[K], float x, int id,
+                                            bool ok) {
+    if (ok && x > val[K - 1]) {
+#pragma unroll
+        for (int i = 0; i < K; ++i) {
+            if (x > val[i]) {
+                const float tv = val[i];
+                const int ti = idx[i];
+                val[i] = x;
+                idx[i] = id;
+                x = tv;
+                id = ti;
+            }
+        }
+    }
+}
+
 template <int D, int KMAX>
 __global__ void __launch_bounds__(kThreads, 1)
 gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restrict__ means,
@@ -203,34 +223,41 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
             const int sb = ti & 1;
             if (!wait_bar(BAR(B_SFULL + sb), (uint32_t)(ti >> 1) & 1u, abort_flag, st)) break;
             tc_fence_after();
-            float val[KMAX];
-            int idx[KMAX];
+            // two independent descending lists (even / odd columns) for instruction-level
+            // parallelism, merged at the end; inside a list, columns arrive in increasing order
+            // and an equal score never displaces an earlier (lower-index) block
+            float val[KMAX], val2[KMAX];
+            int idx[KMAX], idx2[KMAX];
 #pragma unroll
             for (int i = 0; i < KMAX; ++i) {
-                val[i] = -INFINITY;
-                idx[i] = INT_MAX;
+                val[i] = val2[i] = -INFINITY;
+                idx[i] = idx2[i] = INT_MAX;
             }
             const uint32_t s_tmem = tmem + lane_off + (uint32_t)sb * kMaxPast;
             for (int j0 = 0; j0 < c; j0 += 32) {
                 float v[32];
                 tmem_ld32(s_tmem + (uint32_t)j0, v);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    float x = v[e];
-                    int id = j0 + e;
-                    if (id < c && x > val[KMAX - 1]) {
-                        // insertion into the descending list; equal scores keep the lower index
+                for (int e = 0; e < 32; e += 2) {
+                    insert_desc<KMAX>(val, idx, v[e], j0 + e, j0 + e < c);
+                    insert_desc<KMAX>(val2, idx2, v[e + 1], j0 + e + 1, j0 + e + 1 < c);
+                }
+            }
+            // merge: scores from the odd list enter with the full (score, lower index) order
 #pragma unroll
-                        for (int i = 0; i < KMAX; ++i) {
-                            if (x > val[i]) {
-                                const float tv = val[i];
-                                const int tix = idx[i];
-                                val[i] = x;
-                                idx[i] = id;
-                                x = tv;
-                                id = tix;
-                            }
-                        }
+            for (int i = 0; i < KMAX; ++i) {
+                float x = val2[i];
+                int id = idx2[i];
+#pragma unroll
+                for (int k2 = 0; k2 < KMAX; ++k2) {
+                    const bool better = x > val[k2] || (x == val[k2] && id < idx[k2]);
+                    if (better) {
+                        const float tv = val[k2];
+                        const int ti = idx[k2];
+                        val[k2] = x;
+                        idx[k2] = id;
+                        x = tv;
+                        id = ti;
                     }
                 }
             }
@@ -318,6 +345,7 @@ cudaError_t launch_tc_k(const Problem& P, const __nv_bfloat16* q, const float* m
     if (need <= 2) return launch_tc<D, 2>(P, q, means, cu, sel, status, n_max, st);
     if (need <= 4) return launch_tc<D, 4>(P, q, means, cu, sel, status, n_max, st);
     if (need <= 8) return launch_tc<D, 8>(P, q, means, cu, sel, status, n_max, st);
+    if (need <= 11) return launch_tc<D, 11>(P, q, means, cu, sel, status, n_max, st);
     if (need <= 16) return launch_tc<D, 16>(P, q, means, cu, sel, status, n_max, st);
     return launch_tc<D, 32>(P, q, means, cu, sel, status, n_max, st);
 }

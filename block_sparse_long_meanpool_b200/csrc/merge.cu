@@ -5,10 +5,11 @@
 // online-softmax rule.  For partials (o_i, lse_i), i = 0 .. n-1 (slot 0 = own block):
 //   m = max_i lse_i,  w_i = exp(lse_i - m),  o = sum_i w_i o_i / sum_i w_i,
 //   lse = m + log(sum_i w_i).
-// One warp per query row: lane s reads slot s's lse, the maximum and the weights come from
-// warp reductions, then each lane accumulates d/32 consecutive channels with several partial
-// rows in flight (streaming loads).  The output is rounded once to bf16 (nearest even).
-// HBM-bound.
+// A half-warp per query row (two rows per warp): the first partial rows are loaded before the
+// weights are known, lane s reads slot s's lse (and s + 16), the maximum and the weights come
+// from half-warp reductions, and each lane accumulates d/16 consecutive channels with four
+// partial rows in flight (streaming loads).  The output is rounded once to bf16 (nearest
+// even).  HBM-bound.
 #include "moba_internal.cuh"
 
 namespace moba {
@@ -21,67 +22,88 @@ template <int D>
 __global__ void __launch_bounds__(kWarps * 32)
 merge_kernel(const int* __restrict__ cu, const int* __restrict__ sel, Problem P, Workspace ws,
              int t0, int t1, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
-    constexpr int V = D / 32;
-    constexpr int kUnroll = 4;  // partial rows in flight per warp
+    constexpr int V = D / 16;   // channels per lane: a half-warp (16 lanes) owns one row
+    constexpr int kUnroll = 4;  // partial rows in flight per half-warp
     const unsigned full = 0xffffffffu;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int hl = lane & 15, half = lane >> 4;
     const long long n = (long long)(t1 - t0) * P.hq;
-    for (long long r = (long long)blockIdx.x * kWarps + warp; r < n;
-         r += (long long)gridDim.x * kWarps) {
-        const int t = t0 + (int)(r / P.hq);
-        const int h = (int)(r % P.hq);
-        const int ns = ws.nslots[r];  // own block + routed history blocks (routing pass)
-        const size_t pbase = (size_t)r * P.topk;
-        // lane s holds slot s: max and weights by warp reductions
-        const float lv = (lane < ns) ? __ldcs(ws.part_lse + pbase + lane) : -INFINITY;
-        float mx = lv;
+    const long long stride = (long long)gridDim.x * kWarps * 2;
+    for (long long base = ((long long)blockIdx.x * kWarps + warp) * 2; base < n; base += stride) {
+        const long long r = base + half;
+        const bool valid = r < n;
+        const int ns = valid ? (int)ws.nslots[r] : 0;  // own block + routed history blocks
+        const size_t pbase = (size_t)(valid ? r : 0) * P.topk;
+        const float* obase = ws.part_o + pbase * D + hl * V;
+        // first partial rows in flight before the weights are known
+        float x[kUnroll][V];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(full, mx, off));
-        const float wv = (lane < ns) ? expf(lv - mx) : 0.f;
-        float L = wv;
+        for (int u = 0; u < kUnroll; ++u) {
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(full, L, off);
+            for (int e = 0; e < V; e += 4) {
+                float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (u < ns) y = __ldcs(reinterpret_cast<const float4*>(obase + (size_t)u * D + e));
+                x[u][e] = y.x; x[u][e + 1] = y.y; x[u][e + 2] = y.z; x[u][e + 3] = y.w;
+            }
+        }
+        // slot lse: lane hl holds slots hl and hl + 16; max and weights by half-warp reductions
+        const float la = (hl < ns) ? __ldcs(ws.part_lse + pbase + hl) : -INFINITY;
+        const float lb = (hl + 16 < ns) ? __ldcs(ws.part_lse + pbase + hl + 16) : -INFINITY;
+        float mx = fmaxf(la, lb);
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(full, mx, off));
+        const float wa = (hl < ns) ? expf(la - mx) : 0.f;
+        const float wb = (hl + 16 < ns) ? expf(lb - mx) : 0.f;
+        float L = wa + wb;
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) L += __shfl_xor_sync(full, L, off);
         float acc[V];
 #pragma unroll
-        for (int u = 0; u < V; ++u) acc[u] = 0.f;
-        const float* base = ws.part_o + pbase * D + lane * V;
-        for (int s0 = 0; s0 < ns; s0 += kUnroll) {
-            float x[kUnroll][V];
+        for (int e = 0; e < V; ++e) acc[e] = 0.f;
+        const int src0 = half * 16;
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const float w = __shfl_sync(full, wa, src0 + u);
+#pragma unroll
+            for (int e = 0; e < V; ++e) acc[e] = fmaf(w, x[u][e], acc[e]);
+        }
+        const int ns_max = max(__shfl_sync(full, ns, 0), __shfl_sync(full, ns, 16));
+        for (int s0 = kUnroll; s0 < ns_max; s0 += kUnroll) {
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u) {
-                if (s0 + u < ns) {
-                    if constexpr (V == 4) {
-                        const float4 y = __ldcs(reinterpret_cast<const float4*>(base + (size_t)(s0 + u) * D));
-                        x[u][0] = y.x; x[u][1] = y.y; x[u][2] = y.z; x[u][3] = y.w;
-                    } else {
-                        const float2 y = __ldcs(reinterpret_cast<const float2*>(base + (size_t)(s0 + u) * D));
-                        x[u][0] = y.x; x[u][1] = y.y;
-                    }
-                } else {
 #pragma unroll
-                    for (int e = 0; e < V; ++e) x[u][e] = 0.f;
+                for (int e = 0; e < V; e += 4) {
+                    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (s0 + u < ns)
+                        y = __ldcs(reinterpret_cast<const float4*>(obase + (size_t)(s0 + u) * D + e));
+                    x[u][e] = y.x; x[u][e + 1] = y.y; x[u][e + 2] = y.z; x[u][e + 3] = y.w;
                 }
             }
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u) {
-                const float w = __shfl_sync(full, wv, (s0 + u) & 31);
+                const int sl = s0 + u;  // < 32
+                const float w = (sl < 16) ? __shfl_sync(full, wa, src0 + (sl & 15))
+                                          : __shfl_sync(full, wb, src0 + (sl & 15));
 #pragma unroll
                 for (int e = 0; e < V; ++e) acc[e] = fmaf(w, x[u][e], acc[e]);
             }
         }
+        if (!valid) continue;
+        const int t = t0 + (int)(r / P.hq);
+        const int h = (int)(r % P.hq);
         const float inv = 1.f / L;
-        __nv_bfloat16* dst = out + ((size_t)t * P.hq + h) * D + lane * V;
-        if constexpr (V == 4) {
-            __nv_bfloat162 a = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
-            __nv_bfloat162 b = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
-            uint2 pk;
-            pk.x = *reinterpret_cast<uint32_t*>(&a);
-            pk.y = *reinterpret_cast<uint32_t*>(&b);
-            *reinterpret_cast<uint2*>(dst) = pk;
-        } else {
-            *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
+        __nv_bfloat16* dst = out + ((size_t)t * P.hq + h) * D + hl * V;
+        uint32_t pk[V / 2];
+#pragma unroll
+        for (int e = 0; e < V; e += 2) {
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
+            pk[e / 2] = *reinterpret_cast<uint32_t*>(&b2);
         }
-        if (lane == 0) lse[(size_t)h * P.T + t] = mx + logf(L);
+        if constexpr (V == 8)
+            *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        else
+            *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
+        if (hl == 0) lse[(size_t)h * P.T + t] = mx + logf(L);
     }
 }
 
@@ -91,7 +113,7 @@ cudaError_t launch_merge(const Problem& P, const int* cu_seqlens, const int* sel
                          const Workspace& ws, int t0, int t1, __nv_bfloat16* out, float* lse,
                          cudaStream_t st) {
     const long long n = (long long)(t1 - t0) * P.hq;
-    long long grid = (n + kWarps - 1) / kWarps;
+    long long grid = (n + 2 * kWarps - 1) / (2 * kWarps);
     if (grid > 148 * 64) grid = 148 * 64;
     if (grid < 1) grid = 1;
     if (P.d == 64)
