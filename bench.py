@@ -410,7 +410,14 @@ def _hbm_stage_rates(w, st, peaks):
     nb = sum((n + w.chunk_size - 1) // w.chunk_size for n in w.seqlens)
     mean_bytes = T * hkv * d * 2 + nb * hkv * d * 4
     gate_bytes = T * hq * d * 2 + T * hq * w.topk * 4 + nb * hkv * d * 4
-    merge_bytes = T * hq * (w.topk * (d + 1) * 4 + d * 2 + 4)
+    # merge: every row reads its min(topk, c + 1) partials (c = the row's block in its
+    # sequence) as fp32 o + lse and its slot count, and writes bf16 o + fp32 lse
+    slots = 0
+    for n in w.seqlens:
+        for c in range((n + w.chunk_size - 1) // w.chunk_size):
+            rows = min(w.chunk_size, n - c * w.chunk_size)
+            slots += rows * min(w.topk, c + 1)
+    merge_bytes = hq * (slots * (d + 1) * 4 + T * (1 + d * 2 + 4))
     res = {}
     for name, by in (("meanpool", mean_bytes), ("gate", gate_bytes)):
         ms = st[name]
@@ -419,7 +426,7 @@ def _hbm_stage_rates(w, st, peaks):
                      "frac": (gbs / peaks["hbm_gbs"]) if gbs else None}
     ms = st["merge"]
     gbs = merge_bytes / (ms * 1e-3) / 1e9 if ms > 0 else None
-    res["merge"] = {"bytes_upper": merge_bytes, "GB/s": gbs,
+    res["merge"] = {"bytes": merge_bytes, "GB/s": gbs,
                     "frac": (gbs / peaks["hbm_gbs"]) if gbs else None}
     return res
 
@@ -464,7 +471,7 @@ def main():
         ap.error("--warmup must be >= 3")
     from block_sparse_long_meanpool_b200 import workloads as W
 
-    w = W.WORKLOADS[args.workload]
+    w = W.ALL_WORKLOADS[args.workload]
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))

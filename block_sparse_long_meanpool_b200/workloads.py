@@ -67,6 +67,25 @@ WORKLOADS = {
         "1 x 1,048,576 tokens, 32 q / 8 kv heads, d=128, chunk 4096 (256 blocks), top-12"),
 }
 
+# Sweeps on the same kernels.
+# Block granularity at fixed 75% sparsity on 32K tokens: n blocks, n/4 selected (the analysis,
+# §4.2, Figure 4: 8 choose 2 ... 128 choose 32).
+GRANULARITY_32K = {
+    f"fine_32k_{n}_{n // 4}": Workload(
+        f"fine_32k_{n}_{n // 4}", [32768], 32, 8, 128, 32768 // n, n // 4, "k_offsets", 1100 + n,
+        f"1 x 32768 tokens, 32 q / 8 kv heads, d=128, {n} blocks of {32768 // n}, top-{n // 4}")
+    for n in (8, 16, 32, 64, 128)
+}
+# Context length with block count and top-k fixed and the block size growing with the
+# length (the analysis, §4.5: how the 10M-token measurement was set up), Llama-3.1-8B shape.
+LENGTH_SWEEP = {
+    f"prefill_{m}m": Workload(
+        f"prefill_{m}m", [m << 20], 32, 8, 128, (m << 20) // 256, 12, "k_offsets", 1200 + m,
+        f"1 x {m << 20} tokens, 32 q / 8 kv heads, d=128, 256 blocks of {(m << 20) // 256}, top-12")
+    for m in (2, 4)
+}
+ALL_WORKLOADS = {**WORKLOADS, **GRANULARITY_32K, **LENGTH_SWEEP}
+
 
 def custom(name, seqlens, hq, hkv, d, chunk, topk, structure="k_offsets", seed=7):
     """A workload of any shape with the same value recipe (for tests and sweeps)."""

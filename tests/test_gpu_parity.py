@@ -158,13 +158,13 @@ def test_softmax_scale_parameter():
                  ref["out"].reshape(T * 2, -1), ref["lse"].T.reshape(-1))
 
 
-FULL = ["scaling_8k", "long_32k", "varlen_gqa"]
+FULL = ["scaling_8k", "long_32k", "varlen_gqa", "fine_32k_8_2", "fine_32k_128_32"]
 
 
 @pytest.mark.parametrize("name", FULL)
 def test_full_size_workload(name):
     """All means, all selections, sampled output rows; then the oracle-feed mode."""
-    w = W.WORKLOADS[name]
+    w = W.ALL_WORKLOADS[name]
     q, k, v, cu_t = gpu_inputs(w)
     cu = np.asarray(w.cu_seqlens)
     chunk, topk, hq = w.chunk_size, w.topk, w.num_q_heads
