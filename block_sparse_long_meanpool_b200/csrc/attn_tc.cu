@@ -4,25 +4,30 @@
 // mask (rule 1 of §2.3 already excluded every future block), the own block with a causal
 // mask, and the partial softmax results are merged afterwards by their log-sum-exp.
 //
-// Work items (from the routing pass) are 128 query rows against one KV range: a history tile
-// is up to 128 routed rows (any query heads of one KV head) against one whole block, a
-// current-block tile is 128 consecutive tokens of one query head against the causal prefix
-// of their block.  Two persistent CTAs per SM take items from an atomic cursor; each is a
-// single-tile pipeline, and the two run out of phase so that one CTA's softmax overlaps the
-// other's matrix products on the SM's tensor core.
+// Work items (from the routing pass) hold up to two 128-row query tiles against one KV range
+// of one KV head: a history item is up to 256 routed rows (any query heads of that KV head)
+// against one whole block; a current-block item is 128 consecutive tokens of one or two query
+// heads of that KV head against the causal prefix of their block.  Every K/V chunk loaded into
+// shared memory serves both tiles.  One persistent CTA per SM takes items from an atomic cursor.
 //
-// Warp roles per CTA (224 threads):
-//   warps 0-3  softmax + epilogue, thread r owns query row r (TMEM lane r)
-//   warp 4     K/V producer: TMA (SWIZZLE_128B, no multicast) into a 2-stage ring
-//   warp 5     item fetch + Q gather: routed rows by cp.async into a swizzled K-major tile
-//   warp 6     TMEM owner and single-thread MMA issuer
-// Per 128-key chunk n: S_n = Q K_n^T (SS MMA, fp32 in TMEM); the softmax reads S_n twice with
-// tcgen05.ld (row maximum, then p = 2^(s*scale*log2e - m)) and writes P_n as bf16 pairs over
-// the S columns it has already read; then O += P_n V_n (TS MMA: A = P from TMEM, B = V
-// MN-major from shared memory).  The MMA warp issues PV_{n-1} before QK_n, so the barrier
-// that announces S_n also guarantees that O holds every earlier PV: the softmax may rescale
-// O right away.  The running max is only raised (and O rescaled) when it grows by more than
-// 2^8, so O is rarely touched.  TMEM per CTA: S/P 128 columns + O d columns (256 allocated).
+// Warp roles (384 threads; setmaxnreg gives the softmax warps 192 registers, enough to hold a
+// whole 128-score row, and the other warpgroup 120):
+//   warps 0-3   softmax + epilogue of tile 0, thread r owns row r (TMEM lane r)
+//   warps 4-7   softmax + epilogue of tile 1
+//   warp 8      item fetch + Q gather of both tiles (cp.async into swizzled K-major tiles)
+//   warp 9      TMEM owner and single-thread MMA issuer
+//   warp 10     K/V producer: TMA (SWIZZLE_128B, no multicast) into a 4-stage ring
+//   warp 11     idle
+// TMEM (512 columns): S_0, S_1 (128 each; P_t as bf16 pairs over the first 64 columns of S_t),
+// O_0, O_1 (d each).  Per 128-key chunk n the MMA warp issues, tile by tile,
+//   PV_t(n-1): O_t += P_t(n-1) V(n-1)   (TS MMA: A = P from TMEM, B = V MN-major in smem)
+//   QK_t(n):   S_t  = Q_t K(n)^T        (SS MMA, fp32 accumulate)
+// so the tensor core works on one tile while the other tile's softmax runs.  PV_t(n-1) is
+// issued before QK_t(n), so the barrier announcing S_t(n) also guarantees that O_t holds every
+// earlier PV and that no MMA touches O_t until P_t(n) is announced: the softmax may rescale O_t
+// in between.  The softmax reads its row of S once (tcgen05.ld), takes the maximum with
+// three-input max, computes p = 2^(s*scale*log2e - m) with packed two-lane FMAs and the SFU, and
+// raises the running maximum m (rescaling O_t) only when it grows by more than 2^8.
 //
 // Every mbarrier wait is bounded: on expiry the kernel records MOBA_ERR_DEVICE_TIMEOUT in
 // the workspace status word, all roles leave their loops, in-flight copies and MMAs are
@@ -41,27 +46,32 @@ namespace {
 using namespace ptx;
 
 constexpr int kBN = 128;       // keys per chunk
-constexpr int kStages = 2;     // K/V ring depth
-constexpr int kThreads = 224;  // 7 warps
-constexpr int kWarpKV = 4, kWarpQ = 5, kWarpMMA = 6;
-constexpr int kCtasPerSm = 2;
+constexpr int kStages = 4;     // K/V ring depth (entries K0 V0 K1 V1 ...)
+constexpr int kThreads = 384;  // 12 warps
+constexpr int kWarpFetch = 8, kWarpMMA = 9, kWarpKV = 10;
+constexpr int kRegsSoftmax = 192, kRegsOther = 120;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled when max grows > 2^8
 
+// launched with 65536 / 384 -> 168 registers per thread; the split must not exceed that
+static_assert(8 * 32 * kRegsSoftmax + 4 * 32 * kRegsOther <= 168 * kThreads,
+              "setmaxnreg split exceeds the registers the CTA is launched with");
+
 struct ItemSlot {
-    int kind;  // -1 = no more work
+    int kind;    // -1 = no more work
+    int ntiles;  // 1 or 2
     int g, key_start, key_end, nchunks;
-    int pidx[kTileM];
-    int tlim[kTileM];
+    int pidx[kItemRows];  // partial-output index of each row (-1 = no row)
+    int tlim[kTileM];     // last key a row may see (current-block items), else INT_MAX
 };
 
 template <int D>
 struct SmemLayout {
     static constexpr int kTileBytes = kTileM * D * 2;  // 128 rows of bf16 (Q tile, K or V chunk)
-    static constexpr int kQ = 0;                       // one Q buffer
-    static constexpr int kKV = kTileBytes;             // kStages K/V buffers
+    static constexpr int kQ = 0;                       // Q_0, Q_1
+    static constexpr int kKV = 2 * kTileBytes;         // kStages K/V buffers
     static constexpr int kSlots = kKV + kStages * kTileBytes;
     static constexpr int kBars = kSlots + 2 * (int)sizeof(ItemSlot);
-    static constexpr int kNumBars = 16;
+    static constexpr int kNumBars = 24;
     static constexpr int kMisc = kBars + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16 + 1024;  // + slack for 1024-byte alignment
 };
@@ -86,7 +96,7 @@ __device__ __forceinline__ void transpose8x8(float4 (&a)[8], int lane) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+__global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                const __nv_bfloat16* __restrict__ q, Problem P, Workspace ws, int t0, int t1) {
     using L = SmemLayout<D>;
@@ -96,8 +106,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
     constexpr int kKSteps = D / 16;           // QK^T k-steps (16 bf16 each)
     constexpr uint32_t kIdescQK = idesc_bf16(kBN, false);
     constexpr uint32_t kIdescPV = idesc_bf16(D, true);
-    constexpr uint32_t kColS = 0, kColO = kBN;  // TMEM: S (P over its first 64 columns), O
-    constexpr uint32_t kTmemCols = 256;
+    constexpr uint32_t kColO = 2 * kBN;       // TMEM: S_0 at 0, S_1 at 128, O_0, O_1 from 256
+    constexpr uint32_t kTmemCols = 512;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -109,9 +119,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
     const uint32_t sm_base = smem_u32(smem);
     const uint32_t bar0 = sm_base + L::kBars;
     auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-    const int B_INFO = 0, B_ITEM_EMPTY = 2, B_QFULL = 4, B_QEMPTY = 5, B_KV_FULL = 6,
-              B_KV_EMPTY = 6 + kStages, B_SFULL = 6 + 2 * kStages, B_PFULL = B_SFULL + 1,
-              B_OFULL = B_PFULL + 1, B_OEMPTY = B_OFULL + 1, B_FINAL = B_OEMPTY + 1;
+    constexpr int B_INFO = 0, B_ITEM_EMPTY = 2, B_QFULL = 4, B_QEMPTY = 5, B_KV_FULL = 6,
+                  B_KV_EMPTY = B_KV_FULL + kStages, B_SFULL = B_KV_EMPTY + kStages,
+                  B_PFULL = B_SFULL + 2, B_OFULL = B_PFULL + 2, B_OEMPTY = B_OFULL + 2,
+                  B_FINAL = B_OEMPTY + 2;
+    static_assert(B_FINAL < L::kNumBars, "barrier area too small");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int* status = &ws.hdr->status;
@@ -119,7 +131,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(BAR(B_INFO + i), 32);
-            mbar_init(BAR(B_ITEM_EMPTY + i), 128);
+            mbar_init(BAR(B_ITEM_EMPTY + i), 2 * kTileM);
+            mbar_init(BAR(B_SFULL + i), 1);
+            mbar_init(BAR(B_PFULL + i), kTileM);
+            mbar_init(BAR(B_OFULL + i), 1);
+            mbar_init(BAR(B_OEMPTY + i), kTileM);
         }
         for (int i = 0; i < kStages; ++i) {
             mbar_init(BAR(B_KV_FULL + i), 1);
@@ -127,10 +143,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
         }
         mbar_init(BAR(B_QFULL), 32);
         mbar_init(BAR(B_QEMPTY), 1);
-        mbar_init(BAR(B_SFULL), 1);
-        mbar_init(BAR(B_PFULL), 128);
-        mbar_init(BAR(B_OFULL), 1);
-        mbar_init(BAR(B_OEMPTY), 128);
         mbar_init(BAR(B_FINAL), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -144,258 +156,303 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-
-    if (warp == kWarpQ) {
-        // ---------------- item fetch + Q gather ----------------
-        const int n_items = ws.hdr->n_items;
-        constexpr int CK = D / 8;  // 16-byte chunks per row
-        for (int it = 0;; ++it) {
-            const int s = it & 1;
-            const uint32_t ph = (uint32_t)(it >> 1) & 1u;
-            if (it >= 2 && !wait_bar(BAR(B_ITEM_EMPTY + s), ph ^ 1u, abort_flag, status)) break;
-            int idx = 0;
-            if (lane == 0) idx = (int)atomicAdd(&ws.hdr->work_counter, 1u);
-            idx = __shfl_sync(0xffffffffu, idx, 0);
-            ItemSlot& sl = slots[s];
-            if (idx >= n_items) {
-                if (lane == 0) sl.kind = -1;
-                __syncwarp();
-                mbar_arrive(BAR(B_INFO + s));
-                break;
-            }
-            const WorkItem w = ws.items[idx];
-            int g, key_start, key_end;
-            long long qoff[kTileM / 32];
-            if (w.kind == 0) {
-                g = w.a / P.nb_cap;
-                const int b = w.a - g * P.nb_cap;
-                key_start = ws.blk_start[b];
-                key_end = key_start + ws.blk_len[b];
-#pragma unroll
-                for (int i = 0; i < kTileM / 32; ++i) {
-                    const int r = lane + 32 * i;
-                    int pidx = -1;
-                    long long off = -1;
-                    if (r < w.c) {
-                        pidx = ws.entries[w.b + r];
-                        const int rid = pidx / P.topk;
-                        const int t = t0 + rid / P.hq;
-                        const int h = rid - (rid / P.hq) * P.hq;
-                        off = ((long long)t * P.hq + h) * D;
-                    }
-                    sl.pidx[r] = pidx;
-                    sl.tlim[r] = INT_MAX;
-                    qoff[i] = off;
-                }
-            } else {
-                const int b = w.a, h = w.b, qt = w.c;
-                g = h / P.group;
-                key_start = ws.blk_start[b];
-                const int len = ws.blk_len[b];
-                key_end = key_start + min((qt + 1) * kTileM, len);
-#pragma unroll
-                for (int i = 0; i < kTileM / 32; ++i) {
-                    const int r = lane + 32 * i;
-                    const int rr = qt * kTileM + r;
-                    const int t = key_start + rr;
-                    const bool ok = rr < len && t >= t0 && t < t1;
-                    sl.pidx[r] = ok ? ((t - t0) * P.hq + h) * P.topk : -1;
-                    sl.tlim[r] = ok ? t : INT_MAX;
-                    qoff[i] = ok ? ((long long)t * P.hq + h) * D : -1;
-                }
-            }
-            if (lane == 0) {
-                sl.kind = w.kind;
-                sl.g = g;
-                sl.key_start = key_start;
-                sl.key_end = key_end;
-                sl.nchunks = (key_end - key_start + kBN - 1) / kBN;
-            }
-            __syncwarp();
-            mbar_arrive(BAR(B_INFO + s));
-            // the single Q buffer is free once every QK^T of the previous item has completed
-            if (it >= 1 && !wait_bar(BAR(B_QEMPTY), (uint32_t)(it - 1) & 1u, abort_flag, status)) break;
-            const uint32_t qbuf = sm_base + L::kQ;
-#pragma unroll
-            for (int i = 0; i < kTileM / 32; ++i) {
-                const int r = lane + 32 * i;
-                const long long off = qoff[i];
-                const __nv_bfloat16* src = off >= 0 ? q + off : q;
-#pragma unroll
-                for (int c = 0; c < CK; ++c) {
-                    const uint32_t dst = qbuf + (uint32_t)(c >> 3) * kHalfBytes + (uint32_t)r * 128u +
-                                         (uint32_t)(((c & 7) ^ (r & 7)) << 4);
-                    cp_async16(dst, src + (off >= 0 ? c * 8 : 0), off >= 0);
-                }
-            }
-            asm volatile("cp.async.commit_group;" ::: "memory");
-            asm volatile("cp.async.wait_group 0;" ::: "memory");
-            fence_proxy_async();
-            mbar_arrive(BAR(B_QFULL));
-        }
-    } else if (warp == kWarpKV) {
-        // ---------------- K/V producer (TMA), in MMA consumption order K0 V0 K1 V1 ... ----------
-        uint32_t c = 0;  // ring position
-        for (int it = 0;; ++it) {
-            const int s = it & 1;
-            if (!wait_bar(BAR(B_INFO + s), (uint32_t)(it >> 1) & 1u, abort_flag, status)) break;
-            const ItemSlot& sl = slots[s];
-            if (sl.kind < 0) break;
-            const int g = sl.g, key_start = sl.key_start, N = sl.nchunks;
-            bool ok = true;
-            for (int j = 0; j < 2 * N && ok; ++j) {
-                const bool is_v = (j & 1) != 0;
-                const int chunk = j >> 1;
-                const uint32_t st = c % kStages;
-                if (c >= kStages &&
-                    !wait_bar(BAR(B_KV_EMPTY + st), ((c / kStages) - 1u) & 1u, abort_flag, status)) {
-                    ok = false;
+    if (warp >= 8) {
+        // loads, MMA issue (and one idle warp): few registers
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+        if (warp == kWarpFetch) {
+            // ---------------- item fetch + Q gather (both tiles) ----------------
+            const int n_items = ws.hdr->n_items;
+            constexpr int CK = D / 8;  // 16-byte chunks per row
+            for (int it = 0;; ++it) {
+                const int s = it & 1;
+                const uint32_t ph = (uint32_t)(it >> 1) & 1u;
+                if (it >= 2 && !wait_bar(BAR(B_ITEM_EMPTY + s), ph ^ 1u, abort_flag, status)) break;
+                int idx = 0;
+                if (lane == 0) idx = (int)atomicAdd(&ws.hdr->work_counter, 1u);
+                idx = __shfl_sync(0xffffffffu, idx, 0);
+                ItemSlot& sl = slots[s];
+                if (idx >= n_items) {
+                    if (lane == 0) sl.kind = -1;
+                    __syncwarp();
+                    mbar_arrive(BAR(B_INFO + s));
                     break;
                 }
+                const WorkItem w = ws.items[idx];
+                int g, key_start, key_end, ntiles;
+                if (w.kind == 0) {
+                    g = w.a / P.nb_cap;
+                    const int b = w.a - g * P.nb_cap;
+                    key_start = ws.blk_start[b];
+                    key_end = key_start + ws.blk_len[b];
+                    ntiles = w.c > kTileM ? 2 : 1;
+                    for (int r = lane; r < kItemRows; r += 32)
+                        sl.pidx[r] = (r < w.c) ? ws.entries[w.b + r] : -1;
+                    for (int r = lane; r < kTileM; r += 32) sl.tlim[r] = INT_MAX;
+                } else {
+                    const int b = w.a, h0 = w.b, qt = w.c;
+                    ntiles = w.kind == 2 ? 2 : 1;
+                    g = h0 / P.group;
+                    key_start = ws.blk_start[b];
+                    const int len = ws.blk_len[b];
+                    key_end = key_start + min((qt + 1) * kTileM, len);
+                    for (int r = lane; r < kTileM; r += 32) {
+                        const int rr = qt * kTileM + r;
+                        const int t = key_start + rr;
+                        const bool ok = rr < len && t >= t0 && t < t1;
+                        const int base = ((t - t0) * P.hq + h0) * P.topk;  // slot 0 of (t, h0)
+                        sl.pidx[r] = ok ? base : -1;
+                        sl.pidx[kTileM + r] = (ok && ntiles == 2) ? base + P.topk : -1;
+                        sl.tlim[r] = ok ? t : INT_MAX;
+                    }
+                }
+                const int N = (key_end - key_start + kBN - 1) / kBN;  // >= 1
                 if (lane == 0) {
-                    const uint32_t dst = sm_base + L::kKV + st * L::kTileBytes;
-                    mbar_arrive_tx(BAR(B_KV_FULL + st), kChunkBytes);
-                    const void* tm = is_v ? (const void*)&tmap_v : (const void*)&tmap_k;
-#pragma unroll
-                    for (int hh = 0; hh < kHalves; ++hh)
-                        tma_load_3d(dst + hh * kHalfBytes, tm, BAR(B_KV_FULL + st), hh * 64, g,
-                                    key_start + chunk * kBN);
+                    sl.kind = w.kind;
+                    sl.ntiles = ntiles;
+                    sl.g = g;
+                    sl.key_start = key_start;
+                    sl.key_end = key_end;
+                    sl.nchunks = N;
                 }
                 __syncwarp();
-                ++c;
+                mbar_arrive(BAR(B_INFO + s));
+                // the Q buffers are free once every QK^T of the previous item has completed
+                if (it >= 1 && !wait_bar(BAR(B_QEMPTY), (uint32_t)(it - 1) & 1u, abort_flag, status)) break;
+                // a row's partial index encodes (token - t0) * Hq + head, times topk
+#pragma unroll 1
+                for (int r = lane; r < ntiles * kTileM; r += 32) {
+                    const int pi = sl.pidx[r];
+                    const bool valid = pi >= 0;
+                    const __nv_bfloat16* src =
+                        valid ? q + ((long long)t0 * P.hq + pi / P.topk) * D : q;
+                    const int rr = r & (kTileM - 1);
+                    const uint32_t rbase = sm_base + L::kQ + (uint32_t)(r >> 7) * L::kTileBytes +
+                                           (uint32_t)rr * 128u;
+    #pragma unroll
+                    for (int cc = 0; cc < CK; ++cc) {
+                        const uint32_t dst = rbase + (uint32_t)(cc >> 3) * kHalfBytes +
+                                             (uint32_t)(((cc & 7) ^ (rr & 7)) << 4);
+                        cp_async16(dst, src + (valid ? cc * 8 : 0), valid);
+                    }
+                }
+                asm volatile("cp.async.commit_group;" ::: "memory");
+                asm volatile("cp.async.wait_group 0;" ::: "memory");
+                fence_proxy_async();
+                mbar_arrive(BAR(B_QFULL));
             }
-            if (!ok) break;
-        }
-        // drain: every issued load must land before the CTA exits
-        const uint32_t issued = c;
-        for (uint32_t k = (issued > kStages ? issued - kStages : 0); k < issued; ++k)
-            drain_bar(BAR(B_KV_FULL + k % kStages), (k / kStages) & 1u);
-    } else if (warp == kWarpMMA) {
-        // ---------------- MMA issuer: QK0, then per n >= 1: PV_{n-1}, QK_n; finally PV_{N-1} ----
-        uint32_t c = 0;     // ring position
-        uint32_t glob = 0;  // global chunk counter (S / P barrier phases)
-        bool ok = true;
-        const uint32_t s_tmem = tmem + kColS, o_tmem = tmem + kColO;
-        auto wait_stage = [&]() -> uint32_t {
-            const uint32_t st = c % kStages;
-            if (!wait_bar(BAR(B_KV_FULL + st), (c / kStages) & 1u, abort_flag, status)) return ~0u;
-            tc_fence_after();
-            return st;
-        };
-        for (int it = 0; ok; ++it) {
-            const int s = it & 1;
-            if (!wait_bar(BAR(B_INFO + s), (uint32_t)(it >> 1) & 1u, abort_flag, status)) break;
-            const ItemSlot& sl = slots[s];
-            if (sl.kind < 0) break;
-            const int N = sl.nchunks;
-            if (!wait_bar(BAR(B_QFULL), (uint32_t)it & 1u, abort_flag, status)) break;
-            tc_fence_after();
-            const uint32_t qbuf = sm_base + L::kQ;
-            for (int n = 0; n <= N && ok; ++n) {
-                if (n > 0) {
-                    // PV_{n-1}: P from TMEM (16 keys = 8 packed columns per step), V MN-major
-                    const uint32_t pg = glob + (uint32_t)(n - 1);
-                    if (!wait_bar(BAR(B_PFULL), pg & 1u, abort_flag, status)) { ok = false; break; }
-                    if (n == 1 && it >= 1 &&
-                        !wait_bar(BAR(B_OEMPTY), (uint32_t)(it - 1) & 1u, abort_flag, status)) {
+        } else if (warp == kWarpKV) {
+            // ---------------- K/V producer (TMA), in ring order K0 V0 K1 V1 ... ----------------
+            uint32_t c = 0;  // ring position
+            for (int it = 0;; ++it) {
+                const int s = it & 1;
+                if (!wait_bar(BAR(B_INFO + s), (uint32_t)(it >> 1) & 1u, abort_flag, status)) break;
+                const ItemSlot& sl = slots[s];
+                if (sl.kind < 0) break;
+                const int g = sl.g, key_start = sl.key_start, N = sl.nchunks;
+                bool ok = true;
+                for (int j = 0; j < 2 * N; ++j) {
+                    const bool is_v = (j & 1) != 0;
+                    const int chunk = j >> 1;
+                    const uint32_t st = c % kStages;
+                    if (c >= kStages &&
+                        !wait_bar(BAR(B_KV_EMPTY + st), ((c / kStages) - 1u) & 1u, abort_flag, status)) {
                         ok = false;
                         break;
                     }
-                    const uint32_t st = wait_stage();
-                    if (st == ~0u) { ok = false; break; }
-                    const uint32_t vbuf = sm_base + L::kKV + st * L::kTileBytes;
                     if (lane == 0) {
-#pragma unroll
-                        for (int kk = 0; kk < kBN / 16; ++kk)
-                            mma_ts(o_tmem, s_tmem + (uint32_t)kk * 8u,
-                                   smem_desc(vbuf + (uint32_t)kk * 2048u, (uint32_t)kHalfBytes, 1024),
-                                   kIdescPV, (n > 1 || kk > 0) ? 1u : 0u);
-                        mma_commit(BAR(B_KV_EMPTY + st));
-                        if (n == N) mma_commit(BAR(B_OFULL));
+                        const uint32_t dst = sm_base + L::kKV + st * L::kTileBytes;
+                        mbar_arrive_tx(BAR(B_KV_FULL + st), kChunkBytes);
+                        const void* tm = is_v ? (const void*)&tmap_v : (const void*)&tmap_k;
+    #pragma unroll
+                        for (int hh = 0; hh < kHalves; ++hh)
+                            tma_load_3d(dst + hh * kHalfBytes, tm, BAR(B_KV_FULL + st), hh * 64, g,
+                                        key_start + chunk * kBN);
                     }
                     __syncwarp();
                     ++c;
                 }
-                if (n < N) {
-                    // QK_n into S (after PV_{n-1} in issue order, so P_{n-1} has been read)
-                    const uint32_t st = wait_stage();
-                    if (st == ~0u) { ok = false; break; }
-                    const uint32_t kbuf = sm_base + L::kKV + st * L::kTileBytes;
-                    if (lane == 0) {
+                if (!ok) break;
+            }
+            // drain: every issued load must land before the CTA exits
+            const uint32_t issued = c;
+            for (uint32_t k = (issued > kStages ? issued - kStages : 0); k < issued; ++k)
+                drain_bar(BAR(B_KV_FULL + k % kStages), (k / kStages) & 1u);
+        } else if (warp == kWarpMMA) {
+            // ---------------- MMA issuer ----------------
+            // chunk n: [tile 0: PV_0(n-1), QK_0(n)], [tile 1: PV_1(n-1), QK_1(n)]; n = N: PVs only
+            uint32_t c = 0;                 // ring position of the current item's K(0)
+            uint32_t glob[2] = {0u, 0u};    // chunks done per tile (S / P barrier phases)
+            uint32_t uses[2] = {0u, 0u};    // items done per tile (O barrier phases)
+            bool ok = true;
+            auto wait_pos = [&](uint32_t pos) -> uint32_t {
+                const uint32_t st = pos % kStages;
+                if (!wait_bar(BAR(B_KV_FULL + st), (pos / kStages) & 1u, abort_flag, status)) return ~0u;
+                tc_fence_after();
+                return st;
+            };
+            for (int it = 0; ok; ++it) {
+                const int s = it & 1;
+                if (!wait_bar(BAR(B_INFO + s), (uint32_t)(it >> 1) & 1u, abort_flag, status)) break;
+                const ItemSlot& sl = slots[s];
+                if (sl.kind < 0) break;
+                const int N = sl.nchunks, nt = sl.ntiles;
+                if (!wait_bar(BAR(B_QFULL), (uint32_t)it & 1u, abort_flag, status)) break;
+                tc_fence_after();
+                for (int n = 0; n <= N && ok; ++n) {
+                    uint32_t kst = 0, vst = 0;
 #pragma unroll
-                        for (int kk = 0; kk < kKSteps; ++kk) {
-                            const uint32_t koff = (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32u;
-                            mma_ss(s_tmem, smem_desc(qbuf + koff, 16, 1024),
-                                   smem_desc(kbuf + koff, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+                    for (int t = 0; t < 2; ++t) {
+                        if (t >= nt) break;
+                        const uint32_t s_col = tmem + (uint32_t)(kBN * t);
+                        const uint32_t o_col = tmem + kColO + (uint32_t)(D * t);
+                        if (n > 0) {
+                            if (!wait_bar(BAR(B_PFULL + t), (glob[t] + (uint32_t)(n - 1)) & 1u, abort_flag, status) ||
+                                (n == 1 && uses[t] > 0 &&
+                                 !wait_bar(BAR(B_OEMPTY + t), (uses[t] - 1u) & 1u, abort_flag, status))) {
+                                ok = false;
+                                break;
+                            }
+                            if (t == 0 && (vst = wait_pos(c + 2u * (uint32_t)(n - 1) + 1u)) == ~0u) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            const uint32_t vbuf = sm_base + L::kKV + vst * L::kTileBytes;
+                            if (lane == 0) {
+                                // P_t from TMEM (16 keys = 8 packed columns per step), V MN-major
+    #pragma unroll
+                                for (int kk = 0; kk < kBN / 16; ++kk)
+                                    mma_ts(o_col, s_col + (uint32_t)kk * 8u,
+                                           smem_desc(vbuf + (uint32_t)kk * 2048u, (uint32_t)kHalfBytes, 1024),
+                                           kIdescPV, (n > 1 || kk > 0) ? 1u : 0u);
+                                if (t == nt - 1) mma_commit(BAR(B_KV_EMPTY + vst));
+                                if (n == N) mma_commit(BAR(B_OFULL + t));
+                            }
+                            __syncwarp();
                         }
-                        mma_commit(BAR(B_KV_EMPTY + st));
-                        mma_commit(BAR(B_SFULL));
-                        if (n == N - 1) mma_commit(BAR(B_QEMPTY));
+                        if (n < N) {
+                            // QK_t(n) into S_t (after PV_t(n-1) in issue order: P_t has been read)
+                            if (t == 0 && (kst = wait_pos(c + 2u * (uint32_t)n)) == ~0u) {
+                                ok = false;
+                                break;
+                            }
+                            const uint32_t qbuf = sm_base + L::kQ + (uint32_t)t * L::kTileBytes;
+                            const uint32_t kbuf = sm_base + L::kKV + kst * L::kTileBytes;
+                            if (lane == 0) {
+    #pragma unroll
+                                for (int kk = 0; kk < kKSteps; ++kk) {
+                                    const uint32_t koff = (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32u;
+                                    mma_ss(s_col, smem_desc(qbuf + koff, 16, 1024),
+                                           smem_desc(kbuf + koff, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+                                }
+                                mma_commit(BAR(B_SFULL + t));
+                                if (t == nt - 1) {
+                                    mma_commit(BAR(B_KV_EMPTY + kst));
+                                    if (n == N - 1) mma_commit(BAR(B_QEMPTY));
+                                }
+                            }
+                            __syncwarp();
+                        }
                     }
-                    __syncwarp();
-                    ++c;
+                }
+                c += 2u * (uint32_t)N;
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    if (t < nt) {
+                        glob[t] += (uint32_t)N;
+                        uses[t] += 1u;
+                    }
                 }
             }
-            glob += (uint32_t)N;
+            // drain the tensor pipe before TMEM is freed
+            if (lane == 0) mma_commit(BAR(B_FINAL));
+            __syncwarp();
+            drain_bar(BAR(B_FINAL), 0);
         }
-        // drain the tensor pipe before TMEM is freed
-        if (lane == 0) mma_commit(BAR(B_FINAL));
-        __syncwarp();
-        drain_bar(BAR(B_FINAL), 0);
     } else {
-        // ---------------- softmax + epilogue (warps 0-3), thread = query row ----------------
-        const int row = warp * 32 + lane;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        const uint32_t s_tmem = tmem + lane_off + kColS, o_tmem = tmem + lane_off + kColO;
-        uint32_t glob = 0;
+        // softmax: a whole row of S in registers
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+        // ---------------- softmax + epilogue of tile t, thread = query row ----------------
+        const int t = warp >> 2;
+        const int row = (warp & 3) * 32 + lane;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t s_tmem = tmem + lane_off + (uint32_t)(kBN * t);
+        const uint32_t o_tmem = tmem + lane_off + kColO + (uint32_t)(D * t);
+        uint32_t glob = 0, uses = 0;
         const float ln2 = 0.69314718055994531f;
         const float sl2 = P.scale_log2;
+        const float2 sl2x2 = make_float2(sl2, sl2);
         bool ok = true;
         for (int it = 0; ok; ++it) {
             const int s = it & 1;
             if (!wait_bar(BAR(B_INFO + s), (uint32_t)(it >> 1) & 1u, abort_flag, status)) break;
             const ItemSlot& sl = slots[s];
             if (sl.kind < 0) break;
+            if (t >= sl.ntiles) {  // this tile is idle for the item
+                mbar_arrive(BAR(B_ITEM_EMPTY + s));
+                continue;
+            }
             const int N = sl.nchunks, key_start = sl.key_start, key_end = sl.key_end;
-            const int pidx = sl.pidx[row];
+            const int pidx = sl.pidx[t * kTileM + row];
             const int tl = sl.tlim[row];
             float m = -INFINITY;  // running row maximum, log2 units
             float l = 0.f;        // running row sum of p
             for (int n = 0; n < N; ++n) {
-                const uint32_t cg = glob + (uint32_t)n;
-                if (!wait_bar(BAR(B_SFULL), cg & 1u, abort_flag, status)) {
+                if (!wait_bar(BAR(B_SFULL + t), (glob + (uint32_t)n) & 1u, abort_flag, status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                // keys past the block / after the row (current-block tiles only)
+                // keys past the block / after the row (current-block items only)
                 const int lim = min(key_end - 1, tl) - (key_start + n * kBN);
                 const bool masked = __any_sync(0xffffffffu, lim < kBN - 1);
-                // pass 1: row maximum of the raw scores
-                float mh = -INFINITY;
+                float x[kBN];
+                tmem_ld128(s_tmem, x);
+                if (masked) {
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float x[64];
-                    tmem_ld64(s_tmem + 64u * hh, x);
-                    if (masked) {
-#pragma unroll
-                        for (int j = 0; j < 64; ++j) x[j] = (64 * hh + j <= lim) ? x[j] : -INFINITY;
-                    }
-                    float mx[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) mx[j] = x[j];
-#pragma unroll
-                    for (int j = 8; j < 64; ++j) mx[j & 7] = fmaxf(mx[j & 7], x[j]);
-                    mh = fmaxf(mh, fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))));
+                    for (int j = 0; j < kBN; ++j) x[j] = (j <= lim) ? x[j] : -INFINITY;
                 }
-                const float mloc = mh * sl2;
+                // row maximum: 8 chains of three-input max over x[u + 8k]
+                float mx[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    float a = fmax3(x[u], x[u + 8], x[u + 16]);
+#pragma unroll
+                    for (int k = 3; k < 15; k += 2) a = fmax3(a, x[u + 8 * k], x[u + 8 * k + 8]);
+                    mx[u] = fmaxf(a, x[u + 120]);
+                }
+                const float mloc =
+                    fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * sl2;
+                float alpha = 1.f;
                 if (n == 0) {
                     m = mloc;
                 } else if (__any_sync(0xffffffffu, mloc > m + kRescaleThreshold)) {
-                    // S_n was committed after PV_{n-1}: O already holds every earlier PV
                     const float mn = fmaxf(m, mloc);
-                    const float alpha = ex2(m - mn);
+                    alpha = ex2(m - mn);
+                    m = mn;
+                }
+                // p = 2^(s * scale * log2(e) - m), two lanes per FMA / add; bf16 pairs over the
+                // first 64 S columns (every score is already in registers)
+                const float2 negm = make_float2(-m, -m);
+                float2 acc[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) acc[u] = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t w[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int j = 64 * hh + 2 * e;
+                        const float2 tt = __ffma2_rn(make_float2(x[j], x[j + 1]), sl2x2, negm);
+                        const float2 pr = make_float2(ex2(tt.x), ex2(tt.y));
+                        acc[e & 3] = __fadd2_rn(acc[e & 3], pr);
+                        w[e] = pack_bf16(pr.x, pr.y);
+                    }
+                    tmem_st32(s_tmem + 32u * hh, w);
+                }
+                const float2 a03 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+                if (n > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
+                    // no MMA touches O_t between the barriers of S_t(n) and P_t(n)
 #pragma unroll
                     for (int j = 0; j < D / 32; ++j) {
                         float v[32];
@@ -405,40 +462,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                         for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(v[e] * alpha);
                         tmem_st32(o_tmem + 32u * j, w);
                     }
-                    tmem_st_wait();
-                    l *= alpha;
-                    m = mn;
                 }
-                // pass 2: p = 2^(s * scale * log2(e) - m) as bf16 pairs over the read S columns
-                const float negm = -m;
-                float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float x[64];
-                    tmem_ld64(s_tmem + 64u * hh, x);
-                    if (masked) {
-#pragma unroll
-                        for (int j = 0; j < 64; ++j) x[j] = (64 * hh + j <= lim) ? x[j] : -INFINITY;
-                    }
-                    uint32_t w[32];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float p0 = ex2(fmaf(x[2 * e], sl2, negm));
-                        const float p1 = ex2(fmaf(x[2 * e + 1], sl2, negm));
-                        rs0 += p0;
-                        rs1 += p1;
-                        w[e] = pack_bf16(p0, p1);
-                    }
-                    tmem_st32(s_tmem + 32u * hh, w);
-                }
-                l += rs0 + rs1;
+                l = fmaf(l, alpha, a03.x + a03.y);
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(BAR(B_PFULL));
+                mbar_arrive(BAR(B_PFULL + t));
             }
             if (!ok) break;
-            // epilogue: O after the last PV, normalise, write the partial (o, lse)
-            if (!wait_bar(BAR(B_OFULL), (uint32_t)it & 1u, abort_flag, status)) break;
+            // epilogue: O_t after its last PV, normalise, write the partial (o, lse)
+            if (!wait_bar(BAR(B_OFULL + t), uses & 1u, abort_flag, status)) break;
             tc_fence_after();
             const float inv = 1.f / l;
             // Rows are 512-byte partial-output records at scattered addresses.  A thread owns a
@@ -468,9 +500,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
             }
             if (pidx >= 0) ws.part_lse[pidx] = m * ln2 + logf(l);
             tc_fence_before();
-            mbar_arrive(BAR(B_OEMPTY));
+            mbar_arrive(BAR(B_OEMPTY + t));
             mbar_arrive(BAR(B_ITEM_EMPTY + s));
             glob += (uint32_t)N;
+            ++uses;
         }
     }
 
@@ -482,7 +515,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
     }
 }
 
-// ---------------------------------------------------------------------------------------
 // Host side: tensor maps through the driver entry point (no libcuda link dependency)
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -529,7 +561,7 @@ cudaError_t launch_tc_d(const Problem& P, const __nv_bfloat16* q, const __nv_bfl
     const int smem = SmemLayout<D>::kBytes;
     e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_tc_kernel<D><<<num_sms * kCtasPerSm, kThreads, smem, st>>>(mk, mv, q, P, ws, t0, t1);
+    attn_tc_kernel<D><<<num_sms, kThreads, smem, st>>>(mk, mv, q, P, ws, t0, t1);
     return cudaGetLastError();
 }
 

@@ -7,8 +7,9 @@
 
 namespace moba {
 
-// Rows of a routed tile / query tile of the current block.
+// Rows of a query tile (one tensor-core M tile); an attention work item holds up to two.
 constexpr int kTileM = 128;
+constexpr int kItemRows = 2 * kTileM;
 
 // Device-side header at the start of the workspace.
 struct WsHeader {
@@ -20,9 +21,12 @@ struct WsHeader {
     int pad[11];
 };
 
-// One unit of attention work.
-//   kind 0 (history tile): a = list id (g * nb_cap + block), b = first entry, c = rows
-//   kind 1 (current-block tile): a = block, b = query head, c = query tile index
+// One unit of attention work: up to two 128-row query tiles against one KV range of one KV
+// head, so that every K/V chunk loaded serves both tiles.
+//   kind 0 (history): a = list id (g * nb_cap + block), b = first entry, c = rows (<= 256;
+//          rows 0-127 form tile 0, rows 128-255 tile 1)
+//   kind 1 (current block, one head):  a = block, b = query head h, c = query tile index
+//   kind 2 (current block, two heads): as kind 1 for heads h and h + 1 (same KV head)
 struct WorkItem {
     int a, b, c, kind;
 };

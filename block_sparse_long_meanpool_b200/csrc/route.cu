@@ -5,8 +5,9 @@
 // current block separately with a causal mask.  Here, per wave of query tokens [t0, t1):
 //
 //   route_count    histogram of routed rows per (KV head g, global block b)
-//   route_plan     exclusive scan -> list offsets; work items: the history tiles (<= 128 rows
-//                  of one list each), then the current-block tiles, largest first
+//   route_plan     exclusive scan -> list offsets; work items: the history items (<= 256 rows
+//                  of one list each), then the current-block items (one 128-token query tile
+//                  for one head, or for two heads of the same KV head), largest first
 //   route_scatter  writes each routed row's partial-output index into its list
 //
 // A routed entry is the row's partial-output index ((t - t0) * Hq + h) * topk + slot, where
@@ -197,12 +198,12 @@ route_plan_kernel(Problem P, Workspace ws, int t0, int t1) {
         carry += tot;
     }
     if (threadIdx.x == 0) ws.offsets[n_lists] = carry;
-    // 2. history tiles, list by list
+    // 2. history items (up to two tiles of routed rows), list by list
     int tcarry = 0;
     for (int base = 0; base < n_lists; base += kPlanThreads) {
         const int L = base + threadIdx.x;
         const int cnt = (L < n_lists) ? ws.counts[L] : 0;
-        const int nt = (cnt + kTileM - 1) / kTileM;
+        const int nt = (cnt + kItemRows - 1) / kItemRows;
         int tot;
         const int ex = block_exclusive_scan(nt, s_warp, &tot);
         if (L < n_lists && nt > 0) {
@@ -210,8 +211,8 @@ route_plan_kernel(Problem P, Workspace ws, int t0, int t1) {
             for (int i = 0; i < nt; ++i) {
                 WorkItem it;
                 it.a = L;
-                it.b = off + i * kTileM;
-                it.c = min(kTileM, cnt - i * kTileM);
+                it.b = off + i * kItemRows;
+                it.c = min(kItemRows, cnt - i * kItemRows);
                 it.kind = 0;
                 ws.items[tcarry + ex + i] = it;
             }
@@ -219,7 +220,7 @@ route_plan_kernel(Problem P, Workspace ws, int t0, int t1) {
         tcarry += tot;
     }
     const int n_past = tcarry;
-    // 3. current-block tiles of the blocks overlapping [t0, t1), by decreasing tile index
+    // 3. current-block items of the blocks overlapping [t0, t1), by decreasing tile index
     //    (tile q has q + 1 key tiles of work)
     const int nb = ws.hdr->nb_total;
     int lo = 0, hi = nb;  // first block whose end is > t0
@@ -236,6 +237,7 @@ route_plan_kernel(Problem P, Workspace ws, int t0, int t1) {
     }
     const int b_hi = lo;
     const int levels = (P.chunk + kTileM - 1) / kTileM;
+    const int per_block = P.hkv * ((P.group + 1) / 2);  // current-block items per query tile
     int dcarry = n_past;
     for (int qt = levels - 1; qt >= 0; --qt) {
         for (int base = b_lo; base < b_hi; base += kPlanThreads) {
@@ -253,16 +255,21 @@ route_plan_kernel(Problem P, Workspace ws, int t0, int t1) {
             int tot;
             const int ex = block_exclusive_scan(has, s_warp, &tot);
             if (has) {
-                for (int h = 0; h < P.hq; ++h) {
-                    WorkItem it;
-                    it.a = b;
-                    it.b = h;
-                    it.c = qt;
-                    it.kind = 1;
-                    ws.items[dcarry + ex * P.hq + h] = it;
+                // heads of one KV head go in pairs (they read the same keys and values)
+                int k = 0;
+                for (int g = 0; g < P.hkv; ++g) {
+                    for (int j = 0; j < P.group; j += 2) {
+                        WorkItem it;
+                        it.a = b;
+                        it.b = g * P.group + j;
+                        it.c = qt;
+                        it.kind = (j + 1 < P.group) ? 2 : 1;
+                        ws.items[dcarry + ex * per_block + k] = it;
+                        ++k;
+                    }
                 }
             }
-            dcarry += tot * P.hq;
+            dcarry += tot * per_block;
         }
     }
     if (threadIdx.x == 0) {
