@@ -6,18 +6,19 @@
 //
 // Work items (from the routing pass) hold up to two 128-row query tiles against one KV range
 // of one KV head: a history item is up to 256 routed rows (any query heads of that KV head)
-// against one whole block; a current-block item is 128 consecutive tokens of one or two query
-// heads of that KV head against the causal prefix of their block.  Every K/V chunk loaded into
-// shared memory serves both tiles.  One persistent CTA per SM takes items from an atomic cursor.
+// against one whole block; a current-block item is one or two 128-token query tiles (two heads
+// of that KV head, or two tiles of one head) against the causal prefix of their block.  Every
+// K/V chunk loaded into shared memory serves both tiles (a shorter tile stops early).  One
+// persistent CTA per SM takes items from an atomic cursor.
 //
 // Warp roles (384 threads; setmaxnreg gives the softmax warps 192 registers, enough to hold a
 // whole 128-score row, and the other warpgroup 120):
 //   warps 0-3   softmax + epilogue of tile 0, thread r owns row r (TMEM lane r)
 //   warps 4-7   softmax + epilogue of tile 1
-//   warp 8      item fetch + Q gather of both tiles (cp.async into swizzled K-major tiles)
+//   warp 8      item fetch + Q gather of tile 0 (cp.async into a swizzled K-major tile)
 //   warp 9      TMEM owner and single-thread MMA issuer
 //   warp 10     K/V producer: TMA (SWIZZLE_128B, no multicast) into a 4-stage ring
-//   warp 11     idle
+//   warp 11     Q gather of tile 1
 // TMEM (512 columns): S_0, S_1 (128 each; P_t as bf16 pairs over the first 64 columns of S_t),
 // O_0, O_1 (d each).  Per 128-key chunk n the MMA warp issues, tile by tile,
 //   PV_t(n-1): O_t += P_t(n-1) V(n-1)   (TS MMA: A = P from TMEM, B = V MN-major in smem)
@@ -27,7 +28,8 @@
 // earlier PV and that no MMA touches O_t until P_t(n) is announced: the softmax may rescale O_t
 // in between.  The softmax reads its row of S once (tcgen05.ld), takes the maximum with
 // three-input max, computes p = 2^(s*scale*log2e - m) with packed two-lane FMAs and the SFU, and
-// raises the running maximum m (rescaling O_t) only when it grows by more than 2^8.
+// raises the running maximum m (rescaling O_t) only when it grows by more than 2^8.  The
+// epilogue writes the normalised partial output as bf16 (with its fp32 log-sum-exp).
 //
 // Every mbarrier wait is bounded: on expiry the kernel records MOBA_ERR_DEVICE_TIMEOUT in
 // the workspace status word, all roles leave their loops, in-flight copies and MMAs are
@@ -48,7 +50,7 @@ using namespace ptx;
 constexpr int kBN = 128;       // keys per chunk
 constexpr int kStages = 4;     // K/V ring depth (entries K0 V0 K1 V1 ...)
 constexpr int kThreads = 384;  // 12 warps
-constexpr int kWarpFetch = 8, kWarpMMA = 9, kWarpKV = 10;
+constexpr int kWarpFetch = 8, kWarpMMA = 9, kWarpKV = 10, kWarpQ1 = 11;
 constexpr int kRegsSoftmax = 192, kRegsOther = 120;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled when max grows > 2^8
 
@@ -59,9 +61,11 @@ static_assert(8 * 32 * kRegsSoftmax + 4 * 32 * kRegsOther <= 168 * kThreads,
 struct ItemSlot {
     int kind;    // -1 = no more work
     int ntiles;  // 1 or 2
-    int g, key_start, key_end, nchunks;
+    int g, key_start, key_end;
+    int nchunks;          // K/V chunks of the item (= n[0])
+    int n[2];             // chunks of each tile (n[1] <= n[0]; 0 when tile 1 is idle)
     int pidx[kItemRows];  // partial-output index of each row (-1 = no row)
-    int tlim[kTileM];     // last key a row may see (current-block items), else INT_MAX
+    int tlim[kItemRows];  // last key a row may see (current-block items), else INT_MAX
 };
 
 template <int D>
@@ -71,22 +75,22 @@ struct SmemLayout {
     static constexpr int kKV = 2 * kTileBytes;         // kStages K/V buffers
     static constexpr int kSlots = kKV + kStages * kTileBytes;
     static constexpr int kBars = kSlots + 2 * (int)sizeof(ItemSlot);
-    static constexpr int kNumBars = 24;
+    static constexpr int kNumBars = 26;
     static constexpr int kMisc = kBars + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16 + 1024;  // + slack for 1024-byte alignment
 };
 
-// One butterfly stage of an 8x8 transpose of float4 elements across the 8 lanes of a lane
-// group: lanes i and i^DIST exchange the element pairs whose index bit DIST differs from
-// their lane bit.  After stages 4, 2, 1, lane i holds a[j] = original a[i] of lane j.
+// One butterfly stage of a 4x4 transpose of uint4 elements across the 4 lanes of a lane group:
+// lanes i and i^DIST exchange the element pairs whose index bit DIST differs from their lane
+// bit.  After stages 2 and 1, lane i holds a[j] = original a[i] of lane j.
 template <int DIST>
-__device__ __forceinline__ void transpose8x8(float4 (&a)[8], int lane) {
+__device__ __forceinline__ void transpose4x4(uint4 (&a)[4], int lane) {
     const bool up = (lane & DIST) != 0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < 4; ++j) {
         if (j & DIST) continue;
-        const float4 send = up ? a[j] : a[j | DIST];
-        float4 recv;
+        const uint4 send = up ? a[j] : a[j | DIST];
+        uint4 recv;
         recv.x = __shfl_xor_sync(0xffffffffu, send.x, DIST);
         recv.y = __shfl_xor_sync(0xffffffffu, send.y, DIST);
         recv.z = __shfl_xor_sync(0xffffffffu, send.z, DIST);
@@ -119,7 +123,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
     const uint32_t sm_base = smem_u32(smem);
     const uint32_t bar0 = sm_base + L::kBars;
     auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-    constexpr int B_INFO = 0, B_ITEM_EMPTY = 2, B_QFULL = 4, B_QEMPTY = 5, B_KV_FULL = 6,
+    constexpr int B_INFO = 0, B_ITEM_EMPTY = 2, B_QFULL = 4, B_QEMPTY = 6, B_KV_FULL = 8,
                   B_KV_EMPTY = B_KV_FULL + kStages, B_SFULL = B_KV_EMPTY + kStages,
                   B_PFULL = B_SFULL + 2, B_OFULL = B_PFULL + 2, B_OEMPTY = B_OFULL + 2,
                   B_FINAL = B_OEMPTY + 2;
@@ -131,18 +135,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(BAR(B_INFO + i), 32);
-            mbar_init(BAR(B_ITEM_EMPTY + i), 2 * kTileM);
+            mbar_init(BAR(B_ITEM_EMPTY + i), 2 * kTileM + 32);  // softmax threads + warp 11
             mbar_init(BAR(B_SFULL + i), 1);
             mbar_init(BAR(B_PFULL + i), kTileM);
             mbar_init(BAR(B_OFULL + i), 1);
             mbar_init(BAR(B_OEMPTY + i), kTileM);
+            mbar_init(BAR(B_QFULL + i), 32);
+            mbar_init(BAR(B_QEMPTY + i), 1);
         }
         for (int i = 0; i < kStages; ++i) {
             mbar_init(BAR(B_KV_FULL + i), 1);
             mbar_init(BAR(B_KV_EMPTY + i), 1);
         }
-        mbar_init(BAR(B_QFULL), 32);
-        mbar_init(BAR(B_QEMPTY), 1);
         mbar_init(BAR(B_FINAL), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -156,13 +160,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Gathers the rows of tile t of an item into Q_t by cp.async (called by one whole warp);
+    // a row's partial index encodes ((token - t0) * Hq + head) * topk + slot.
+    auto gather_q = [&](const ItemSlot& sl, int t) {
+        constexpr int CK = D / 8;  // 16-byte chunks per row
+#pragma unroll 1
+        for (int rr = lane; rr < kTileM; rr += 32) {
+            const int pi = sl.pidx[t * kTileM + rr];
+            const bool valid = pi >= 0;
+            const __nv_bfloat16* src = valid ? q + ((long long)t0 * P.hq + pi / P.topk) * D : q;
+            const uint32_t rbase = sm_base + L::kQ + (uint32_t)t * L::kTileBytes + (uint32_t)rr * 128u;
+#pragma unroll
+            for (int cc = 0; cc < CK; ++cc) {
+                const uint32_t dst = rbase + (uint32_t)(cc >> 3) * kHalfBytes +
+                                     (uint32_t)(((cc & 7) ^ (rr & 7)) << 4);
+                cp_async16(dst, src + (valid ? cc * 8 : 0), valid);
+            }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        fence_proxy_async();
+    };
+
     if (warp >= 8) {
-        // loads, MMA issue (and one idle warp): few registers
+        // loads and MMA issue: few registers
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
         if (warp == kWarpFetch) {
-            // ---------------- item fetch + Q gather (both tiles) ----------------
+            // ---------------- item fetch + Q gather of tile 0 ----------------
             const int n_items = ws.hdr->n_items;
-            constexpr int CK = D / 8;  // 16-byte chunks per row
             for (int it = 0;; ++it) {
                 const int s = it & 1;
                 const uint32_t ph = (uint32_t)(it >> 1) & 1u;
@@ -178,67 +203,79 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                     break;
                 }
                 const WorkItem w = ws.items[idx];
-                int g, key_start, key_end, ntiles;
+                int g, key_start, key_end, ntiles, n0, n1;
                 if (w.kind == 0) {
                     g = w.a / P.nb_cap;
                     const int b = w.a - g * P.nb_cap;
                     key_start = ws.blk_start[b];
                     key_end = key_start + ws.blk_len[b];
                     ntiles = w.c > kTileM ? 2 : 1;
-                    for (int r = lane; r < kItemRows; r += 32)
+                    n0 = (key_end - key_start + kBN - 1) / kBN;
+                    n1 = ntiles == 2 ? n0 : 0;
+                    for (int r = lane; r < kItemRows; r += 32) {
                         sl.pidx[r] = (r < w.c) ? ws.entries[w.b + r] : -1;
-                    for (int r = lane; r < kTileM; r += 32) sl.tlim[r] = INT_MAX;
+                        sl.tlim[r] = INT_MAX;
+                    }
                 } else {
-                    const int b = w.a, h0 = w.b, qt = w.c;
-                    ntiles = w.kind == 2 ? 2 : 1;
-                    g = h0 / P.group;
+                    // tile 0 covers (head h0, query tile qt0), tile 1 (h1, qt1); qt0 >= qt1
+                    const int b = w.a;
                     key_start = ws.blk_start[b];
                     const int len = ws.blk_len[b];
-                    key_end = key_start + min((qt + 1) * kTileM, len);
-                    for (int r = lane; r < kTileM; r += 32) {
-                        const int rr = qt * kTileM + r;
-                        const int t = key_start + rr;
-                        const bool ok = rr < len && t >= t0 && t < t1;
-                        const int base = ((t - t0) * P.hq + h0) * P.topk;  // slot 0 of (t, h0)
-                        sl.pidx[r] = ok ? base : -1;
-                        sl.pidx[kTileM + r] = (ok && ntiles == 2) ? base + P.topk : -1;
-                        sl.tlim[r] = ok ? t : INT_MAX;
+                    int h0 = w.b, h1 = w.b, qt0 = w.c, qt1 = w.c;
+                    ntiles = 1;
+                    if (w.kind == 2) {
+                        h1 = h0 + 1;
+                        ntiles = 2;
+                    } else if (w.kind == 3) {
+                        qt0 = (len + kTileM - 1) / kTileM - 1 - w.c;
+                        ntiles = 2;
+                    }
+                    g = h0 / P.group;
+                    key_end = key_start + min((qt0 + 1) * kTileM, len);
+                    n0 = qt0 + 1;
+                    n1 = ntiles == 2 ? qt1 + 1 : 0;
+                    for (int r = lane; r < kItemRows; r += 32) {
+                        const int tt = r / kTileM;
+                        const int rr = (tt ? qt1 : qt0) * kTileM + (r - tt * kTileM);
+                        const int tok = key_start + rr;
+                        const bool ok = tt < ntiles && rr < len && tok >= t0 && tok < t1;
+                        sl.pidx[r] = ok ? ((tok - t0) * P.hq + (tt ? h1 : h0)) * P.topk : -1;
+                        sl.tlim[r] = ok ? tok : INT_MAX;
                     }
                 }
-                const int N = (key_end - key_start + kBN - 1) / kBN;  // >= 1
                 if (lane == 0) {
                     sl.kind = w.kind;
                     sl.ntiles = ntiles;
                     sl.g = g;
                     sl.key_start = key_start;
                     sl.key_end = key_end;
-                    sl.nchunks = N;
+                    sl.nchunks = n0;
+                    sl.n[0] = n0;
+                    sl.n[1] = n1;
                 }
                 __syncwarp();
                 mbar_arrive(BAR(B_INFO + s));
-                // the Q buffers are free once every QK^T of the previous item has completed
+                // Q_0 is free once every QK^T of tile 0 of the previous item has completed
                 if (it >= 1 && !wait_bar(BAR(B_QEMPTY), (uint32_t)(it - 1) & 1u, abort_flag, status)) break;
-                // a row's partial index encodes (token - t0) * Hq + head, times topk
-#pragma unroll 1
-                for (int r = lane; r < ntiles * kTileM; r += 32) {
-                    const int pi = sl.pidx[r];
-                    const bool valid = pi >= 0;
-                    const __nv_bfloat16* src =
-                        valid ? q + ((long long)t0 * P.hq + pi / P.topk) * D : q;
-                    const int rr = r & (kTileM - 1);
-                    const uint32_t rbase = sm_base + L::kQ + (uint32_t)(r >> 7) * L::kTileBytes +
-                                           (uint32_t)rr * 128u;
-    #pragma unroll
-                    for (int cc = 0; cc < CK; ++cc) {
-                        const uint32_t dst = rbase + (uint32_t)(cc >> 3) * kHalfBytes +
-                                             (uint32_t)(((cc & 7) ^ (rr & 7)) << 4);
-                        cp_async16(dst, src + (valid ? cc * 8 : 0), valid);
-                    }
-                }
-                asm volatile("cp.async.commit_group;" ::: "memory");
-                asm volatile("cp.async.wait_group 0;" ::: "memory");
-                fence_proxy_async();
+                gather_q(sl, 0);
                 mbar_arrive(BAR(B_QFULL));
+            }
+        } else if (warp == kWarpQ1) {
+            // ---------------- Q gather of tile 1 ----------------
+            uint32_t uses1 = 0;  // earlier items with tile 1 active
+            for (int it = 0;; ++it) {
+                const int s = it & 1;
+                if (!wait_bar(BAR(B_INFO + s), (uint32_t)(it >> 1) & 1u, abort_flag, status)) break;
+                const ItemSlot& sl = slots[s];
+                if (sl.kind < 0) break;
+                if (sl.ntiles == 2) {
+                    if (uses1 >= 1 && !wait_bar(BAR(B_QEMPTY + 1), (uses1 - 1u) & 1u, abort_flag, status)) break;
+                    gather_q(sl, 1);
+                    mbar_arrive(BAR(B_QFULL + 1));
+                    ++uses1;
+                }
+                // the slot may be reused only after this warp is done with it
+                mbar_arrive(BAR(B_ITEM_EMPTY + s));
             }
         } else if (warp == kWarpKV) {
             // ---------------- K/V producer (TMA), in ring order K0 V0 K1 V1 ... ----------------
@@ -279,10 +316,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                 drain_bar(BAR(B_KV_FULL + k % kStages), (k / kStages) & 1u);
         } else if (warp == kWarpMMA) {
             // ---------------- MMA issuer ----------------
-            // chunk n: [tile 0: PV_0(n-1), QK_0(n)], [tile 1: PV_1(n-1), QK_1(n)]; n = N: PVs only
-            uint32_t c = 0;                 // ring position of the current item's K(0)
-            uint32_t glob[2] = {0u, 0u};    // chunks done per tile (S / P barrier phases)
-            uint32_t uses[2] = {0u, 0u};    // items done per tile (O barrier phases)
+            // chunk n: [tile 0: PV_0(n-1), QK_0(n)], [tile 1: PV_1(n-1), QK_1(n)]; tile t stops
+            // after its n_t chunks (n_1 <= n_0); n = n_0: PVs only
+            uint32_t c = 0;               // ring position of the current item's K(0)
+            uint32_t glob[2] = {0u, 0u};  // chunks done per tile (S / P barrier phases)
+            uint32_t uses[2] = {0u, 0u};  // items done per tile (Q / O barrier phases)
             bool ok = true;
             auto wait_pos = [&](uint32_t pos) -> uint32_t {
                 const uint32_t st = pos % kStages;
@@ -296,23 +334,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                 const ItemSlot& sl = slots[s];
                 if (sl.kind < 0) break;
                 const int N = sl.nchunks, nt = sl.ntiles;
-                if (!wait_bar(BAR(B_QFULL), (uint32_t)it & 1u, abort_flag, status)) break;
-                tc_fence_after();
+                const int nn[2] = {sl.n[0], nt == 2 ? sl.n[1] : 0};
                 for (int n = 0; n <= N && ok; ++n) {
-                    uint32_t kst = 0, vst = 0;
+                    uint32_t kst = ~0u, vst = ~0u;
+                    // the last tile to use K(n) / V(n-1) releases its ring stage
+                    const int last_qk = (n < nn[1]) ? 1 : 0;
+                    const int last_pv = (n - 1 < nn[1]) ? 1 : 0;
 #pragma unroll
                     for (int t = 0; t < 2; ++t) {
-                        if (t >= nt) break;
+                        const int Nt = nn[t];
                         const uint32_t s_col = tmem + (uint32_t)(kBN * t);
                         const uint32_t o_col = tmem + kColO + (uint32_t)(D * t);
-                        if (n > 0) {
+                        if (n > 0 && n <= Nt) {
                             if (!wait_bar(BAR(B_PFULL + t), (glob[t] + (uint32_t)(n - 1)) & 1u, abort_flag, status) ||
                                 (n == 1 && uses[t] > 0 &&
                                  !wait_bar(BAR(B_OEMPTY + t), (uses[t] - 1u) & 1u, abort_flag, status))) {
                                 ok = false;
                                 break;
                             }
-                            if (t == 0 && (vst = wait_pos(c + 2u * (uint32_t)(n - 1) + 1u)) == ~0u) {
+                            if (vst == ~0u && (vst = wait_pos(c + 2u * (uint32_t)(n - 1) + 1u)) == ~0u) {
                                 ok = false;
                                 break;
                             }
@@ -320,36 +360,39 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                             const uint32_t vbuf = sm_base + L::kKV + vst * L::kTileBytes;
                             if (lane == 0) {
                                 // P_t from TMEM (16 keys = 8 packed columns per step), V MN-major
-    #pragma unroll
+#pragma unroll
                                 for (int kk = 0; kk < kBN / 16; ++kk)
                                     mma_ts(o_col, s_col + (uint32_t)kk * 8u,
                                            smem_desc(vbuf + (uint32_t)kk * 2048u, (uint32_t)kHalfBytes, 1024),
                                            kIdescPV, (n > 1 || kk > 0) ? 1u : 0u);
-                                if (t == nt - 1) mma_commit(BAR(B_KV_EMPTY + vst));
-                                if (n == N) mma_commit(BAR(B_OFULL + t));
+                                if (t == last_pv) mma_commit(BAR(B_KV_EMPTY + vst));
+                                if (n == Nt) mma_commit(BAR(B_OFULL + t));
                             }
                             __syncwarp();
                         }
-                        if (n < N) {
+                        if (n < Nt) {
                             // QK_t(n) into S_t (after PV_t(n-1) in issue order: P_t has been read)
-                            if (t == 0 && (kst = wait_pos(c + 2u * (uint32_t)n)) == ~0u) {
+                            if (n == 0 && !wait_bar(BAR(B_QFULL + t), uses[t] & 1u, abort_flag, status)) {
                                 ok = false;
                                 break;
                             }
+                            if (kst == ~0u && (kst = wait_pos(c + 2u * (uint32_t)n)) == ~0u) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
                             const uint32_t qbuf = sm_base + L::kQ + (uint32_t)t * L::kTileBytes;
                             const uint32_t kbuf = sm_base + L::kKV + kst * L::kTileBytes;
                             if (lane == 0) {
-    #pragma unroll
+#pragma unroll
                                 for (int kk = 0; kk < kKSteps; ++kk) {
                                     const uint32_t koff = (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32u;
                                     mma_ss(s_col, smem_desc(qbuf + koff, 16, 1024),
                                            smem_desc(kbuf + koff, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
                                 }
                                 mma_commit(BAR(B_SFULL + t));
-                                if (t == nt - 1) {
-                                    mma_commit(BAR(B_KV_EMPTY + kst));
-                                    if (n == N - 1) mma_commit(BAR(B_QEMPTY));
-                                }
+                                if (t == last_qk) mma_commit(BAR(B_KV_EMPTY + kst));
+                                if (n == Nt - 1) mma_commit(BAR(B_QEMPTY + t));
                             }
                             __syncwarp();
                         }
@@ -358,8 +401,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                 c += 2u * (uint32_t)N;
 #pragma unroll
                 for (int t = 0; t < 2; ++t) {
-                    if (t < nt) {
-                        glob[t] += (uint32_t)N;
+                    if (nn[t] > 0) {
+                        glob[t] += (uint32_t)nn[t];
                         uses[t] += 1u;
                     }
                 }
@@ -392,9 +435,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                 mbar_arrive(BAR(B_ITEM_EMPTY + s));
                 continue;
             }
-            const int N = sl.nchunks, key_start = sl.key_start, key_end = sl.key_end;
+            const int N = sl.n[t], key_start = sl.key_start, key_end = sl.key_end;
             const int pidx = sl.pidx[t * kTileM + row];
-            const int tl = sl.tlim[row];
+            const int tl = sl.tlim[t * kTileM + row];
             float m = -INFINITY;  // running row maximum, log2 units
             float l = 0.f;        // running row sum of p
             for (int n = 0; n < N; ++n) {
@@ -473,30 +516,31 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
             if (!wait_bar(BAR(B_OFULL + t), uses & 1u, abort_flag, status)) break;
             tc_fence_after();
             const float inv = 1.f / l;
-            // Rows are 512-byte partial-output records at scattered addresses.  A thread owns a
-            // row, so storing straight from registers would touch 32 cache lines per warp
-            // store.  Instead each group of 8 lanes transposes 8x8 blocks of float4 by shuffles
-            // and every store instruction writes 128 contiguous bytes of 4 rows.
-            int prow[8];
+            // Rows are 2d-byte bf16 partial-output records at scattered addresses.  A thread owns
+            // a row, so storing straight from registers would touch 32 rows per warp store.
+            // Instead each group of 4 lanes transposes 4x4 blocks of 16-byte pieces by shuffles
+            // and every store instruction writes 64 contiguous bytes of each of 8 rows.
+            int prow[4];
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) prow[jj] = __shfl_sync(0xffffffffu, pidx, (lane & ~7) + jj);
-            const int seg = lane & 7;
+            for (int jj = 0; jj < 4; ++jj) prow[jj] = __shfl_sync(0xffffffffu, pidx, (lane & ~3) + jj);
+            const int sub = lane & 3;
 #pragma unroll
             for (int j = 0; j < D / 32; ++j) {
                 float v[32];
                 tmem_ld32(o_tmem + 32u * j, v);
-                float4 a[8];
+                uint4 a[4];
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    a[e] = make_float4(v[4 * e] * inv, v[4 * e + 1] * inv, v[4 * e + 2] * inv,
-                                       v[4 * e + 3] * inv);
-                transpose8x8<4>(a, lane);
-                transpose8x8<2>(a, lane);
-                transpose8x8<1>(a, lane);
+                for (int e = 0; e < 4; ++e)
+                    a[e] = make_uint4(pack_bf16(v[8 * e] * inv, v[8 * e + 1] * inv),
+                                      pack_bf16(v[8 * e + 2] * inv, v[8 * e + 3] * inv),
+                                      pack_bf16(v[8 * e + 4] * inv, v[8 * e + 5] * inv),
+                                      pack_bf16(v[8 * e + 6] * inv, v[8 * e + 7] * inv));
+                transpose4x4<2>(a, lane);
+                transpose4x4<1>(a, lane);
 #pragma unroll
-                for (int jj = 0; jj < 8; ++jj)
+                for (int jj = 0; jj < 4; ++jj)
                     if (prow[jj] >= 0)
-                        *reinterpret_cast<float4*>(ws.part_o + (size_t)prow[jj] * D + 32 * j + 4 * seg) = a[jj];
+                        *reinterpret_cast<uint4*>(ws.part_o + (size_t)prow[jj] * D + 32 * j + 8 * sub) = a[jj];
             }
             if (pidx >= 0) ws.part_lse[pidx] = m * ln2 + logf(l);
             tc_fence_before();

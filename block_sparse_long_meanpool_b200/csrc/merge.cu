@@ -5,6 +5,8 @@
 // online-softmax rule.  For partials (o_i, lse_i), i = 0 .. n-1 (slot 0 = own block):
 //   m = max_i lse_i,  w_i = exp(lse_i - m),  o = sum_i w_i o_i / sum_i w_i,
 //   lse = m + log(sum_i w_i).
+// The partial outputs o_i are bf16 (the precision an attention call returns its output in),
+// the lse_i fp32; the combination is computed in fp32.
 // A half-warp per query row (two rows per warp): the first partial rows are loaded before the
 // weights are known, lane s reads slot s's lse (and s + 16), the maximum and the weights come
 // from half-warp reductions, and each lane accumulates d/16 consecutive channels with four
@@ -17,6 +19,28 @@ namespace moba {
 namespace {
 
 constexpr int kWarps = 8;
+
+// V consecutive bf16 channels of one partial row (streaming load), widened to fp32; zeros
+// when the slot is unused.
+template <int V>
+__device__ __forceinline__ void load_row(const __nv_bfloat16* p, bool valid, float (&x)[V]) {
+    uint32_t w[V / 2];
+    if constexpr (V == 8) {
+        uint4 y = make_uint4(0u, 0u, 0u, 0u);
+        if (valid) y = __ldcs(reinterpret_cast<const uint4*>(p));
+        w[0] = y.x; w[1] = y.y; w[2] = y.z; w[3] = y.w;
+    } else {
+        uint2 y = make_uint2(0u, 0u);
+        if (valid) y = __ldcs(reinterpret_cast<const uint2*>(p));
+        w[0] = y.x; w[1] = y.y;
+    }
+#pragma unroll
+    for (int e = 0; e < V / 2; ++e) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+        x[2 * e] = f.x;
+        x[2 * e + 1] = f.y;
+    }
+}
 
 template <int D>
 __global__ void __launch_bounds__(kWarps * 32)
@@ -34,18 +58,11 @@ merge_kernel(const int* __restrict__ cu, const int* __restrict__ sel, Problem P,
         const bool valid = r < n;
         const int ns = valid ? (int)ws.nslots[r] : 0;  // own block + routed history blocks
         const size_t pbase = (size_t)(valid ? r : 0) * P.topk;
-        const float* obase = ws.part_o + pbase * D + hl * V;
+        const __nv_bfloat16* obase = ws.part_o + pbase * D + hl * V;
         // first partial rows in flight before the weights are known
         float x[kUnroll][V];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-#pragma unroll
-            for (int e = 0; e < V; e += 4) {
-                float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (u < ns) y = __ldcs(reinterpret_cast<const float4*>(obase + (size_t)u * D + e));
-                x[u][e] = y.x; x[u][e + 1] = y.y; x[u][e + 2] = y.z; x[u][e + 3] = y.w;
-            }
-        }
+        for (int u = 0; u < kUnroll; ++u) load_row<V>(obase + (size_t)u * D, u < ns, x[u]);
         // slot lse: lane hl holds slots hl and hl + 16; max and weights by half-warp reductions
         const float la = (hl < ns) ? __ldcs(ws.part_lse + pbase + hl) : -INFINITY;
         const float lb = (hl + 16 < ns) ? __ldcs(ws.part_lse + pbase + hl + 16) : -INFINITY;
@@ -70,15 +87,7 @@ merge_kernel(const int* __restrict__ cu, const int* __restrict__ sel, Problem P,
         const int ns_max = max(__shfl_sync(full, ns, 0), __shfl_sync(full, ns, 16));
         for (int s0 = kUnroll; s0 < ns_max; s0 += kUnroll) {
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-#pragma unroll
-                for (int e = 0; e < V; e += 4) {
-                    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (s0 + u < ns)
-                        y = __ldcs(reinterpret_cast<const float4*>(obase + (size_t)(s0 + u) * D + e));
-                    x[u][e] = y.x; x[u][e + 1] = y.y; x[u][e + 2] = y.z; x[u][e + 3] = y.w;
-                }
-            }
+            for (int u = 0; u < kUnroll; ++u) load_row<V>(obase + (size_t)(s0 + u) * D, s0 + u < ns, x[u]);
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u) {
                 const int sl = s0 + u;  // < 32

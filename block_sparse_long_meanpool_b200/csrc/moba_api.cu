@@ -110,7 +110,7 @@ Layout make_layout(const moba_params& p) {
     L.cursor = take(4ull * lists);
     L.entries = take(4ull * routed);
     L.items = take(sizeof(WorkItem) * L.max_items);
-    L.part_o = take(4ull * W * p.num_q_heads * p.topk * p.head_dim);
+    L.part_o = take(2ull * W * p.num_q_heads * p.topk * p.head_dim);  // bf16
     L.part_lse = take(4ull * W * p.num_q_heads * p.topk);
     L.nslots = take(1ull * W * p.num_q_heads);
     L.total = o;
@@ -243,7 +243,7 @@ moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, co
     ws.cursor = reinterpret_cast<int*>(base + L.cursor);
     ws.entries = reinterpret_cast<int*>(base + L.entries);
     ws.items = reinterpret_cast<WorkItem*>(base + L.items);
-    ws.part_o = reinterpret_cast<float*>(base + L.part_o);
+    ws.part_o = reinterpret_cast<__nv_bfloat16*>(base + L.part_o);
     ws.part_lse = reinterpret_cast<float*>(base + L.part_lse);
     ws.nslots = reinterpret_cast<unsigned char*>(base + L.nslots);
 

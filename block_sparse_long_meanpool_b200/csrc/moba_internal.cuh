@@ -27,6 +27,8 @@ struct WsHeader {
 //          rows 0-127 form tile 0, rows 128-255 tile 1)
 //   kind 1 (current block, one head):  a = block, b = query head h, c = query tile index
 //   kind 2 (current block, two heads): as kind 1 for heads h and h + 1 (same KV head)
+//   kind 3 (current block, two query tiles of one head): a = block, b = head h, c = tile p;
+//          the other tile is lv - 1 - p (lv = query tiles of the block), which comes first
 struct WorkItem {
     int a, b, c, kind;
 };
@@ -55,7 +57,7 @@ struct Workspace {
     int* cursor;      // [hkv * nb_cap]
     int* entries;     // [wave * hq * (topk - 1)]
     WorkItem* items;  // [max_items]
-    float* part_o;    // [wave * hq * topk, d]
+    __nv_bfloat16* part_o;  // [wave * hq * topk, d]: normalised partial outputs
     float* part_lse;  // [wave * hq * topk]
     unsigned char* nslots;  // [wave * hq]: 1 + routed history blocks of each row
 };

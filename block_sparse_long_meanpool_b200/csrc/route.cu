@@ -237,39 +237,80 @@ route_plan_kernel(Problem P, Workspace ws, int t0, int t1) {
     }
     const int b_hi = lo;
     const int levels = (P.chunk + kTileM - 1) / kTileM;
-    const int per_block = P.hkv * ((P.group + 1) / 2);  // current-block items per query tile
+    // does query tile qt of block b (a block of length len) hold a token of [t0, t1)?
+    auto overlaps = [&](int b, int len, int qt) {
+        const int r0 = qt * kTileM;
+        if (r0 >= len) return false;
+        const int a = ws.blk_start[b] + r0;
+        const int e = ws.blk_start[b] + min(r0 + kTileM, len);
+        return a < t1 && e > t0;
+    };
     int dcarry = n_past;
-    for (int qt = levels - 1; qt >= 0; --qt) {
-        for (int base = b_lo; base < b_hi; base += kPlanThreads) {
-            const int b = base + threadIdx.x;
-            int has = 0;
-            if (b < b_hi) {
-                const int r0 = qt * kTileM;
-                const int len = ws.blk_len[b];
-                if (r0 < len) {
-                    const int a = ws.blk_start[b] + r0;
-                    const int e = ws.blk_start[b] + min(r0 + kTileM, len);
-                    has = (a < t1 && e > t0) ? 1 : 0;
-                }
-            }
-            int tot;
-            const int ex = block_exclusive_scan(has, s_warp, &tot);
-            if (has) {
-                // heads of one KV head go in pairs (they read the same keys and values)
-                int k = 0;
-                for (int g = 0; g < P.hkv; ++g) {
-                    for (int j = 0; j < P.group; j += 2) {
-                        WorkItem it;
-                        it.a = b;
-                        it.b = g * P.group + j;
-                        it.c = qt;
-                        it.kind = (j + 1 < P.group) ? 2 : 1;
-                        ws.items[dcarry + ex * per_block + k] = it;
-                        ++k;
+    if (P.group > 1) {
+        // heads of one KV head go in pairs (same keys and values); largest query tile first
+        // (tile qt has qt + 1 key chunks of work)
+        const int per_block = P.hkv * ((P.group + 1) / 2);  // items per query tile
+        for (int qt = levels - 1; qt >= 0; --qt) {
+            for (int base = b_lo; base < b_hi; base += kPlanThreads) {
+                const int b = base + threadIdx.x;
+                const int has = (b < b_hi && overlaps(b, ws.blk_len[b], qt)) ? 1 : 0;
+                int tot;
+                const int ex = block_exclusive_scan(has, s_warp, &tot);
+                if (has) {
+                    int k = 0;
+                    for (int g = 0; g < P.hkv; ++g) {
+                        for (int j = 0; j < P.group; j += 2) {
+                            WorkItem it;
+                            it.a = b;
+                            it.b = g * P.group + j;
+                            it.c = qt;
+                            it.kind = (j + 1 < P.group) ? 2 : 1;
+                            ws.items[dcarry + ex * per_block + k] = it;
+                            ++k;
+                        }
                     }
                 }
+                dcarry += tot * per_block;
             }
-            dcarry += tot * per_block;
+        }
+    } else {
+        // one query head per KV head: query tiles lv-1-p and p of the same head and block go
+        // together (same keys and values; every pair spans lv + 1 key chunks)
+        for (int p = 0; p < (levels + 1) / 2; ++p) {
+            for (int base = b_lo; base < b_hi; base += kPlanThreads) {
+                const int b = base + threadIdx.x;
+                int kind = -1, qt = 0;
+                if (b < b_hi) {
+                    const int len = ws.blk_len[b];
+                    const int lv = (len + kTileM - 1) / kTileM;
+                    if (p < (lv + 1) / 2) {
+                        const int qa = lv - 1 - p;
+                        const bool ha = overlaps(b, len, qa);
+                        const bool hb = p != qa && overlaps(b, len, p);
+                        if (ha && hb) {
+                            kind = 3;
+                            qt = p;
+                        } else if (ha || hb) {
+                            kind = 1;
+                            qt = ha ? qa : p;
+                        }
+                    }
+                }
+                const int has = kind >= 0 ? 1 : 0;
+                int tot;
+                const int ex = block_exclusive_scan(has, s_warp, &tot);
+                if (has) {
+                    for (int h = 0; h < P.hq; ++h) {
+                        WorkItem it;
+                        it.a = b;
+                        it.b = h;
+                        it.c = qt;
+                        it.kind = kind;
+                        ws.items[dcarry + ex * P.hq + h] = it;
+                    }
+                }
+                dcarry += tot * P.hq;
+            }
         }
     }
     if (threadIdx.x == 0) {

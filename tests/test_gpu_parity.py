@@ -38,6 +38,10 @@ SMALL = [
     W.custom("topk32", [4500], 2, 1, 128, 128, 32, "k_offsets", 15),
     # one block longer than the sequence
     W.custom("single_block", [300, 77], 2, 1, 128, 512, 3, "k_offsets", 16),
+    # odd GQA group (3 query heads per KV head): paired and single heads in current-block work
+    W.custom("odd_group", [1500, 900], 6, 2, 128, 384, 3, "k_offsets", 17),
+    # MHA with 3 query tiles per block and partial blocks: paired and single query tiles
+    W.custom("mha_odd_tiles", [1000, 1700], 3, 3, 64, 384, 3, "qk_offsets", 18),
 ]
 
 
