@@ -300,7 +300,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                         const uint32_t dst = sm_base + L::kKV + st * L::kTileBytes;
                         mbar_arrive_tx(BAR(B_KV_FULL + st), kChunkBytes);
                         const void* tm = is_v ? (const void*)&tmap_v : (const void*)&tmap_k;
-    #pragma unroll
+#pragma unroll
                         for (int hh = 0; hh < kHalves; ++hh)
                             tma_load_3d(dst + hh * kHalfBytes, tm, BAR(B_KV_FULL + st), hh * 64, g,
                                         key_start + chunk * kBN);
@@ -322,6 +322,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
             uint32_t glob[2] = {0u, 0u};  // chunks done per tile (S / P barrier phases)
             uint32_t uses[2] = {0u, 0u};  // items done per tile (Q / O barrier phases)
             bool ok = true;
+            // Shared-memory matrix descriptors: one base per operand form; an operand's descriptor
+            // is the base plus its byte offset / 16 (shared addresses stay below 2^18 bytes, so the
+            // 14-bit start-address field never carries).  Keeps the single issuing thread's
+            // instruction stream short: each MMA is one add per operand plus the MMA itself.
+            const uint64_t desc_kmaj = smem_desc(sm_base, 16, 1024);                     // Q, K
+            const uint64_t desc_mnmaj = smem_desc(sm_base, (uint32_t)kHalfBytes, 1024);  // V
             auto wait_pos = [&](uint32_t pos) -> uint32_t {
                 const uint32_t st = pos % kStages;
                 if (!wait_bar(BAR(B_KV_FULL + st), (pos / kStages) & 1u, abort_flag, status)) return ~0u;
@@ -357,14 +363,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                                 break;
                             }
                             tc_fence_after();
-                            const uint32_t vbuf = sm_base + L::kKV + vst * L::kTileBytes;
+                            const uint64_t vdesc = desc_mnmaj + ((uint32_t)(L::kKV + vst * L::kTileBytes) >> 4);
                             if (lane == 0) {
                                 // P_t from TMEM (16 keys = 8 packed columns per step), V MN-major
+                                // (16 keys = 2048 bytes per step)
+                                mma_ts(o_col, s_col, vdesc, kIdescPV, n > 1 ? 1u : 0u);
 #pragma unroll
-                                for (int kk = 0; kk < kBN / 16; ++kk)
-                                    mma_ts(o_col, s_col + (uint32_t)kk * 8u,
-                                           smem_desc(vbuf + (uint32_t)kk * 2048u, (uint32_t)kHalfBytes, 1024),
-                                           kIdescPV, (n > 1 || kk > 0) ? 1u : 0u);
+                                for (int kk = 1; kk < kBN / 16; ++kk)
+                                    mma_ts(o_col, s_col + (uint32_t)kk * 8u, vdesc + (uint64_t)(kk * 128), kIdescPV, 1u);
                                 if (t == last_pv) mma_commit(BAR(B_KV_EMPTY + vst));
                                 if (n == Nt) mma_commit(BAR(B_OFULL + t));
                             }
@@ -381,14 +387,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                                 break;
                             }
                             tc_fence_after();
-                            const uint32_t qbuf = sm_base + L::kQ + (uint32_t)t * L::kTileBytes;
-                            const uint32_t kbuf = sm_base + L::kKV + kst * L::kTileBytes;
+                            const uint64_t qdesc = desc_kmaj + ((uint32_t)(L::kQ + t * L::kTileBytes) >> 4);
+                            const uint64_t kdesc = desc_kmaj + ((uint32_t)(L::kKV + kst * L::kTileBytes) >> 4);
                             if (lane == 0) {
+                                // 16 d-columns per step: 32 bytes inside a 128-byte swizzle row, then
+                                // the next [128 x 64] half
 #pragma unroll
                                 for (int kk = 0; kk < kKSteps; ++kk) {
-                                    const uint32_t koff = (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32u;
-                                    mma_ss(s_col, smem_desc(qbuf + koff, 16, 1024),
-                                           smem_desc(kbuf + koff, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+                                    const uint64_t koff = (uint64_t)((kk >> 2) * (kHalfBytes >> 4) + (kk & 3) * 2);
+                                    mma_ss(s_col, qdesc + koff, kdesc + koff, kIdescQK, kk > 0 ? 1u : 0u);
                                 }
                                 mma_commit(BAR(B_SFULL + t));
                                 if (t == last_qk) mma_commit(BAR(B_KV_EMPTY + kst));
