@@ -17,13 +17,16 @@
 //   warps 4-7   softmax + epilogue of tile 1
 //   warp 8      item fetch + Q gather of tile 0 (cp.async into a swizzled K-major tile)
 //   warp 9      TMEM owner and single-thread MMA issuer
-//   warp 10     K/V producer: TMA (SWIZZLE_128B, no multicast) into a 4-stage ring
+//   warp 10     K/V producer: TMA (SWIZZLE_128B, no multicast) into a 2-slot ring
 //   warp 11     Q gather of tile 1
 // TMEM (512 columns): S_0, S_1 (128 each; P_t as bf16 pairs over the first 64 columns of S_t),
 // O_0, O_1 (d each).  Per 128-key chunk n the MMA warp issues, tile by tile,
 //   PV_t(n-1): O_t += P_t(n-1) V(n-1)   (TS MMA: A = P from TMEM, B = V MN-major in smem)
 //   QK_t(n):   S_t  = Q_t K(n)^T        (SS MMA, fp32 accumulate)
-// so the tensor core works on one tile while the other tile's softmax runs.  PV_t(n-1) is
+// so the tensor core works on one tile while the other tile's softmax runs.  Each tile's
+// PV_t(n-1) and QK_t(n) go out as one uninterrupted run of MMAs with every wait hoisted in
+// front of it: the tensor pipe drains whenever the issuing thread stops issuing, so the waits
+// and commits between runs are kept to three each per chunk.  PV_t(n-1) is
 // issued before QK_t(n), so the barrier announcing S_t(n) also guarantees that O_t holds every
 // earlier PV and that no MMA touches O_t until P_t(n) is announced: the softmax may rescale O_t
 // in between.  The softmax reads its row of S once (tcgen05.ld), takes the maximum with
@@ -48,7 +51,7 @@ namespace {
 using namespace ptx;
 
 constexpr int kBN = 128;       // keys per chunk
-constexpr int kStages = 4;     // K/V ring depth (entries K0 V0 K1 V1 ...)
+constexpr int kSlots = 2;      // K/V ring: slot = K and V of one 128-key chunk, one barrier
 constexpr int kThreads = 384;  // 12 warps
 constexpr int kWarpFetch = 8, kWarpMMA = 9, kWarpKV = 10, kWarpQ1 = 11;
 constexpr int kRegsSoftmax = 192, kRegsOther = 120;
@@ -72,9 +75,9 @@ template <int D>
 struct SmemLayout {
     static constexpr int kTileBytes = kTileM * D * 2;  // 128 rows of bf16 (Q tile, K or V chunk)
     static constexpr int kQ = 0;                       // Q_0, Q_1
-    static constexpr int kKV = 2 * kTileBytes;         // kStages K/V buffers
-    static constexpr int kSlots = kKV + kStages * kTileBytes;
-    static constexpr int kBars = kSlots + 2 * (int)sizeof(ItemSlot);
+    static constexpr int kKV = 2 * kTileBytes;         // kSlots x (K chunk, V chunk)
+    static constexpr int kItems = kKV + kSlots * 2 * kTileBytes;
+    static constexpr int kBars = kItems + 2 * (int)sizeof(ItemSlot);
     static constexpr int kNumBars = 26;
     static constexpr int kMisc = kBars + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16 + 1024;  // + slack for 1024-byte alignment
@@ -116,7 +119,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    ItemSlot* slots = reinterpret_cast<ItemSlot*>(smem + L::kSlots);
+    ItemSlot* slots = reinterpret_cast<ItemSlot*>(smem + L::kItems);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
@@ -124,7 +127,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
     const uint32_t bar0 = sm_base + L::kBars;
     auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
     constexpr int B_INFO = 0, B_ITEM_EMPTY = 2, B_QFULL = 4, B_QEMPTY = 6, B_KV_FULL = 8,
-                  B_KV_EMPTY = B_KV_FULL + kStages, B_SFULL = B_KV_EMPTY + kStages,
+                  B_KV_EMPTY = B_KV_FULL + kSlots, B_SFULL = B_KV_EMPTY + kSlots,
                   B_PFULL = B_SFULL + 2, B_OFULL = B_PFULL + 2, B_OEMPTY = B_OFULL + 2,
                   B_FINAL = B_OEMPTY + 2;
     static_assert(B_FINAL < L::kNumBars, "barrier area too small");
@@ -143,7 +146,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
             mbar_init(BAR(B_QFULL + i), 32);
             mbar_init(BAR(B_QEMPTY + i), 1);
         }
-        for (int i = 0; i < kStages; ++i) {
+        for (int i = 0; i < kSlots; ++i) {
             mbar_init(BAR(B_KV_FULL + i), 1);
             mbar_init(BAR(B_KV_EMPTY + i), 1);
         }
@@ -278,8 +281,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                 mbar_arrive(BAR(B_ITEM_EMPTY + s));
             }
         } else if (warp == kWarpKV) {
-            // ---------------- K/V producer (TMA), in ring order K0 V0 K1 V1 ... ----------------
-            uint32_t c = 0;  // ring position
+            // ---------------- K/V producer (TMA): chunk c of the CTA goes to slot c % 2 ----------
+            uint32_t c = 0;  // chunks issued so far
             for (int it = 0;; ++it) {
                 const int s = it & 1;
                 if (!wait_bar(BAR(B_INFO + s), (uint32_t)(it >> 1) & 1u, abort_flag, status)) break;
@@ -287,23 +290,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                 if (sl.kind < 0) break;
                 const int g = sl.g, key_start = sl.key_start, N = sl.nchunks;
                 bool ok = true;
-                for (int j = 0; j < 2 * N; ++j) {
-                    const bool is_v = (j & 1) != 0;
-                    const int chunk = j >> 1;
-                    const uint32_t st = c % kStages;
-                    if (c >= kStages &&
-                        !wait_bar(BAR(B_KV_EMPTY + st), ((c / kStages) - 1u) & 1u, abort_flag, status)) {
+                for (int chunk = 0; chunk < N; ++chunk) {
+                    const uint32_t st = c % kSlots;
+                    if (c >= kSlots &&
+                        !wait_bar(BAR(B_KV_EMPTY + st), ((c / kSlots) - 1u) & 1u, abort_flag, status)) {
                         ok = false;
                         break;
                     }
                     if (lane == 0) {
-                        const uint32_t dst = sm_base + L::kKV + st * L::kTileBytes;
-                        mbar_arrive_tx(BAR(B_KV_FULL + st), kChunkBytes);
-                        const void* tm = is_v ? (const void*)&tmap_v : (const void*)&tmap_k;
+                        const uint32_t dst = sm_base + L::kKV + st * 2u * L::kTileBytes;
+                        mbar_arrive_tx(BAR(B_KV_FULL + st), 2u * kChunkBytes);
 #pragma unroll
-                        for (int hh = 0; hh < kHalves; ++hh)
-                            tma_load_3d(dst + hh * kHalfBytes, tm, BAR(B_KV_FULL + st), hh * 64, g,
+                        for (int hh = 0; hh < kHalves; ++hh) {
+                            tma_load_3d(dst + hh * kHalfBytes, &tmap_k, BAR(B_KV_FULL + st), hh * 64, g,
                                         key_start + chunk * kBN);
+                            tma_load_3d(dst + L::kTileBytes + hh * kHalfBytes, &tmap_v, BAR(B_KV_FULL + st),
+                                        hh * 64, g, key_start + chunk * kBN);
+                        }
                     }
                     __syncwarp();
                     ++c;
@@ -312,112 +315,104 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
             }
             // drain: every issued load must land before the CTA exits
             const uint32_t issued = c;
-            for (uint32_t k = (issued > kStages ? issued - kStages : 0); k < issued; ++k)
-                drain_bar(BAR(B_KV_FULL + k % kStages), (k / kStages) & 1u);
+            for (uint32_t k = (issued > kSlots ? issued - kSlots : 0); k < issued; ++k)
+                drain_bar(BAR(B_KV_FULL + k % kSlots), (k / kSlots) & 1u);
         } else if (warp == kWarpMMA) {
             // ---------------- MMA issuer ----------------
-            // chunk n: [tile 0: PV_0(n-1), QK_0(n)], [tile 1: PV_1(n-1), QK_1(n)]; tile t stops
-            // after its n_t chunks (n_1 <= n_0); n = n_0: PVs only
-            uint32_t c = 0;               // ring position of the current item's K(0)
-            uint32_t glob[2] = {0u, 0u};  // chunks done per tile (S / P barrier phases)
-            uint32_t uses[2] = {0u, 0u};  // items done per tile (Q / O barrier phases)
-            bool ok = true;
-            // Shared-memory matrix descriptors: one base per operand form; an operand's descriptor
-            // is the base plus its byte offset / 16 (shared addresses stay below 2^18 bytes, so the
-            // 14-bit start-address field never carries).  Keeps the single issuing thread's
-            // instruction stream short: each MMA is one add per operand plus the MMA itself.
-            const uint64_t desc_kmaj = smem_desc(sm_base, 16, 1024);                     // Q, K
-            const uint64_t desc_mnmaj = smem_desc(sm_base, (uint32_t)kHalfBytes, 1024);  // V
-            auto wait_pos = [&](uint32_t pos) -> uint32_t {
-                const uint32_t st = pos % kStages;
-                if (!wait_bar(BAR(B_KV_FULL + st), (pos / kStages) & 1u, abort_flag, status)) return ~0u;
-                tc_fence_after();
-                return st;
-            };
-            for (int it = 0; ok; ++it) {
-                const int s = it & 1;
-                if (!wait_bar(BAR(B_INFO + s), (uint32_t)(it >> 1) & 1u, abort_flag, status)) break;
-                const ItemSlot& sl = slots[s];
-                if (sl.kind < 0) break;
-                const int N = sl.nchunks, nt = sl.ntiles;
-                const int nn[2] = {sl.n[0], nt == 2 ? sl.n[1] : 0};
-                for (int n = 0; n <= N && ok; ++n) {
-                    uint32_t kst = ~0u, vst = ~0u;
-                    // the last tile to use K(n) / V(n-1) releases its ring stage
-                    const int last_qk = (n < nn[1]) ? 1 : 0;
-                    const int last_pv = (n - 1 < nn[1]) ? 1 : 0;
+            // chunk n, tile by tile: PV_t(n-1) then QK_t(n) as one run of MMAs; tile t stops
+            // after its n_t chunks (n_1 <= n_0); n = n_0: the last PVs only.  One thread runs
+            // this role (waits without warp votes, no warp syncs between runs).
+            if (lane == 0) {
+                uint32_t c = 0;               // CTA chunk index of the current item's chunk 0
+                uint32_t glob[2] = {0u, 0u};  // chunks done per tile (S / P barrier phases)
+                uint32_t uses[2] = {0u, 0u};  // items done per tile (Q / O barrier phases)
+                bool ok = true;
+                // Shared-memory matrix descriptors: one base per operand form; an operand's
+                // descriptor is the base plus its byte offset / 16 (shared addresses stay below
+                // 2^18 bytes, so the 14-bit start-address field never carries).
+                const uint64_t desc_kmaj = smem_desc(sm_base, 16, 1024);                     // Q, K
+                const uint64_t desc_mnmaj = smem_desc(sm_base, (uint32_t)kHalfBytes, 1024);  // V
+                for (int it = 0; ok; ++it) {
+                    const int s = it & 1;
+                    if (!wait_bar1(BAR(B_INFO + s), (uint32_t)(it >> 1) & 1u, abort_flag, status)) break;
+                    const ItemSlot& sl = slots[s];
+                    if (sl.kind < 0) break;
+                    const int N = sl.nchunks, nt = sl.ntiles;
+                    const int nn[2] = {sl.n[0], nt == 2 ? sl.n[1] : 0};
+                    for (int n = 0; n <= N && ok; ++n) {
+                        const uint32_t kslot = (c + (uint32_t)n) % kSlots;         // K(n)
+                        const uint32_t vslot = (c + (uint32_t)n + 1u) % kSlots;    // V(n-1)
+                        // the last tile to read V(n-1) releases its slot
+                        const int last_pv = (n - 1 < nn[1]) ? 1 : 0;
 #pragma unroll
-                    for (int t = 0; t < 2; ++t) {
-                        const int Nt = nn[t];
-                        const uint32_t s_col = tmem + (uint32_t)(kBN * t);
-                        const uint32_t o_col = tmem + kColO + (uint32_t)(D * t);
-                        if (n > 0 && n <= Nt) {
-                            if (!wait_bar(BAR(B_PFULL + t), (glob[t] + (uint32_t)(n - 1)) & 1u, abort_flag, status) ||
-                                (n == 1 && uses[t] > 0 &&
-                                 !wait_bar(BAR(B_OEMPTY + t), (uses[t] - 1u) & 1u, abort_flag, status))) {
+                        for (int t = 0; t < 2; ++t) {
+                            const int Nt = nn[t];
+                            const bool pv = n > 0 && n <= Nt, qk = n < Nt;
+                            if (!pv && !qk) continue;
+                            // every wait of the run first
+                            if (pv && (!wait_bar1(BAR(B_PFULL + t), (glob[t] + (uint32_t)(n - 1)) & 1u, abort_flag, status) ||
+                                       (n == 1 && uses[t] > 0 &&
+                                        !wait_bar1(BAR(B_OEMPTY + t), (uses[t] - 1u) & 1u, abort_flag, status)))) {
                                 ok = false;
                                 break;
                             }
-                            if (vst == ~0u && (vst = wait_pos(c + 2u * (uint32_t)(n - 1) + 1u)) == ~0u) {
+                            if (qk && n == 0 && !wait_bar1(BAR(B_QFULL + t), uses[t] & 1u, abort_flag, status)) {
+                                ok = false;
+                                break;
+                            }
+                            // K(n) and V(n) arrive together; V(n-1) was waited for with K(n-1)
+                            if (qk && t == 0 &&
+                                !wait_bar1(BAR(B_KV_FULL + kslot), ((c + (uint32_t)n) / kSlots) & 1u, abort_flag, status)) {
                                 ok = false;
                                 break;
                             }
                             tc_fence_after();
-                            const uint64_t vdesc = desc_mnmaj + ((uint32_t)(L::kKV + vst * L::kTileBytes) >> 4);
-                            if (lane == 0) {
+                            const uint32_t s_col = tmem + (uint32_t)(kBN * t);
+                            const uint32_t o_col = tmem + kColO + (uint32_t)(D * t);
+                            if (pv) {
                                 // P_t from TMEM (16 keys = 8 packed columns per step), V MN-major
                                 // (16 keys = 2048 bytes per step)
+                                const uint64_t vdesc = desc_mnmaj +
+                                    ((uint32_t)(L::kKV + (2u * vslot + 1u) * L::kTileBytes) >> 4);
                                 mma_ts(o_col, s_col, vdesc, kIdescPV, n > 1 ? 1u : 0u);
 #pragma unroll
                                 for (int kk = 1; kk < kBN / 16; ++kk)
                                     mma_ts(o_col, s_col + (uint32_t)kk * 8u, vdesc + (uint64_t)(kk * 128), kIdescPV, 1u);
-                                if (t == last_pv) mma_commit(BAR(B_KV_EMPTY + vst));
-                                if (n == Nt) mma_commit(BAR(B_OFULL + t));
                             }
-                            __syncwarp();
-                        }
-                        if (n < Nt) {
-                            // QK_t(n) into S_t (after PV_t(n-1) in issue order: P_t has been read)
-                            if (n == 0 && !wait_bar(BAR(B_QFULL + t), uses[t] & 1u, abort_flag, status)) {
-                                ok = false;
-                                break;
-                            }
-                            if (kst == ~0u && (kst = wait_pos(c + 2u * (uint32_t)n)) == ~0u) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
-                            const uint64_t qdesc = desc_kmaj + ((uint32_t)(L::kQ + t * L::kTileBytes) >> 4);
-                            const uint64_t kdesc = desc_kmaj + ((uint32_t)(L::kKV + kst * L::kTileBytes) >> 4);
-                            if (lane == 0) {
-                                // 16 d-columns per step: 32 bytes inside a 128-byte swizzle row, then
-                                // the next [128 x 64] half
+                            if (qk) {
+                                // QK_t(n) into S_t (after PV_t(n-1) in issue order: P_t has been
+                                // read); 16 d-columns per step: 32 bytes inside a 128-byte swizzle
+                                // row, then the next [128 x 64] half
+                                const uint64_t qdesc = desc_kmaj + ((uint32_t)(L::kQ + t * L::kTileBytes) >> 4);
+                                const uint64_t kdesc = desc_kmaj + ((uint32_t)(L::kKV + 2u * kslot * L::kTileBytes) >> 4);
 #pragma unroll
                                 for (int kk = 0; kk < kKSteps; ++kk) {
                                     const uint64_t koff = (uint64_t)((kk >> 2) * (kHalfBytes >> 4) + (kk & 3) * 2);
                                     mma_ss(s_col, qdesc + koff, kdesc + koff, kIdescQK, kk > 0 ? 1u : 0u);
                                 }
                                 mma_commit(BAR(B_SFULL + t));
-                                if (t == last_qk) mma_commit(BAR(B_KV_EMPTY + kst));
                                 if (n == Nt - 1) mma_commit(BAR(B_QEMPTY + t));
                             }
-                            __syncwarp();
+                            if (pv) {
+                                if (n == Nt) mma_commit(BAR(B_OFULL + t));
+                                if (t == last_pv) mma_commit(BAR(B_KV_EMPTY + vslot));
+                            }
+                        }
+                    }
+                    c += (uint32_t)N;
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        if (nn[t] > 0) {
+                            glob[t] += (uint32_t)nn[t];
+                            uses[t] += 1u;
                         }
                     }
                 }
-                c += 2u * (uint32_t)N;
-#pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    if (nn[t] > 0) {
-                        glob[t] += (uint32_t)nn[t];
-                        uses[t] += 1u;
-                    }
-                }
+                // drain the tensor pipe before TMEM is freed
+                mma_commit(BAR(B_FINAL));
+                drain_bar(BAR(B_FINAL), 0);
             }
-            // drain the tensor pipe before TMEM is freed
-            if (lane == 0) mma_commit(BAR(B_FINAL));
             __syncwarp();
-            drain_bar(BAR(B_FINAL), 0);
         }
     } else {
         // softmax: a whole row of S in registers

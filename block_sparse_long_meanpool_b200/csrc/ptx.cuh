@@ -203,6 +203,21 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     return __all_sync(0xffffffffu, ok);
 }
 
+// Bounded wait by a single thread (no warp vote): for a role that runs on one lane.  Returns
+// false when the CTA is aborting (this wait expired or another role's did).
+__device__ __forceinline__ bool wait_bar1(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int* status) {
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 63u && *abort_flag) return false;
+    }
+    if (!*abort_flag) {
+        *abort_flag = 1;
+        atomicExch(status, kTimeoutStatus);
+    }
+    return false;
+}
+
 // Bounded wait that ignores the abort flag (used to drain in-flight work on the way out).
 __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
     for (uint32_t i = 0; i < kSpinLimit; ++i)
