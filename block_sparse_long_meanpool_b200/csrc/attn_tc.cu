@@ -24,9 +24,11 @@
 //   PV_t(n-1): O_t += P_t(n-1) V(n-1)   (TS MMA: A = P from TMEM, B = V MN-major in smem)
 //   QK_t(n):   S_t  = Q_t K(n)^T        (SS MMA, fp32 accumulate)
 // so the tensor core works on one tile while the other tile's softmax runs.  Each tile's
-// PV_t(n-1) and QK_t(n) go out as one uninterrupted run of MMAs with every wait hoisted in
-// front of it: the tensor pipe drains whenever the issuing thread stops issuing, so the waits
-// and commits between runs are kept to three each per chunk.  PV_t(n-1) is
+// PV_t(n-1) and QK_t(n) go out as one uninterrupted run of MMAs.  The tensor pipe drains
+// whenever the issuing thread stops issuing (and a commit holds the thread until the queued
+// MMAs are dispatched), so the run's operands come in one ring slot -- step n of an item
+// loads K(n) and V(n-1) together, behind one barrier, two steps ahead -- and tile 1's waits
+// are done while tile 0's MMAs are still queued, before tile 0's commits.  PV_t(n-1) is
 // issued before QK_t(n), so the barrier announcing S_t(n) also guarantees that O_t holds every
 // earlier PV and that no MMA touches O_t until P_t(n) is announced: the softmax may rescale O_t
 // in between.  The softmax reads its row of S once (tcgen05.ld), takes the maximum with
@@ -51,7 +53,7 @@ namespace {
 using namespace ptx;
 
 constexpr int kBN = 128;       // keys per chunk
-constexpr int kSlots = 2;      // K/V ring: slot = K and V of one 128-key chunk, one barrier
+constexpr int kSlots = 2;      // K/V ring: step j of an item loads K(j) and V(j-1) into one slot
 constexpr int kThreads = 384;  // 12 warps
 constexpr int kWarpFetch = 8, kWarpMMA = 9, kWarpKV = 10, kWarpQ1 = 11;
 constexpr int kRegsSoftmax = 192, kRegsOther = 120;
@@ -281,8 +283,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                 mbar_arrive(BAR(B_ITEM_EMPTY + s));
             }
         } else if (warp == kWarpKV) {
-            // ---------------- K/V producer (TMA): chunk c of the CTA goes to slot c % 2 ----------
-            uint32_t c = 0;  // chunks issued so far
+            // ---------------- K/V producer (TMA) ----------------
+            // step j = 0..N of an item fills ring slot (CTA step count) % 2 with K(j) (j < N)
+            // and V(j-1) (j > 0): exactly the operands of the MMA runs of step j
+            uint32_t c = 0;  // steps issued so far
             for (int it = 0;; ++it) {
                 const int s = it & 1;
                 if (!wait_bar(BAR(B_INFO + s), (uint32_t)(it >> 1) & 1u, abort_flag, status)) break;
@@ -290,7 +294,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                 if (sl.kind < 0) break;
                 const int g = sl.g, key_start = sl.key_start, N = sl.nchunks;
                 bool ok = true;
-                for (int chunk = 0; chunk < N; ++chunk) {
+                for (int j = 0; j <= N; ++j) {
                     const uint32_t st = c % kSlots;
                     if (c >= kSlots &&
                         !wait_bar(BAR(B_KV_EMPTY + st), ((c / kSlots) - 1u) & 1u, abort_flag, status)) {
@@ -299,13 +303,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                     }
                     if (lane == 0) {
                         const uint32_t dst = sm_base + L::kKV + st * 2u * L::kTileBytes;
-                        mbar_arrive_tx(BAR(B_KV_FULL + st), 2u * kChunkBytes);
+                        mbar_arrive_tx(BAR(B_KV_FULL + st),
+                                       (j < N ? kChunkBytes : 0u) + (j > 0 ? kChunkBytes : 0u));
 #pragma unroll
                         for (int hh = 0; hh < kHalves; ++hh) {
-                            tma_load_3d(dst + hh * kHalfBytes, &tmap_k, BAR(B_KV_FULL + st), hh * 64, g,
-                                        key_start + chunk * kBN);
-                            tma_load_3d(dst + L::kTileBytes + hh * kHalfBytes, &tmap_v, BAR(B_KV_FULL + st),
-                                        hh * 64, g, key_start + chunk * kBN);
+                            if (j < N)
+                                tma_load_3d(dst + hh * kHalfBytes, &tmap_k, BAR(B_KV_FULL + st), hh * 64, g,
+                                            key_start + j * kBN);
+                            if (j > 0)
+                                tma_load_3d(dst + L::kTileBytes + hh * kHalfBytes, &tmap_v, BAR(B_KV_FULL + st),
+                                            hh * 64, g, key_start + (j - 1) * kBN);
                         }
                     }
                     __syncwarp();
@@ -319,11 +326,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                 drain_bar(BAR(B_KV_FULL + k % kSlots), (k / kSlots) & 1u);
         } else if (warp == kWarpMMA) {
             // ---------------- MMA issuer ----------------
-            // chunk n, tile by tile: PV_t(n-1) then QK_t(n) as one run of MMAs; tile t stops
-            // after its n_t chunks (n_1 <= n_0); n = n_0: the last PVs only.  One thread runs
-            // this role (waits without warp votes, no warp syncs between runs).
+            // step n = 0..N of an item, tile by tile: PV_t(n-1) then QK_t(n) as one run of MMAs
+            // (tile t runs while n <= n_t; n_1 <= n_0 = N).  One thread runs this role (waits
+            // without warp votes, no warp syncs between runs).
             if (lane == 0) {
-                uint32_t c = 0;               // CTA chunk index of the current item's chunk 0
+                uint32_t cs = 0;              // CTA step index of the current item's step 0
                 uint32_t glob[2] = {0u, 0u};  // chunks done per tile (S / P barrier phases)
                 uint32_t uses[2] = {0u, 0u};  // items done per tile (Q / O barrier phases)
                 bool ok = true;
@@ -332,80 +339,87 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                 // 2^18 bytes, so the 14-bit start-address field never carries).
                 const uint64_t desc_kmaj = smem_desc(sm_base, 16, 1024);                     // Q, K
                 const uint64_t desc_mnmaj = smem_desc(sm_base, (uint32_t)kHalfBytes, 1024);  // V
+                // the waits of tile t's run at step n (besides its ring slot)
+                auto run_waits = [&](int t, int n) -> bool {
+                    if (n > 0) {
+                        if (!wait_bar1(BAR(B_PFULL + t), (glob[t] + (uint32_t)(n - 1)) & 1u, abort_flag, status))
+                            return false;
+                        if (n == 1 && uses[t] > 0 &&
+                            !wait_bar1(BAR(B_OEMPTY + t), (uses[t] - 1u) & 1u, abort_flag, status))
+                            return false;
+                    } else if (!wait_bar1(BAR(B_QFULL + t), uses[t] & 1u, abort_flag, status)) {
+                        return false;
+                    }
+                    return true;
+                };
+                auto run_mmas = [&](int t, int n, int Nt, uint32_t slot) {
+                    const uint32_t s_col = tmem + (uint32_t)(kBN * t);
+                    const uint32_t o_col = tmem + kColO + (uint32_t)(D * t);
+                    if (n > 0) {
+                        // PV_t(n-1): P_t from TMEM (16 keys = 8 packed columns per step), V(n-1)
+                        // MN-major from the slot (16 keys = 2048 bytes per step)
+                        const uint64_t vdesc = desc_mnmaj + ((uint32_t)(L::kKV + (2u * slot + 1u) * L::kTileBytes) >> 4);
+                        mma_ts(o_col, s_col, vdesc, kIdescPV, n > 1 ? 1u : 0u);
+#pragma unroll
+                        for (int kk = 1; kk < kBN / 16; ++kk)
+                            mma_ts(o_col, s_col + (uint32_t)kk * 8u, vdesc + (uint64_t)(kk * 128), kIdescPV, 1u);
+                    }
+                    if (n < Nt) {
+                        // QK_t(n) into S_t (after PV_t(n-1) in issue order: P_t has been read);
+                        // 16 d-columns per step: 32 bytes inside a 128-byte swizzle row, then the
+                        // next [128 x 64] half
+                        const uint64_t qdesc = desc_kmaj + ((uint32_t)(L::kQ + t * L::kTileBytes) >> 4);
+                        const uint64_t kdesc = desc_kmaj + ((uint32_t)(L::kKV + 2u * slot * L::kTileBytes) >> 4);
+#pragma unroll
+                        for (int kk = 0; kk < kKSteps; ++kk) {
+                            const uint64_t koff = (uint64_t)((kk >> 2) * (kHalfBytes >> 4) + (kk & 3) * 2);
+                            mma_ss(s_col, qdesc + koff, kdesc + koff, kIdescQK, kk > 0 ? 1u : 0u);
+                        }
+                    }
+                };
+                auto run_commits = [&](int t, int n, int Nt, uint32_t slot, bool release) {
+                    if (n < Nt) {
+                        mma_commit(BAR(B_SFULL + t));
+                        if (n == Nt - 1) mma_commit(BAR(B_QEMPTY + t));
+                    }
+                    if (n > 0 && n == Nt) mma_commit(BAR(B_OFULL + t));
+                    if (release) mma_commit(BAR(B_KV_EMPTY + slot));  // the slot's last reader
+                };
                 for (int it = 0; ok; ++it) {
                     const int s = it & 1;
                     if (!wait_bar1(BAR(B_INFO + s), (uint32_t)(it >> 1) & 1u, abort_flag, status)) break;
                     const ItemSlot& sl = slots[s];
                     if (sl.kind < 0) break;
-                    const int N = sl.nchunks, nt = sl.ntiles;
-                    const int nn[2] = {sl.n[0], nt == 2 ? sl.n[1] : 0};
-                    for (int n = 0; n <= N && ok; ++n) {
-                        const uint32_t kslot = (c + (uint32_t)n) % kSlots;         // K(n)
-                        const uint32_t vslot = (c + (uint32_t)n + 1u) % kSlots;    // V(n-1)
-                        // the last tile to read V(n-1) releases its slot
-                        const int last_pv = (n - 1 < nn[1]) ? 1 : 0;
-#pragma unroll
-                        for (int t = 0; t < 2; ++t) {
-                            const int Nt = nn[t];
-                            const bool pv = n > 0 && n <= Nt, qk = n < Nt;
-                            if (!pv && !qk) continue;
-                            // every wait of the run first
-                            if (pv && (!wait_bar1(BAR(B_PFULL + t), (glob[t] + (uint32_t)(n - 1)) & 1u, abort_flag, status) ||
-                                       (n == 1 && uses[t] > 0 &&
-                                        !wait_bar1(BAR(B_OEMPTY + t), (uses[t] - 1u) & 1u, abort_flag, status)))) {
-                                ok = false;
-                                break;
-                            }
-                            if (qk && n == 0 && !wait_bar1(BAR(B_QFULL + t), uses[t] & 1u, abort_flag, status)) {
-                                ok = false;
-                                break;
-                            }
-                            // K(n) and V(n) arrive together; V(n-1) was waited for with K(n-1)
-                            if (qk && t == 0 &&
-                                !wait_bar1(BAR(B_KV_FULL + kslot), ((c + (uint32_t)n) / kSlots) & 1u, abort_flag, status)) {
-                                ok = false;
-                                break;
-                            }
+                    const int N = sl.nchunks;
+                    const int N1 = sl.ntiles == 2 ? sl.n[1] : 0;
+                    for (int n = 0; n <= N; ++n) {
+                        const uint32_t step = cs + (uint32_t)n, slot = step % kSlots;
+                        const bool act1 = N1 > 0 && n <= N1;
+                        if (!wait_bar1(BAR(B_KV_FULL + slot), (step / kSlots) & 1u, abort_flag, status) ||
+                            !run_waits(0, n)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        run_mmas(0, n, N, slot);
+                        // tile 1's waits while tile 0's MMAs are still queued
+                        if (act1 && !run_waits(1, n)) {
+                            ok = false;
+                            break;
+                        }
+                        run_commits(0, n, N, slot, !act1);
+                        if (act1) {
                             tc_fence_after();
-                            const uint32_t s_col = tmem + (uint32_t)(kBN * t);
-                            const uint32_t o_col = tmem + kColO + (uint32_t)(D * t);
-                            if (pv) {
-                                // P_t from TMEM (16 keys = 8 packed columns per step), V MN-major
-                                // (16 keys = 2048 bytes per step)
-                                const uint64_t vdesc = desc_mnmaj +
-                                    ((uint32_t)(L::kKV + (2u * vslot + 1u) * L::kTileBytes) >> 4);
-                                mma_ts(o_col, s_col, vdesc, kIdescPV, n > 1 ? 1u : 0u);
-#pragma unroll
-                                for (int kk = 1; kk < kBN / 16; ++kk)
-                                    mma_ts(o_col, s_col + (uint32_t)kk * 8u, vdesc + (uint64_t)(kk * 128), kIdescPV, 1u);
-                            }
-                            if (qk) {
-                                // QK_t(n) into S_t (after PV_t(n-1) in issue order: P_t has been
-                                // read); 16 d-columns per step: 32 bytes inside a 128-byte swizzle
-                                // row, then the next [128 x 64] half
-                                const uint64_t qdesc = desc_kmaj + ((uint32_t)(L::kQ + t * L::kTileBytes) >> 4);
-                                const uint64_t kdesc = desc_kmaj + ((uint32_t)(L::kKV + 2u * kslot * L::kTileBytes) >> 4);
-#pragma unroll
-                                for (int kk = 0; kk < kKSteps; ++kk) {
-                                    const uint64_t koff = (uint64_t)((kk >> 2) * (kHalfBytes >> 4) + (kk & 3) * 2);
-                                    mma_ss(s_col, qdesc + koff, kdesc + koff, kIdescQK, kk > 0 ? 1u : 0u);
-                                }
-                                mma_commit(BAR(B_SFULL + t));
-                                if (n == Nt - 1) mma_commit(BAR(B_QEMPTY + t));
-                            }
-                            if (pv) {
-                                if (n == Nt) mma_commit(BAR(B_OFULL + t));
-                                if (t == last_pv) mma_commit(BAR(B_KV_EMPTY + vslot));
-                            }
+                            run_mmas(1, n, N1, slot);
+                            run_commits(1, n, N1, slot, true);
                         }
                     }
-                    c += (uint32_t)N;
-#pragma unroll
-                    for (int t = 0; t < 2; ++t) {
-                        if (nn[t] > 0) {
-                            glob[t] += (uint32_t)nn[t];
-                            uses[t] += 1u;
-                        }
+                    cs += (uint32_t)N + 1u;
+                    glob[0] += (uint32_t)N;
+                    uses[0] += 1u;
+                    if (N1 > 0) {
+                        glob[1] += (uint32_t)N1;
+                        uses[1] += 1u;
                     }
                 }
                 // drain the tensor pipe before TMEM is freed
