@@ -411,13 +411,13 @@ def _hbm_stage_rates(w, st, peaks):
     mean_bytes = T * hkv * d * 2 + nb * hkv * d * 4
     gate_bytes = T * hq * d * 2 + T * hq * w.topk * 4 + nb * hkv * d * 4
     # merge: every row reads its min(topk, c + 1) partials (c = the row's block in its
-    # sequence) as fp32 o + lse and its slot count, and writes bf16 o + fp32 lse
+    # sequence) as bf16 o + fp32 lse and its slot count, and writes bf16 o + fp32 lse
     slots = 0
     for n in w.seqlens:
         for c in range((n + w.chunk_size - 1) // w.chunk_size):
             rows = min(w.chunk_size, n - c * w.chunk_size)
             slots += rows * min(w.topk, c + 1)
-    merge_bytes = hq * (slots * (d + 1) * 4 + T * (1 + d * 2 + 4))
+    merge_bytes = hq * (slots * (d * 2 + 4) + T * (1 + d * 2 + 4))
     res = {}
     for name, by in (("meanpool", mean_bytes), ("gate", gate_bytes)):
         ms = st[name]
@@ -431,15 +431,30 @@ def _hbm_stage_rates(w, st, peaks):
     return res
 
 
+def _attention_source_hash():
+    """sha256 over the attention kernel's sources (the kernel the traffic figure belongs to)."""
+    import hashlib
+
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_sparse_long_meanpool_b200", "csrc")
+    for f in ("attn_tc.cu", "ptx.cuh", "moba_internal.cuh"):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
 def _read_traffic(workload):
-    """DRAM bytes per attention launch from the committed ncu summary, when it matches the
-    current kernel (profiles/attention_<workload>.json)."""
+    """DRAM bytes per attention launch from the committed ncu summary
+    (profiles/attention_<workload>.json), or None when it was taken on other kernel sources."""
     path = os.path.join(ROOT, "profiles", f"attention_{workload}.json")
     try:
         with open(path) as f:
-            return json.load(f).get("traffic_bytes_per_launch")
+            rec = json.load(f)
     except Exception:
         return None
+    if rec.get("kernel_source_sha256") != _attention_source_hash():
+        return None
+    return rec.get("traffic_bytes_per_launch")
 
 
 def _gpu_id(dev):
