@@ -84,6 +84,13 @@ LENGTH_SWEEP = {
         f"1 x {m << 20} tokens, 32 q / 8 kv heads, d=128, 256 blocks of {(m << 20) // 256}, top-12")
     for m in (2, 4)
 }
+# 10M tokens with the same 256 blocks and top-12 (blocks of 40,960 tokens).  A 32 q / 8 kv-head
+# layer does not fit one GPU at this length (q and out alone are 168 GB), so this is one GPU's
+# share of it when the layer is split four ways by KV-head group: 8 q / 2 kv heads.
+LENGTH_SWEEP["prefill_10m"] = Workload(
+    "prefill_10m", [10 << 20], 8, 2, 128, (10 << 20) // 256, 12, "k_offsets", 1210,
+    "1 x 10485760 tokens, 8 q / 2 kv heads (a quarter of a 32/8-head layer), d=128, "
+    "256 blocks of 40960, top-12")
 ALL_WORKLOADS = {**WORKLOADS, **GRANULARITY_32K, **LENGTH_SWEEP}
 
 
