@@ -43,22 +43,42 @@ struct GateSmem {
 };
 
 // Inserts (x, id) into a descending list of K (score, index) pairs when it beats the last
-// entry; an equal score never displaces an entry already in the list.
+// entry; an equal score never displaces an entry already in the list.  Every position is
+// updated independently of the others (x is compared with all entries first, then entry i
+// keeps its value, takes x, or takes its left neighbour's old value), so an insertion is one
+// level of selects rather than a chain of K dependent compare-and-swaps.
 template <int K>
 __device__ __forceinline__ void insert_desc(float (&val)[K], int (&idx)[K], float x, int id,
                                             bool ok) {
     if (ok && x > val[K - 1]) {
+        bool gt[K];
 #pragma unroll
-        for (int i = 0; i < K; ++i) {
-            if (x > val[i]) {
-                const float tv = val[i];
-                const int ti = idx[i];
-                val[i] = x;
-                idx[i] = id;
-                x = tv;
-                id = ti;
-            }
+        for (int i = 0; i < K; ++i) gt[i] = x > val[i];
+#pragma unroll
+        for (int i = K - 1; i > 0; --i) {
+            val[i] = gt[i] ? (gt[i - 1] ? val[i - 1] : x) : val[i];
+            idx[i] = gt[i] ? (gt[i - 1] ? idx[i - 1] : id) : idx[i];
         }
+        val[0] = gt[0] ? x : val[0];
+        idx[0] = gt[0] ? id : idx[0];
+    }
+}
+
+// Inserts (x, id) into a list sorted by (score descending, index ascending) under that same
+// order (used to merge two lists); positions are updated independently as above.
+template <int K>
+__device__ __forceinline__ void insert_ordered(float (&val)[K], int (&idx)[K], float x, int id) {
+    bool gt[K];
+#pragma unroll
+    for (int i = 0; i < K; ++i) gt[i] = x > val[i] || (x == val[i] && id < idx[i]);
+    if (gt[K - 1]) {
+#pragma unroll
+        for (int i = K - 1; i > 0; --i) {
+            val[i] = gt[i] ? (gt[i - 1] ? val[i - 1] : x) : val[i];
+            idx[i] = gt[i] ? (gt[i - 1] ? idx[i - 1] : id) : idx[i];
+        }
+        val[0] = gt[0] ? x : val[0];
+        idx[0] = gt[0] ? id : idx[0];
     }
 }
 
@@ -245,22 +265,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
             }
             // merge: scores from the odd list enter with the full (score, lower index) order
 #pragma unroll
-            for (int i = 0; i < KMAX; ++i) {
-                float x = val2[i];
-                int id = idx2[i];
-#pragma unroll
-                for (int k2 = 0; k2 < KMAX; ++k2) {
-                    const bool better = x > val[k2] || (x == val[k2] && id < idx[k2]);
-                    if (better) {
-                        const float tv = val[k2];
-                        const int ti = idx[k2];
-                        val[k2] = x;
-                        idx[k2] = id;
-                        x = tv;
-                        id = ti;
-                    }
-                }
-            }
+            for (int i = 0; i < KMAX; ++i) insert_ordered<KMAX>(val, idx, val2[i], idx2[i]);
             tc_fence_before();
             mbar_arrive(BAR(B_SEMPTY + sb));
             const int rr = qt * kTileM + r;
