@@ -8,6 +8,7 @@
 
 #include "moba.h"
 #include "moba_internal.cuh"
+#include "ptx.cuh"
 
 using namespace moba;
 
@@ -318,6 +319,39 @@ moba_status moba_device_status(const moba_params* p, const void* workspace, void
     if (e != cudaSuccess) return cuda_fail(e, "status read");
     if (word == 0) return MOBA_OK;
     return fail((moba_status)word, "device status word %d", word);
+}
+
+// ---------------------------------------------------------------------------------------
+// Self-test of the bounded device waits (no counterpart in the pages).  One warp waits on an
+// mbarrier that nothing completes, through the same bounded wait the attention and gate
+// kernels use, with a short poll limit: the wait must give up, raise the CTA's abort flag and
+// record MOBA_ERR_DEVICE_TIMEOUT in the status word.  A wait that wrongly succeeds writes -1.
+
+namespace {
+
+__global__ void __launch_bounds__(32, 1) timeout_probe_kernel(int* status, uint32_t polls) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        moba::ptx::mbar_init(moba::ptx::smem_u32(&bar), 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+    const bool ok = moba::ptx::wait_bar(moba::ptx::smem_u32(&bar), 0u,
+                                        reinterpret_cast<volatile int*>(&abort_flag), status, polls);
+    if (ok && threadIdx.x == 0) atomicExch(status, -1);
+}
+
+}  // namespace
+
+extern "C" moba_status moba_selftest_timeout(int* status_dev, unsigned polls, void* stream) {
+    if (!status_dev) return fail(MOBA_ERR_INVALID_ARG, "status word is NULL");
+    if (polls == 0 || polls > (1u << 20)) return fail(MOBA_ERR_INVALID_ARG, "polls must be in [1, 2^20]");
+    timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(status_dev, polls);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "timeout probe launch");
+    return MOBA_OK;
 }
 
 const char* moba_status_string(moba_status s) {

@@ -187,9 +187,9 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // Bounded wait, called by all 32 lanes of a warp; the result is warp-uniform.  Returns false
 // when the CTA is aborting (this wait expired or another role's did).
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                         int* status) {
+                                         int* status, uint32_t limit = kSpinLimit) {
     bool ok = false;
-    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    for (uint32_t i = 0; i < limit; ++i) {
         if (mbar_try_wait(bar, parity)) {
             ok = true;
             break;

@@ -23,6 +23,7 @@ EXPORTS = (
     "moba_attn_fwd",
     "moba_attn_fwd_noalloc",
     "moba_device_status",
+    "moba_selftest_timeout",
     "moba_status_string",
     "moba_last_error",
 )
@@ -92,6 +93,8 @@ def load_library(path=LIB_PATH):
     lib.moba_attn_fwd_noalloc.restype = ctypes.c_int
     lib.moba_device_status.argtypes = [P, vp, vp]
     lib.moba_device_status.restype = ctypes.c_int
+    lib.moba_selftest_timeout.argtypes = [vp, ctypes.c_uint, vp]
+    lib.moba_selftest_timeout.restype = ctypes.c_int
     lib.moba_status_string.argtypes = [ctypes.c_int]
     lib.moba_status_string.restype = ctypes.c_char_p
     lib.moba_last_error.argtypes = []
@@ -182,6 +185,15 @@ def gate_topk(q, k_mean, cu_seqlens, chunk_size, topk, num_kv_heads=None):
     _check(load_library().moba_gate_topk(ctypes.byref(p), _ptr(q), _ptr(k_mean), _ptr(cu_seqlens),
                                          _ptr(sel), _stream(q.device)))
     return sel
+
+
+def selftest_timeout(device=None, polls=4096):
+    """moba_selftest_timeout: runs the bounded-wait self-test on `device` and returns the status
+    word it left (MOBA_ERR_DEVICE_TIMEOUT when the wait expired as it must)."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    word = torch.zeros(1, dtype=torch.int32, device=dev)
+    _check(load_library().moba_selftest_timeout(_ptr(word), int(polls), _stream(dev)))
+    return int(word.item())
 
 
 def choose_wave_tokens(T, hq, hkv, d, chunk_size, topk, batch, budget_bytes):

@@ -143,6 +143,19 @@ moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, co
  * Waits for the stream. */
 moba_status moba_device_status(const moba_params* p, const void* workspace, void* stream);
 
+/* ---- Self-test of the bounded device waits (no counterpart in the paper) ---------------
+ *
+ * Launches, on `stream`, one warp that waits on an mbarrier nothing completes, through the
+ * same bounded wait the attention and gate kernels use, giving up after `polls` polls
+ * (1 <= polls <= 2^20; each poll is one mbarrier.try_wait, which may itself suspend the warp
+ * for a short hardware-defined time).  The wait must expire: the kernel then writes
+ * MOBA_ERR_DEVICE_TIMEOUT (5) to *status_dev (a caller-owned device int, which should hold 0
+ * before the call) and returns; a wait that wrongly succeeds writes -1.  Nothing faults,
+ * traps or hangs, and the context stays usable.  Returns MOBA_ERR_INVALID_ARG for a NULL
+ * status word or polls out of range, MOBA_ERR_CUDA on a launch error, else MOBA_OK; the
+ * result is in *status_dev once the stream has reached the kernel's end. */
+moba_status moba_selftest_timeout(int* status_dev, unsigned polls, void* stream);
+
 /* ---- Allocation-free forward (no counterpart in the paper) -----------------------------
  *
  * Some callers cannot allocate device memory or hand over a workspace: plugin hosts that own
