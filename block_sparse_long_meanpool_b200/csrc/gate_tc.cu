@@ -42,46 +42,6 @@ struct GateSmem {
     static constexpr int kBytes(int n) { return kBars(n) + 8 * 8 + 16 + 1024; }
 };
 
-// Inserts (x, id) into a descending list of K (score, index) pairs when it beats the last
-// entry; an equal score never displaces an entry already in the list.  Every position is
-// updated independently of the others (x is compared with all entries first, then entry i
-// keeps its value, takes x, or takes its left neighbour's old value), so an insertion is one
-// level of selects rather than a chain of K dependent compare-and-swaps.
-template <int K>
-__device__ __forceinline__ void insert_desc(float (&val)[K], int (&idx)[K], float x, int id,
-                                            bool ok) {
-    if (ok && x > val[K - 1]) {
-        bool gt[K];
-#pragma unroll
-        for (int i = 0; i < K; ++i) gt[i] = x > val[i];
-#pragma unroll
-        for (int i = K - 1; i > 0; --i) {
-            val[i] = gt[i] ? (gt[i - 1] ? val[i - 1] : x) : val[i];
-            idx[i] = gt[i] ? (gt[i - 1] ? idx[i - 1] : id) : idx[i];
-        }
-        val[0] = gt[0] ? x : val[0];
-        idx[0] = gt[0] ? id : idx[0];
-    }
-}
-
-// Inserts (x, id) into a list sorted by (score descending, index ascending) under that same
-// order (used to merge two lists); positions are updated independently as above.
-template <int K>
-__device__ __forceinline__ void insert_ordered(float (&val)[K], int (&idx)[K], float x, int id) {
-    bool gt[K];
-#pragma unroll
-    for (int i = 0; i < K; ++i) gt[i] = x > val[i] || (x == val[i] && id < idx[i]);
-    if (gt[K - 1]) {
-#pragma unroll
-        for (int i = K - 1; i > 0; --i) {
-            val[i] = gt[i] ? (gt[i - 1] ? val[i - 1] : x) : val[i];
-            idx[i] = gt[i] ? (gt[i - 1] ? idx[i - 1] : id) : idx[i];
-        }
-        val[0] = gt[0] ? x : val[0];
-        idx[0] = gt[0] ? id : idx[0];
-    }
-}
-
 template <int D, int KMAX>
 __global__ void __launch_bounds__(kThreads, 1)
 gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restrict__ means,

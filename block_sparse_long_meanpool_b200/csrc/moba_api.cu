@@ -307,6 +307,67 @@ moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, co
     return MOBA_OK;
 }
 
+// ---- decode step ----------------------------------------------------------------------
+
+namespace {
+
+struct DecodeLayout {
+    size_t sel, nsl, part_o, part_lse, total;
+};
+
+DecodeLayout make_decode_layout(const moba_params& p) {
+    DecodeLayout L;
+    const size_t rows = (size_t)p.batch * p.num_q_heads;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o = align_up(o + bytes);
+        return at;
+    };
+    L.sel = take(4 * rows * p.topk);
+    L.nsl = take(4 * rows);
+    L.part_o = take(4 * rows * p.topk * p.head_dim);
+    L.part_lse = take(4 * rows * p.topk);
+    L.total = o;
+    return L;
+}
+
+}  // namespace
+
+size_t moba_decode_workspace_size(const moba_params* p) {
+    if (check_params(p) != MOBA_OK) return 0;
+    return make_decode_layout(*p).total;
+}
+
+moba_status moba_decode_fwd(const moba_params* p, const void* q, const void* k, const void* v,
+                            const int* cu_seqlens, const float* k_mean, void* workspace,
+                            size_t ws_bytes, void* out, float* lse, void* stream) {
+    moba_status s = check_params(p);
+    if (s != MOBA_OK) return s;
+    if (p->batch > 65535)
+        return fail(MOBA_ERR_UNSUPPORTED, "decode batch %d unsupported (<= 65535)", p->batch);
+    if (!q || !cu_seqlens || !workspace || !out || !lse || (p->total_tokens > 0 && (!k || !v || !k_mean)))
+        return fail(MOBA_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned16(q) || !aligned16(out) || !aligned16(workspace) ||
+        (p->total_tokens > 0 && (!aligned16(k) || !aligned16(v) || !aligned16(k_mean))))
+        return fail(MOBA_ERR_INVALID_ARG, "q, k, v, k_mean, out and workspace must be 16-byte aligned");
+    const DecodeLayout L = make_decode_layout(*p);
+    if (ws_bytes < L.total)
+        return fail(MOBA_ERR_WORKSPACE, "decode workspace too small: %zu < %zu bytes", ws_bytes, L.total);
+    const Problem P = make_problem(*p, blocks_bound(*p));
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    DecodeWorkspace ws;
+    ws.sel = reinterpret_cast<int*>(base + L.sel);
+    ws.nsl = reinterpret_cast<int*>(base + L.nsl);
+    ws.part_o = reinterpret_cast<float*>(base + L.part_o);
+    ws.part_lse = reinterpret_cast<float*>(base + L.part_lse);
+    cudaError_t e = launch_decode(P, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                                  static_cast<const __nv_bfloat16*>(v), cu_seqlens, k_mean, ws,
+                                  static_cast<__nv_bfloat16*>(out), lse, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    return MOBA_OK;
+}
+
 moba_status moba_device_status(const moba_params* p, const void* workspace, void* stream) {
     moba_status s = check_params(p);
     if (s != MOBA_OK) return s;

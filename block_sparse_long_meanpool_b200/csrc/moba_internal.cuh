@@ -100,6 +100,47 @@ __device__ __forceinline__ int for_each_routed(const int* __restrict__ row, int 
     return n;
 }
 
+// Top-k lists kept in registers (gate and decode gate).
+// Inserts (x, id) into a descending list of K (score, index) pairs when it beats the last
+// entry; an equal score never displaces an entry already in the list.  Every position is
+// updated independently of the others (x is compared with all entries first, then entry i
+// keeps its value, takes x, or takes its left neighbour's old value), so an insertion is one
+// level of selects rather than a chain of K dependent compare-and-swaps.
+template <int K>
+__device__ __forceinline__ void insert_desc(float (&val)[K], int (&idx)[K], float x, int id,
+                                            bool ok) {
+    if (ok && x > val[K - 1]) {
+        bool gt[K];
+#pragma unroll
+        for (int i = 0; i < K; ++i) gt[i] = x > val[i];
+#pragma unroll
+        for (int i = K - 1; i > 0; --i) {
+            val[i] = gt[i] ? (gt[i - 1] ? val[i - 1] : x) : val[i];
+            idx[i] = gt[i] ? (gt[i - 1] ? idx[i - 1] : id) : idx[i];
+        }
+        val[0] = gt[0] ? x : val[0];
+        idx[0] = gt[0] ? id : idx[0];
+    }
+}
+
+// Inserts (x, id) into a list sorted by (score descending, index ascending) under that same
+// order (used to merge two lists); positions are updated independently as above.
+template <int K>
+__device__ __forceinline__ void insert_ordered(float (&val)[K], int (&idx)[K], float x, int id) {
+    bool gt[K];
+#pragma unroll
+    for (int i = 0; i < K; ++i) gt[i] = x > val[i] || (x == val[i] && id < idx[i]);
+    if (gt[K - 1]) {
+#pragma unroll
+        for (int i = K - 1; i > 0; --i) {
+            val[i] = gt[i] ? (gt[i - 1] ? val[i - 1] : x) : val[i];
+            idx[i] = gt[i] ? (gt[i - 1] ? idx[i - 1] : id) : idx[i];
+        }
+        val[0] = gt[0] ? x : val[0];
+        idx[0] = gt[0] ? id : idx[0];
+    }
+}
+
 // ---------------------------------------------------------------------------------------
 // Launchers (defined in the .cu files).  Each returns cudaGetLastError() of its launch.
 
@@ -123,6 +164,18 @@ cudaError_t launch_attention(const Problem& P, const __nv_bfloat16* q, const __n
 cudaError_t launch_merge(const Problem& P, const int* cu_seqlens, const int* sel,
                          const Workspace& ws, int t0, int t1, __nv_bfloat16* out, float* lse,
                          cudaStream_t st);
+
+// Views into the workspace of one decode step (P.batch sequences, one query row each).
+struct DecodeWorkspace {
+    int* sel;         // [batch * hq, topk]: own block, routed blocks best-first, then -1
+    int* nsl;         // [batch * hq]: 1 + routed blocks (0 for an empty sequence)
+    float* part_o;    // [batch * hq * topk, d]: normalised partial outputs
+    float* part_lse;  // [batch * hq * topk]
+};
+cudaError_t launch_decode(const Problem& P, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                          const __nv_bfloat16* v, const int* cu_seqlens, const float* means,
+                          const DecodeWorkspace& ws, __nv_bfloat16* out, float* lse,
+                          cudaStream_t st);
 
 }  // namespace moba
 

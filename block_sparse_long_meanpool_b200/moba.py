@@ -22,6 +22,8 @@ EXPORTS = (
     "moba_gate_topk",
     "moba_attn_fwd",
     "moba_attn_fwd_noalloc",
+    "moba_decode_workspace_size",
+    "moba_decode_fwd",
     "moba_device_status",
     "moba_selftest_timeout",
     "moba_status_string",
@@ -91,6 +93,10 @@ def load_library(path=LIB_PATH):
     lib.moba_attn_fwd.restype = ctypes.c_int
     lib.moba_attn_fwd_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
     lib.moba_attn_fwd_noalloc.restype = ctypes.c_int
+    lib.moba_decode_workspace_size.argtypes = [P]
+    lib.moba_decode_workspace_size.restype = ctypes.c_size_t
+    lib.moba_decode_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp, vp]
+    lib.moba_decode_fwd.restype = ctypes.c_int
     lib.moba_device_status.argtypes = [P, vp, vp]
     lib.moba_device_status.restype = ctypes.c_int
     lib.moba_selftest_timeout.argtypes = [vp, ctypes.c_uint, vp]
@@ -185,6 +191,39 @@ def gate_topk(q, k_mean, cu_seqlens, chunk_size, topk, num_kv_heads=None):
     _check(load_library().moba_gate_topk(ctypes.byref(p), _ptr(q), _ptr(k_mean), _ptr(cu_seqlens),
                                          _ptr(sel), _stream(q.device)))
     return sel
+
+
+def decode_fwd(q, k, v, cu_seqlens, k_mean, chunk_size, topk, softmax_scale=None,
+               workspace=None, out=None, lse=None):
+    """Decode step (moba_decode_fwd): one new query per sequence against its KV cache.
+
+    q bf16 [batch, Hq, d] (the new token's query of each sequence); k, v bf16 [T, Hkv, d]
+    packed caches whose last row per sequence is the new token; cu_seqlens int32 [batch + 1];
+    k_mean fp32 block means of these caches (``meanpool``).  Returns (out bf16 [batch, Hq, d],
+    lse fp32 [Hq, batch]).
+    """
+    _check_qkv(q, k, v)
+    batch, hq, d = q.shape
+    T, hkv, _ = k.shape
+    _require(cu_seqlens.is_cuda and cu_seqlens.dtype == torch.int32 and cu_seqlens.numel() == batch + 1,
+             "cu_seqlens must be a CUDA int32 tensor of batch + 1 entries")
+    _require(k_mean.is_cuda and k_mean.dtype == torch.float32 and k_mean.is_contiguous(),
+             "k_mean must be a contiguous CUDA fp32 tensor")
+    p = make_params(batch, T, hq, hkv, d, chunk_size, topk, softmax_scale)
+    lib = load_library()
+    n = lib.moba_decode_workspace_size(ctypes.byref(p))
+    if n == 0:
+        raise MobaError(ERR_INVALID_ARG, lib.moba_last_error().decode())
+    if workspace is None:
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((batch, hq, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((hq, batch), dtype=torch.float32, device=q.device)
+    _check(lib.moba_decode_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens),
+                               _ptr(k_mean), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+                               _ptr(out), _ptr(lse), _stream(q.device)))
+    return out, lse
 
 
 def selftest_timeout(device=None, polls=4096):

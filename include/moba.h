@@ -143,6 +143,29 @@ moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, co
  * Waits for the stream. */
 moba_status moba_device_status(const moba_params* p, const void* workspace, void* stream);
 
+/* ---- Decode step -------------------------------------------------------------------------
+ *
+ * One new query per sequence against its KV cache (the analysis page of the MoBA paper,
+ * §2.2-§2.3, applied to the query at the last cache row t = L-1 of each sequence; the
+ * partial results per block are merged as in §3.2).  Exactly the prefill forward's row t:
+ * the own block c = (L-1) / chunk_size is forced (attended whole), the topk-1 best earlier
+ * blocks by q . mean_j are routed (ties to the lower index), softmax over the union.
+ *   p->batch         number of sequences (= query rows); p->total_tokens = T, the cache rows
+ *   q                bf16 [batch, Hq, d]: the new token's query of each sequence
+ *   k, v             bf16 [T, Hkv, d] packed caches (cu_seqlens); each sequence's last row is
+ *                    the new token's key / value
+ *   cu_seqlens       int32 [batch + 1], device; an empty sequence yields out = 0, lse = -inf
+ *   k_mean           fp32 [moba_num_blocks_bound(p), Hkv, d]: the block means moba_meanpool
+ *                    computes for these caches (only complete earlier blocks are read)
+ *   workspace        moba_decode_workspace_size(p) bytes, caller-owned device memory
+ *   out              bf16 [batch, Hq, d]; lse fp32 [Hq, batch] (natural log, scale included)
+ * Runs on the CUDA cores (HBM-bound: it streams the selected K/V blocks).  Asynchronous on
+ * `stream`; argument errors return before any launch.  batch <= 65535. */
+size_t moba_decode_workspace_size(const moba_params* p);
+moba_status moba_decode_fwd(const moba_params* p, const void* q, const void* k, const void* v,
+                            const int* cu_seqlens, const float* k_mean, void* workspace,
+                            size_t ws_bytes, void* out, float* lse, void* stream);
+
 /* ---- Self-test of the bounded device waits (no counterpart in the paper) ---------------
  *
  * Launches, on `stream`, one warp that waits on an mbarrier nothing completes, through the

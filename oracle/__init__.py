@@ -27,5 +27,6 @@ from .moba_ref import (  # noqa: F401
     attend_rows,
     attention_masked_dense,
     moba_forward,
+    moba_decode,
     attended_keys,
 )

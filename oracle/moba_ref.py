@@ -303,3 +303,55 @@ def moba_forward(q, k, v, cu_seqlens, chunk, topk, scale=None, sel=None):
         sel = select_blocks(q, means, cu_seqlens, chunk, topk)
     out, lse = attention_masked_dense(q, k, v, cu_seqlens, chunk, sel, scale)
     return {"out": out, "lse": lse, "sel": sel, "means": means}
+
+
+class _LastRowQueries:
+    """``q[t, h]`` view for the decode step: the new query of the sequence whose last row is
+    ``t``.  Only those rows exist (the per-row functions read nothing else)."""
+
+    def __init__(self, q_new, cu_seqlens):
+        self.q_new = np.asarray(q_new, dtype=np.float64)
+        cu = np.asarray(cu_seqlens, dtype=np.int64).reshape(-1)
+        self.row_of = {int(cu[b + 1]) - 1: b for b in range(len(cu) - 1) if cu[b + 1] > cu[b]}
+        self.shape = (int(cu[-1]),) + self.q_new.shape[1:]
+
+    def __getitem__(self, th):
+        t, h = th
+        return self.q_new[self.row_of[int(t)], h]
+
+
+def moba_decode(q_new, k, v, cu_seqlens, chunk, topk, scale=None):
+    """Decode step: one new query per sequence against its KV cache.
+
+    The cache of sequence b is rows ``cu[b] .. cu[b+1]-1`` of ``k`` / ``v``; its last row is
+    the new token's key and value, so the new query sits at position ``t = cu[b+1] - 1`` and
+    the rule of the analysis (§2.2-§2.3) applies to it unchanged: its own block
+    ``c = (t - cu[b]) // chunk`` is forced (all cached tokens of that block precede or equal t),
+    the ``topk - 1`` best earlier blocks by ``q . mean_j`` are routed, and the softmax runs over
+    the union.  This is exactly the prefill forward's row t, computed row by row.
+
+    ``q_new`` is ``[batch, Hq, d]``.  Returns ``out [batch, Hq, d]``, ``lse [Hq, batch]`` and
+    ``sel [batch, Hq, topk]`` (float64 / int64); an empty sequence has no query: zeros, -inf
+    and an all ``-1`` selection.
+    """
+    q_new = np.asarray(q_new, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    cu = np.asarray(cu_seqlens, dtype=np.int64).reshape(-1)
+    batch, Hq, d = q_new.shape
+    out = np.zeros((batch, Hq, d), dtype=np.float64)
+    lse = np.full((Hq, batch), -np.inf, dtype=np.float64)
+    sel = np.full((batch, Hq, topk), -1, dtype=np.int64)
+    rows = [(int(cu[b + 1]) - 1, h) for b in range(batch) if cu[b + 1] > cu[b] for h in range(Hq)]
+    if not rows:
+        return {"out": out, "lse": lse, "sel": sel}
+    qv = _LastRowQueries(q_new, cu)
+    means = block_means(k, cu, chunk)
+    s_rows = select_blocks_rows(qv, means, cu, chunk, topk, rows)
+    o_rows, l_rows = attend_rows(qv, k, v, cu, chunk, s_rows, rows, scale)
+    for r, (t, h) in enumerate(rows):
+        b = qv.row_of[t]
+        out[b, h] = o_rows[r]
+        lse[h, b] = l_rows[r]
+        sel[b, h] = s_rows[r]
+    return {"out": out, "lse": lse, "sel": sel}

@@ -378,3 +378,60 @@ def test_selected_block_flops_counts_attended_keys(seqlens, chunk, topk):
         for h in range(hq):
             n += len(oracle.attended_keys(t, sel[h, t], cu, chunk))
     assert W.selected_block_flops(seqlens, hq, d, chunk, topk) == 4 * d * n
+
+
+# ----------------------------------------------------------------------------------------
+# Decode step: the same rule applied to the last row of every cache
+
+
+def _decode_inputs(seqlens, hq, hkv, d, seed):
+    rng = np.random.default_rng(seed)
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int64)
+    T = int(cu[-1])
+    q = rng.standard_normal((T, hq, d))
+    k = rng.standard_normal((T, hkv, d)) + 0.5 * rng.standard_normal((1, hkv, d))
+    v = rng.standard_normal((T, hkv, d))
+    q_new = np.stack([q[cu[b + 1] - 1] if seqlens[b] > 0 else np.zeros((hq, d))
+                      for b in range(len(seqlens))])
+    return cu, q, k, v, q_new
+
+
+@pytest.mark.parametrize("seqlens,hq,hkv,chunk,topk", [
+    ([700, 0, 600, 1], 4, 2, 128, 3),        # empty and 1-token caches, partial blocks
+    ([1024, 385], 2, 2, 128, 4),            # a full last block, MHA
+    ([2000], 6, 2, 256, 2),                 # odd GQA group
+])
+def test_decode_equals_prefill_last_rows(seqlens, hq, hkv, chunk, topk):
+    """Decode (row-wise gather) equals the prefill forward's last row of every sequence
+    (masked-dense formulation), selections included."""
+    cu, q, k, v, q_new = _decode_inputs(seqlens, hq, hkv, 16, 40 + len(seqlens))
+    full = oracle.moba_forward(q, k, v, cu, chunk, topk)
+    dec = oracle.moba_decode(q_new, k, v, cu, chunk, topk)
+    for b, n in enumerate(seqlens):
+        if n == 0:
+            assert np.all(dec["out"][b] == 0) and np.all(np.isneginf(dec["lse"][:, b]))
+            assert np.all(dec["sel"][b] == -1)
+            continue
+        t = int(cu[b + 1]) - 1
+        np.testing.assert_allclose(dec["out"][b], full["out"][t], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dec["lse"][:, b], full["lse"][:, t], rtol=0, atol=1e-12)
+        assert np.array_equal(dec["sel"][b], full["sel"][:, t])
+
+
+def test_decode_with_every_block_selected_is_dense_attention_of_the_last_row():
+    """topk >= blocks: the new query attends to its whole cache (torch fp64 SDPA)."""
+    seqlens, hq, hkv, d = [900, 333], 4, 2, 16
+    cu, q, k, v, q_new = _decode_inputs(seqlens, hq, hkv, d, 7)
+    dec = oracle.moba_decode(q_new, k, v, cu, 128, 16)
+    scale = 1.0 / math.sqrt(d)
+    for b in range(len(seqlens)):
+        s, e = int(cu[b]), int(cu[b + 1])
+        for h in range(hq):
+            g = h // (hq // hkv)
+            qt = torch.from_numpy(q_new[b, h])[None, None, None]
+            kt = torch.from_numpy(k[s:e, g])[None, None]
+            vt = torch.from_numpy(v[s:e, g])[None, None]
+            o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=scale)
+            z = (kt[0, 0] @ qt[0, 0, 0]) * scale
+            np.testing.assert_allclose(dec["out"][b, h], o[0, 0, 0].numpy(), rtol=0, atol=1e-12)
+            assert abs(dec["lse"][h, b] - torch.logsumexp(z, 0).item()) < 1e-12
