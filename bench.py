@@ -404,6 +404,169 @@ def run_ours(args, w, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_decode(args, w, world, rank, local):
+    """Decode step: one moba_decode_fwd per step over caches of the workload's shape."""
+    import torch
+
+    import oracle
+    from block_sparse_long_meanpool_b200 import build as _build
+    from block_sparse_long_meanpool_b200 import moba
+    from block_sparse_long_meanpool_b200 import workloads as W
+
+    if rank == 0:
+        _build.build()
+    barrier(world)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    x = W.make_inputs(w, device=dev, seed=rank_seed(w, rank))
+    k, v, cu = x["k"], x["v"], x["cu_seqlens"]
+    B, hq, hkv, d = len(w.seqlens), w.num_q_heads, w.num_kv_heads, w.head_dim
+    chunk, topk = w.chunk_size, w.topk
+    last = torch.tensor([c - 1 for c in w.cu_seqlens[1:]], device=dev)
+    q_new = x["q"][last].contiguous()
+    means = moba.meanpool(k, cu, chunk)  # cache state, kept outside the timed step
+    p = moba.make_params(B, w.total_tokens, hq, hkv, d, chunk, topk)
+    ws = torch.empty(moba.load_library().moba_decode_workspace_size(p), dtype=torch.uint8, device=dev)
+    out = torch.empty((B, hq, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((hq, B), dtype=torch.float32, device=dev)
+
+    def step():
+        moba.decode_fwd(q_new, k, v, cu, means, chunk, topk, workspace=ws, out=out, lse=lse)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(_gpu_id(dev))
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(args.steps):
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier(world)
+    ms = max_over_ranks(start.elapsed_time(end) / args.steps, world)
+
+    peaks = read_peaks()
+    keys = W.decode_attended_keys(w.seqlens, chunk, topk)
+    algo_bytes = keys * hq * d * 2 * 2 + B * hq * d * 2 + B * hq * (d * 2 + 4)
+    gbs = algo_bytes / (ms * 1e-3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        qh = q_new.cpu().pin_memory()
+        outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        lseh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+        def e2e_step():
+            q_new.copy_(qh, non_blocking=True)
+            step()
+            outh.copy_(out, non_blocking=True)
+            lseh.copy_(lse, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+        e2e = {"value": B * world / (e_ms * 1e-3), "unit": "sequences/s",
+               "h2d_bytes_per_step": qh.numel() * 2,
+               "d2h_bytes_per_step": outh.numel() * 2 + lseh.numel() * 4, "ms_per_step": e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # the oracle on the first sequence's cache (means included), as it stands
+        n0 = w.seqlens[0]
+        kh = k[:n0].double().cpu().numpy()
+        vh = v[:n0].double().cpu().numpy()
+        qh1 = q_new[:1].double().cpu().numpy()
+        t0 = time.time()
+        oracle.moba_decode(qh1, kh, vh, [0, n0], chunk, topk)
+        dt = time.time() - t0
+        cpu = {"value": 1.0 / dt, "unit": "sequences/s", "cores": os.cpu_count(), "kind": "oracle",
+               "sample": f"1 of {B} sequences (its whole {n0}-token cache: block means, gate, attention)"}
+
+    if rank == 0:
+        line = {
+            "metric": "MoBA decode sequences/s (one new token per sequence, all heads of one attention layer)",
+            "value": B * world / (ms * 1e-3),
+            "unit": "sequences/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded, generated on device)",
+            "config": {"workload": w.name, "description": w.description, "sequences": B,
+                       "cache_tokens": w.total_tokens, "q_heads": hq, "kv_heads": hkv,
+                       "head_dim": d, "chunk_size": chunk, "topk": topk,
+                       "means": "cached block means (moba_meanpool once, outside the step)",
+                       "l2": "caches larger than L2 (no flush)", "parallelism": f"dp{world}"},
+            "roofline": {"bound": "hbm", "kernel": "decode step (gate, block attention, merge)",
+                         "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "peak_kind": "HBM copy (measured)",
+                         "traffic": None,
+                         "bytes_per_step": algo_bytes,
+                         "note": "selected blocks' K and V per query head; query heads of one KV head that pick the same block share it through L2"},
+            "clocks": clocks,
+            "gpu_launches": 3 * args.steps,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_decode_reference(args, w, world, rank):
+    """The float64 oracle's decode step on the host cores, one sequence's cache per step."""
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+
+    import oracle
+    from block_sparse_long_meanpool_b200 import workloads as W
+
+    n0 = w.seqlens[0]
+    one = W.custom(w.name + "_seq0", [n0], w.num_q_heads, w.num_kv_heads, w.head_dim,
+                   w.chunk_size, w.topk, w.structure, w.seed)
+    x = W.make_inputs(one, device="cpu")
+    k = x["k"].double().numpy()
+    v = x["v"].double().numpy()
+    q1 = x["q"][n0 - 1:n0].double().numpy()
+    oracle.moba_decode(q1, k, v, [0, n0], w.chunk_size, w.topk)  # warm-up
+    t0 = time.time()
+    for _ in range(args.steps):
+        oracle.moba_decode(q1, k, v, [0, n0], w.chunk_size, w.topk)
+    dt = (time.time() - t0) / args.steps
+    value = 1.0 / dt
+    print(json.dumps({
+        "impl": "reference",
+        "metric": "MoBA decode sequences/s (one new token per sequence, all heads of one attention layer)",
+        "value": value, "unit": "sequences/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": w.name, "description": w.description},
+        "cpu_baseline": {"value": value, "unit": "sequences/s", "cores": os.cpu_count(),
+                         "kind": "oracle", "sample": f"1 of {len(w.seqlens)} sequences per step"},
+        "e2e": {"value": value, "unit": "sequences/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
 def _hbm_stage_rates(w, st, peaks):
     """Achieved GB/s of the HBM-bound stages from their algorithmic bytes."""
     T, hq, hkv, d = w.total_tokens, w.num_q_heads, w.num_kv_heads, w.head_dim
@@ -481,11 +644,29 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--decode", action="store_true",
+                    help="time the decode step (workloads.DECODE_WORKLOADS) instead of the prefill")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from block_sparse_long_meanpool_b200 import workloads as W
 
+    if args.decode:
+        name = args.workload if args.workload in W.DECODE_WORKLOADS else "decode_32k_b64"
+        w = W.DECODE_WORKLOADS[name]
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        if args.impl == "reference":
+            run_decode_reference(args, w, world, rank)
+            return
+        world, rank, local = dist_setup()
+        try:
+            run_decode(args, w, world, rank, local)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
+        return
     w = W.ALL_WORKLOADS[args.workload]
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -93,6 +93,31 @@ LENGTH_SWEEP["prefill_10m"] = Workload(
     "256 blocks of 40960, top-12")
 ALL_WORKLOADS = {**WORKLOADS, **GRANULARITY_32K, **LENGTH_SWEEP}
 
+# Decode step: caches of these shapes, one new query per sequence (its last row).
+DECODE_WORKLOADS = {
+    "decode_32k_b64": Workload(
+        "decode_32k_b64", [32768] * 64, 32, 8, 128, 512, 3, "k_offsets", 1301,
+        "64 caches of 32768 tokens, 32 q / 8 kv heads, d=128, chunk 512 (64 blocks), top-3"),
+    "decode_128k_b16": Workload(
+        "decode_128k_b16", [131072] * 16, 32, 8, 128, 2048, 8, "k_offsets", 1302,
+        "16 caches of 131072 tokens, 32 q / 8 kv heads, d=128, chunk 2048 (64 blocks), top-8"),
+    "decode_1m_b1": Workload(
+        "decode_1m_b1", [1 << 20], 32, 8, 128, 4096, 12, "k_offsets", 1303,
+        "1 cache of 1,048,576 tokens, 32 q / 8 kv heads, d=128, chunk 4096 (256 blocks), top-12"),
+}
+
+
+def decode_attended_keys(seqlens, chunk, topk):
+    """Keys one new query attends to, summed over the sequences: its own block up to the new
+    token plus min(topk - 1, c) whole earlier blocks.  A measurement formula."""
+    keys = 0
+    for n in seqlens:
+        if n <= 0:
+            continue
+        c = (n - 1) // chunk
+        keys += (n - c * chunk) + chunk * min(topk - 1, c)
+    return keys
+
 
 def custom(name, seqlens, hq, hkv, d, chunk, topk, structure="k_offsets", seed=7):
     """A workload of any shape with the same value recipe (for tests and sweeps)."""
