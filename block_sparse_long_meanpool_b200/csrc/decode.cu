@@ -9,7 +9,9 @@
 // (sequence, head), so the step streams whole K/V blocks and is HBM-bound: it runs on the CUDA
 // cores.
 //   decode_gate_kernel   one warp per (sequence, query head): fp32 scores, top-(k-1)
-//   decode_attn_kernel   one CTA per (slot, query head, sequence): one block's keys in tiles
+//   decode_attn_kernel   one CTA per (slot, key range, query head, sequence): a selected
+//                        block's keys in tiles (a block is cut into several ranges when there
+//                        are too few (sequence, head, block) tasks to fill the GPU)
 //   decode_merge_kernel  one warp per (sequence, query head)
 #include <climits>
 
@@ -118,8 +120,9 @@ decode_gate_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict_
     for (int i = 1 + n_route + lane; i < P.topk; i += 32) srow[i] = -1;
 }
 
-// One (sequence, head, slot): softmax attention of the new query over one selected block,
-// written as a normalised fp32 partial (o, lse).  Keys stream through shared memory in tiles
+// One (sequence, head, slot, range): softmax attention of the new query over one key range of
+// one selected block, written as a normalised fp32 partial (o, lse); an empty range writes
+// o = 0, lse = -inf, which the merge weighs by zero.  Keys stream through shared memory in tiles
 // of 64 rows (K and V, 16-byte loads; rows padded by 16 bytes so that the four threads that
 // score one key, reading every fourth bf16 pair, hit distinct banks).  Scores are kept in
 // log2 units (q pre-scaled by scale * log2 e); the running maximum and sum follow the
@@ -129,7 +132,7 @@ __global__ void __launch_bounds__(kAttnThreads)
 decode_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                    const __nv_bfloat16* __restrict__ v, const int* __restrict__ cu, Problem P,
                    const int* __restrict__ sel, const int* __restrict__ nsl,
-                   float* __restrict__ part_o, float* __restrict__ part_lse) {
+                   float* __restrict__ part_o, float* __restrict__ part_lse, int splits) {
     constexpr int kRowWords = D / 2 + 4;  // 32-bit words per padded smem row
     constexpr int kSub = kAttnThreads / D;  // threads per output dimension
     __shared__ float2 qs[D / 2];
@@ -139,14 +142,24 @@ decode_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
     __shared__ float bcast[2];
     __shared__ float accs[kSub][D];
 
-    const int slot = blockIdx.x, h = blockIdx.y, seq = blockIdx.z;
+    const int slot = blockIdx.x / splits, rng = blockIdx.x - slot * splits;
+    const int h = blockIdx.y, seq = blockIdx.z;
     const int w = seq * P.hq + h;
     if (slot >= __ldg(nsl + w)) return;  // uniform over the CTA
     const int j = __ldg(sel + (size_t)w * P.topk + slot);
     const int start = __ldg(cu + seq), L = __ldg(cu + seq + 1) - start;
-    const int k0 = start + j * P.chunk, k1 = start + min((j + 1) * P.chunk, L);
+    const int b0 = start + j * P.chunk, b1 = start + min((j + 1) * P.chunk, L);
+    // this CTA's range: whole 64-key tiles of the block, cut into `splits` contiguous parts
+    const int per = ((b1 - b0 + kKeyTile - 1) / kKeyTile + splits - 1) / splits * kKeyTile;
+    const int k0 = b0 + rng * per, k1 = min(b1, k0 + per);
     const int g = h / P.group;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const size_t pi = ((size_t)w * P.topk + slot) * splits + rng;
+    if (k0 >= k1) {
+        if (tid < D) part_o[pi * D + tid] = 0.f;
+        if (tid == 0) part_lse[pi] = -INFINITY;
+        return;
+    }
 
     for (int i = tid; i < D / 2; i += kAttnThreads) {
         const __nv_bfloat162 b2 = reinterpret_cast<const __nv_bfloat162*>(q + (size_t)w * D)[i];
@@ -219,7 +232,6 @@ decode_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
         float o = 0.f;
 #pragma unroll
         for (int s = 0; s < kSub; ++s) o += accs[s][tid];
-        const size_t pi = (size_t)w * P.topk + slot;
         part_o[pi * D + tid] = o / bcast[0];
         if (tid == 0) part_lse[pi] = bcast[1] * 0.69314718055994531f + logf(bcast[0]);
     }
@@ -232,13 +244,13 @@ template <int D>
 __global__ void __launch_bounds__(kGateWarps * 32)
 decode_merge_kernel(const int* __restrict__ nsl, const float* __restrict__ part_o,
                     const float* __restrict__ part_lse, Problem P, __nv_bfloat16* __restrict__ out,
-                    float* __restrict__ lse) {
+                    float* __restrict__ lse, int splits) {
     constexpr int V = D / 32;  // channels per lane
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int w = blockIdx.x * kGateWarps + warp;
     if (w >= P.batch * P.hq) return;
     const int seq = w / P.hq, h = w - seq * P.hq;
-    const int ns = __ldg(nsl + w);
+    const int ns = __ldg(nsl + w) * splits;  // partials of the row: its blocks' key ranges
     __nv_bfloat16* dst = out + (size_t)w * D + lane * V;
     if (ns == 0) {
 #pragma unroll
@@ -246,20 +258,23 @@ decode_merge_kernel(const int* __restrict__ nsl, const float* __restrict__ part_
         if (lane == 0) lse[(size_t)h * P.batch + seq] = -INFINITY;
         return;
     }
-    const size_t pbase = (size_t)w * P.topk;
-    const float li = (lane < ns) ? __ldg(part_lse + pbase + lane) : -INFINITY;
-    float mx = li;
+    const size_t pbase = (size_t)w * P.topk * splits;
+    // lane s holds partials s and s + 32 (at most 64 per row)
+    const float la = (lane < ns) ? __ldg(part_lse + pbase + lane) : -INFINITY;
+    const float lb = (lane + 32 < ns) ? __ldg(part_lse + pbase + lane + 32) : -INFINITY;
+    float mx = fmaxf(la, lb);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    const float wi = (lane < ns) ? expf(li - mx) : 0.f;
-    float L = wi;
+    const float wa = (lane < ns) ? expf(la - mx) : 0.f;
+    const float wb = (lane + 32 < ns) ? expf(lb - mx) : 0.f;
+    float L = wa + wb;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
     float acc[V];
 #pragma unroll
     for (int e = 0; e < V; ++e) acc[e] = 0.f;
     for (int i = 0; i < ns; ++i) {
-        const float wgt = __shfl_sync(0xffffffffu, wi, i);
+        const float wgt = (i < 32) ? __shfl_sync(0xffffffffu, wa, i & 31) : __shfl_sync(0xffffffffu, wb, i & 31);
         const float* src = part_o + (pbase + i) * D + lane * V;
 #pragma unroll
         for (int e = 0; e < V; ++e) acc[e] = fmaf(wgt, __ldg(src + e), acc[e]);
@@ -288,11 +303,12 @@ cudaError_t launch_decode_d(const Problem& P, const __nv_bfloat16* q, const __nv
         decode_gate_kernel<D, 32><<<row_blocks, kGateWarps * 32, 0, st>>>(q, means, cu, P, ws.sel, ws.nsl);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    decode_attn_kernel<D><<<dim3(P.topk, P.hq, P.batch), kAttnThreads, 0, st>>>(
-        q, k, v, cu, P, ws.sel, ws.nsl, ws.part_o, ws.part_lse);
+    decode_attn_kernel<D><<<dim3(P.topk * ws.splits, P.hq, P.batch), kAttnThreads, 0, st>>>(
+        q, k, v, cu, P, ws.sel, ws.nsl, ws.part_o, ws.part_lse, ws.splits);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    decode_merge_kernel<D><<<row_blocks, kGateWarps * 32, 0, st>>>(ws.nsl, ws.part_o, ws.part_lse, P, out, lse);
+    decode_merge_kernel<D><<<row_blocks, kGateWarps * 32, 0, st>>>(ws.nsl, ws.part_o, ws.part_lse, P, out, lse,
+                                                                   ws.splits);
     return cudaGetLastError();
 }
 

@@ -318,6 +318,7 @@ struct DecodeLayout {
 DecodeLayout make_decode_layout(const moba_params& p) {
     DecodeLayout L;
     const size_t rows = (size_t)p.batch * p.num_q_heads;
+    const size_t parts = (size_t)p.topk * decode_splits(p.batch, p.num_q_heads, p.topk, p.chunk_size);
     size_t o = 0;
     auto take = [&](size_t bytes) {
         const size_t at = o;
@@ -326,8 +327,8 @@ DecodeLayout make_decode_layout(const moba_params& p) {
     };
     L.sel = take(4 * rows * p.topk);
     L.nsl = take(4 * rows);
-    L.part_o = take(4 * rows * p.topk * p.head_dim);
-    L.part_lse = take(4 * rows * p.topk);
+    L.part_o = take(4 * rows * parts * p.head_dim);
+    L.part_lse = take(4 * rows * parts);
     L.total = o;
     return L;
 }
@@ -361,6 +362,7 @@ moba_status moba_decode_fwd(const moba_params* p, const void* q, const void* k, 
     ws.nsl = reinterpret_cast<int*>(base + L.nsl);
     ws.part_o = reinterpret_cast<float*>(base + L.part_o);
     ws.part_lse = reinterpret_cast<float*>(base + L.part_lse);
+    ws.splits = decode_splits(p->batch, p->num_q_heads, p->topk, p->chunk_size);
     cudaError_t e = launch_decode(P, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
                                   static_cast<const __nv_bfloat16*>(v), cu_seqlens, k_mean, ws,
                                   static_cast<__nv_bfloat16*>(out), lse, static_cast<cudaStream_t>(stream));

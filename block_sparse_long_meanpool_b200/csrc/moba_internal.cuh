@@ -169,9 +169,18 @@ cudaError_t launch_merge(const Problem& P, const int* cu_seqlens, const int* sel
 struct DecodeWorkspace {
     int* sel;         // [batch * hq, topk]: own block, routed blocks best-first, then -1
     int* nsl;         // [batch * hq]: 1 + routed blocks (0 for an empty sequence)
-    float* part_o;    // [batch * hq * topk, d]: normalised partial outputs
-    float* part_lse;  // [batch * hq * topk]
+    float* part_o;    // [batch * hq * topk * splits, d]: normalised partial outputs
+    float* part_lse;  // [batch * hq * topk * splits]
+    int splits;       // key ranges per selected block (a power of two, topk * splits <= 64)
 };
+// Key ranges per selected block for a decode step: enough (row, block, range) tasks to fill
+// the GPU, while every row's partials still fit one warp's merge (topk * splits <= 64, two per
+// lane) and a range keeps at least 128 keys.  A function of the parameters only.
+inline int decode_splits(int batch, int hq, int topk, int chunk) {
+    int s = 1;
+    while ((long long)batch * hq * topk * s < 1184 && topk * s * 2 <= 64 && chunk / (s * 2) >= 128) s *= 2;
+    return s;
+}
 cudaError_t launch_decode(const Problem& P, const __nv_bfloat16* q, const __nv_bfloat16* k,
                           const __nv_bfloat16* v, const int* cu_seqlens, const float* means,
                           const DecodeWorkspace& ws, __nv_bfloat16* out, float* lse,
