@@ -276,3 +276,22 @@ class _QView:
     def __getitem__(self, idx):
         t, h = idx
         return self.rows[int(t)][h]
+
+
+def test_cuda_core_gate_above_257_blocks():
+    """More than 257 blocks in one call select the CUDA-core gate (csrc/gate.cu) instead of the
+    tensor-core one: its selections against the oracle's, outside the near-tie band."""
+    w = W.custom("gate_267_blocks", [20000, 14000], 2, 1, 64, 128, 4, "k_offsets", 25)
+    q, k, _, cu_t = gpu_inputs(w)
+    cu = np.asarray(w.cu_seqlens)
+    chunk, topk, group = w.chunk_size, w.topk, w.num_q_heads // w.num_kv_heads
+    p = moba.make_params(len(w.seqlens), w.total_tokens, w.num_q_heads, w.num_kv_heads,
+                         w.head_dim, chunk, topk)
+    assert moba.num_blocks_bound(p) > 257
+    means = moba.meanpool(k, cu_t, chunk)
+    sel = moba.gate_topk(q, means, cu_t, chunk, topk)
+    torch.cuda.synchronize()
+    q_np, k_np = PT.host(q), PT.host(k)
+    om = oracle.block_means(k_np, cu, chunk)
+    osel = oracle.select_blocks(q_np, om, cu, chunk, topk)
+    full_sel_check(PT.host(sel, np.int64), osel, q_np, om, cu, chunk, topk, group)
