@@ -137,3 +137,42 @@ def test_wave_choice_respects_budget(lib):
     p = moba.make_params(1, 1 << 20, 32, 8, 128, 4096, 12, None, w)
     assert lib.moba_workspace_size(ctypes.byref(p)) <= 8 << 30
     assert moba.choose_wave_tokens(2048, 4, 4, 64, 256, 3, 1, 1 << 30) == 0
+
+
+def test_decode_workspace_size_and_argument_checks(lib):
+    p = params()
+    need = lib.moba_decode_workspace_size(ctypes.byref(p))
+    assert need > 0
+    bad = params(head_dim=96)
+    assert lib.moba_decode_workspace_size(ctypes.byref(bad)) == 0
+    assert lib.moba_decode_fwd(None, None, None, None, None, None, None, 0, None, None, None) == moba.ERR_INVALID_ARG
+    assert lib.moba_decode_fwd(ctypes.byref(p), None, None, None, None, None, None, need,
+                               None, None, None) == moba.ERR_INVALID_ARG
+    big = params(batch=70000)
+    assert lib.moba_decode_workspace_size(ctypes.byref(big)) > 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="hands fake device addresses to the library: host-only check")
+def test_decode_checks_precede_any_launch(lib):
+    p = params()
+    fake = ctypes.c_void_p(1 << 20)
+    need = lib.moba_decode_workspace_size(ctypes.byref(p))
+    rc = lib.moba_decode_fwd(ctypes.byref(p), fake, fake, fake, fake, fake, fake, need - 1,
+                             fake, fake, None)
+    assert rc == moba.ERR_WORKSPACE
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    rc = lib.moba_decode_fwd(ctypes.byref(p), odd, fake, fake, fake, fake, fake, need,
+                             fake, fake, None)
+    assert rc == moba.ERR_INVALID_ARG
+    big = params(batch=70000)
+    rc = lib.moba_decode_fwd(ctypes.byref(big), fake, fake, fake, fake, fake, fake,
+                             lib.moba_decode_workspace_size(ctypes.byref(big)), fake, fake, None)
+    assert rc == moba.ERR_UNSUPPORTED
+
+
+def test_selftest_argument_checks(lib):
+    assert lib.moba_selftest_timeout(None, 16, None) == moba.ERR_INVALID_ARG
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.moba_selftest_timeout(fake, 0, None) == moba.ERR_INVALID_ARG
+    assert lib.moba_selftest_timeout(fake, (1 << 20) + 1, None) == moba.ERR_INVALID_ARG
