@@ -21,6 +21,8 @@ figures).  No function is "parity unpinned".
 from .moba_ref import (  # noqa: F401
     block_table,
     block_means,
+    block_minmax,
+    minmax_scores_row,
     gate_scores_row,
     select_blocks,
     select_blocks_rows,

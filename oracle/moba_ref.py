@@ -95,6 +95,43 @@ def block_means(k, cu_seqlens, chunk):
     return means
 
 
+def block_minmax(k, cu_seqlens, chunk):
+    """Per-channel minimum and maximum key of every block, per KV head.
+
+    The analysis (§1.3 and its list of limitations, §5.1 item 6) names Quest as the MoBA
+    variant with min/max pooling in place of the mean and calls it the stronger block
+    summary (§6.3 lists it as the gate's next step), without writing the summary out.  Reading: Quest's published one (Tang et al.,
+    2024, "Quest: Query-Aware Sparsity for Efficient Long-Context LLM Inference"), the
+    element-wise minimum and maximum of the block's keys, over its valid tokens.
+
+    Returns ``(kmin, kmax)``, each ``[NB, Hkv, d]`` float64.
+    """
+    k = np.asarray(k, dtype=np.float64)
+    tab = block_table(cu_seqlens, chunk)
+    nb = len(tab["start"])
+    kmin = np.zeros((nb, k.shape[1], k.shape[2]), dtype=np.float64)
+    kmax = np.zeros_like(kmin)
+    for b in range(nb):
+        rows = k[tab["start"][b]:tab["end"][b]]
+        kmin[b] = rows.min(axis=0)
+        kmax[b] = rows.max(axis=0)
+    return kmin, kmax
+
+
+def minmax_scores_row(q_row, minmax_rows):
+    """Min/max gate affinities of one query row against a list of block summaries.
+
+    Quest's block score (the reading of :func:`block_minmax`): per channel i the larger of
+    ``q_i * kmax_i`` and ``q_i * kmin_i``, summed over the channels.  It is the largest value
+    ``<q, x>`` takes over the box ``kmin <= x <= kmax``, so an upper bound of ``<q, k>`` over
+    every key of the block.  ``minmax_rows`` is ``[n, 2, d]`` (index 0 = min, 1 = max);
+    returns ``[n]``.
+    """
+    q_row = np.asarray(q_row, dtype=np.float64)
+    mm = np.asarray(minmax_rows, dtype=np.float64)
+    return np.maximum(mm[:, 0, :] * q_row, mm[:, 1, :] * q_row).sum(axis=1)
+
+
 def gate_scores_row(q_row, means_rows):
     """Gate affinities of one query row against a list of block means.
 
@@ -158,12 +195,15 @@ def select_blocks(q, means, cu_seqlens, chunk, topk):
     return sel
 
 
-def select_blocks_rows(q, means, cu_seqlens, chunk, topk, rows):
+def select_blocks_rows(q, means, cu_seqlens, chunk, topk, rows, score=gate_scores_row):
     """Selection for a list of ``(t, h)`` rows, one row at a time.
 
     Same definition as :func:`select_blocks` (the analysis, §2.2-§2.3), for
-    sampled rows of inputs too large to select in full.  Returns
-    ``[len(rows), topk]`` int64.
+    sampled rows of inputs too large to select in full.  ``means`` is the block
+    summary indexed ``[block, kv_head, ...]`` and ``score(q_row, summaries)``
+    the gate affinity: the mean gate by default, or the stacked
+    ``[NB, Hkv, 2, d]`` min/max summary with :func:`minmax_scores_row`.
+    Returns ``[len(rows), topk]`` int64.
     """
     means = np.asarray(means)
     Hq, Hkv = q.shape[1], means.shape[1]
@@ -178,8 +218,7 @@ def select_blocks_rows(q, means, cu_seqlens, chunk, topk, rows):
         b0 = int(tab["cu_blocks"][i])
         n_route = min(topk - 1, c)
         if n_route > 0:
-            sc = gate_scores_row(q[t, h].astype(np.float64),
-                                 means[b0:b0 + c, h // group].astype(np.float64))
+            sc = score(q[t, h].astype(np.float64), means[b0:b0 + c, h // group].astype(np.float64))
             out[r, :n_route] = _route_past(sc[None, :], n_route)[0]
         out[r, n_route] = c
     return out
@@ -320,7 +359,7 @@ class _LastRowQueries:
         return self.q_new[self.row_of[int(t)], h]
 
 
-def moba_decode(q_new, k, v, cu_seqlens, chunk, topk, scale=None):
+def moba_decode(q_new, k, v, cu_seqlens, chunk, topk, scale=None, gate="mean"):
     """Decode step: one new query per sequence against its KV cache.
 
     The cache of sequence b is rows ``cu[b] .. cu[b+1]-1`` of ``k`` / ``v``; its last row is
@@ -329,6 +368,9 @@ def moba_decode(q_new, k, v, cu_seqlens, chunk, topk, scale=None):
     ``c = (t - cu[b]) // chunk`` is forced (all cached tokens of that block precede or equal t),
     the ``topk - 1`` best earlier blocks by ``q . mean_j`` are routed, and the softmax runs over
     the union.  This is exactly the prefill forward's row t, computed row by row.
+
+    ``gate="minmax"`` scores the earlier blocks with the min/max summary instead
+    (:func:`block_minmax`, :func:`minmax_scores_row`); everything else is unchanged.
 
     ``q_new`` is ``[batch, Hq, d]``.  Returns ``out [batch, Hq, d]``, ``lse [Hq, batch]`` and
     ``sel [batch, Hq, topk]`` (float64 / int64); an empty sequence has no query: zeros, -inf
@@ -346,8 +388,14 @@ def moba_decode(q_new, k, v, cu_seqlens, chunk, topk, scale=None):
     if not rows:
         return {"out": out, "lse": lse, "sel": sel}
     qv = _LastRowQueries(q_new, cu)
-    means = block_means(k, cu, chunk)
-    s_rows = select_blocks_rows(qv, means, cu, chunk, topk, rows)
+    if gate == "mean":
+        s_rows = select_blocks_rows(qv, block_means(k, cu, chunk), cu, chunk, topk, rows)
+    elif gate == "minmax":
+        kmin, kmax = block_minmax(k, cu, chunk)
+        s_rows = select_blocks_rows(qv, np.stack([kmin, kmax], axis=2), cu, chunk, topk, rows,
+                                    score=minmax_scores_row)
+    else:
+        raise ValueError("gate must be 'mean' or 'minmax'")
     o_rows, l_rows = attend_rows(qv, k, v, cu, chunk, s_rows, rows, scale)
     for r, (t, h) in enumerate(rows):
         b = qv.row_of[t]

@@ -435,3 +435,127 @@ def test_decode_with_every_block_selected_is_dense_attention_of_the_last_row():
             z = (kt[0, 0] @ qt[0, 0, 0]) * scale
             np.testing.assert_allclose(dec["out"][b, h], o[0, 0, 0].numpy(), rtol=0, atol=1e-12)
             assert abs(dec["lse"][h, b] - torch.logsumexp(z, 0).item()) < 1e-12
+
+
+# ---- min/max (Quest-style) gate: block_minmax, minmax_scores_row, moba_decode(gate="minmax")
+
+def _corner_max(q_row, lo, hi):
+    """max of <q, x> over the box lo <= x <= hi, by enumerating its 2^d corners."""
+    best = -np.inf
+    for pick in itertools.product((0, 1), repeat=len(q_row)):
+        x = np.where(np.array(pick) == 1, hi, lo)
+        best = max(best, float(np.dot(q_row, x)))
+    return best
+
+
+def test_minmax_score_is_the_largest_inner_product_over_the_box():
+    """The score equals the maximum of <q, x> over the box's corners (a linear function
+    peaks at a corner), bounds <q, k> of every key of the block from above, and equals
+    <q, k> for a one-token block."""
+    rng = np.random.default_rng(11)
+    for trial in range(60):
+        d = int(rng.integers(1, 6))
+        n = int(rng.integers(1, 7))
+        keys = rng.standard_normal((n, 1, d))
+        q = rng.standard_normal(d)
+        q[rng.random(d) < 0.2] = 0.0
+        kmin, kmax = oracle.block_minmax(keys, np.array([0, n]), n)
+        s = oracle.minmax_scores_row(q, np.stack([kmin[:, 0], kmax[:, 0]], axis=1))[0]
+        assert abs(s - _corner_max(q, kmin[0, 0], kmax[0, 0])) < 1e-12, trial
+        assert s >= max(float(q @ keys[i, 0]) for i in range(n)) - 1e-12
+        if n == 1:
+            assert abs(s - float(q @ keys[0, 0])) < 1e-12
+
+
+def test_block_minmax_closed_forms():
+    """Keys linear in the position inside their sequence: each channel's minimum and
+    maximum sit at the block's first or last valid row, by the sign of the slope; the
+    partial final block and a one-token block included."""
+    seqlens, chunk, hkv, d = [23, 1, 16], 8, 2, 3
+    cu = np.concatenate([[0], np.cumsum(seqlens)])
+    slope = np.array([[1.5, -2.0, 0.0], [-0.25, 3.0, 1.0]])
+    off = np.array([[0.5, 1.0, -7.0], [2.0, -1.0, 0.0]])
+    k = np.zeros((int(cu[-1]), hkv, d))
+    for b, n in enumerate(seqlens):
+        for p in range(n):
+            k[cu[b] + p] = slope * p + off
+    kmin, kmax = oracle.block_minmax(k, cu, chunk)
+    blk = 0
+    for b, n in enumerate(seqlens):
+        for j in range(-(-n // chunk)):
+            first, last = j * chunk, min((j + 1) * chunk, n) - 1
+            a, z = slope * first + off, slope * last + off
+            np.testing.assert_array_equal(kmin[blk], np.minimum(a, z))
+            np.testing.assert_array_equal(kmax[blk], np.maximum(a, z))
+            blk += 1
+    assert blk == kmin.shape[0] == 3 + 1 + 2
+
+
+def test_minmax_decode_selection_matches_brute_force():
+    """Decode with the min/max gate routes the (k-1)-subset of earlier blocks with the
+    largest sum of box maxima (block summaries restated from the keys, scores from the
+    corners), over varlen caches, GQA and empty caches."""
+    rng = np.random.default_rng(12)
+    for trial in range(25):
+        hq, hkv, d = 4, 2, 3
+        chunk = int(rng.integers(1, 5))
+        seqlens = [int(x) for x in rng.integers(0, 20, size=3)]
+        topk = int(rng.integers(1, 5))
+        cu, q, k, v, q_new = _decode_inputs(seqlens, hq, hkv, d, 100 + trial)
+        dec = oracle.moba_decode(q_new, k, v, cu, chunk, topk, gate="minmax")
+        for b, n in enumerate(seqlens):
+            if n == 0:
+                assert np.all(dec["sel"][b] == -1)
+                continue
+            s = int(cu[b])
+            c = (n - 1) // chunk
+            for h in range(hq):
+                g = h // (hq // hkv)
+                score = []
+                for j in range(c):
+                    rows = k[s + j * chunk:s + (j + 1) * chunk, g]
+                    score.append(_corner_max(q_new[b, h], rows.min(axis=0), rows.max(axis=0)))
+                m = min(topk - 1, c)
+                best, best_set = -np.inf, ()
+                for subset in itertools.combinations(range(c), m):
+                    val = sum(score[j] for j in subset)
+                    if val > best:
+                        best, best_set = val, subset
+                expect = sorted(best_set) + [c] + [-1] * (topk - m - 1)
+                assert list(dec["sel"][b, h]) == expect, (trial, b, h)
+
+
+def test_minmax_gate_finds_the_single_matching_key_the_mean_dilutes():
+    """The case the analysis (§5.1 item 6) gives for a stronger summary: block 1 holds one
+    key aligned with q among zeros, so its mean (4/16) loses to block 0's uniform 0.5 while
+    its box maximum (4) wins.  The output is softmax attention over blocks {1, 3} (torch
+    fp64 SDPA)."""
+    chunk, d = 16, 2
+    k = np.zeros((53, 1, d))
+    k[0:16, 0] = [0.5, 0.0]
+    k[16 + 7, 0] = [4.0, 0.0]
+    k[32:48, 0] = [-1.0, 0.0]
+    k[48:53, 0] = [0.0, 1.0]
+    v = np.random.default_rng(3).standard_normal((53, 1, d))
+    cu = np.array([0, 53])
+    q_new = np.array([[[1.0, 0.0]]])
+    mean_dec = oracle.moba_decode(q_new, k, v, cu, chunk, 2)
+    mm_dec = oracle.moba_decode(q_new, k, v, cu, chunk, 2, gate="minmax")
+    assert list(mean_dec["sel"][0, 0]) == [0, 3]
+    assert list(mm_dec["sel"][0, 0]) == [1, 3]
+    keys = np.r_[16:32, 48:53]
+    qt = torch.tensor(q_new[0, 0])[None, None, None]
+    kt = torch.from_numpy(k[keys, 0])[None, None]
+    vt = torch.from_numpy(v[keys, 0])[None, None]
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=1 / math.sqrt(d))
+    np.testing.assert_allclose(mm_dec["out"][0, 0], o[0, 0, 0].numpy(), rtol=0, atol=1e-12)
+
+
+def test_minmax_decode_with_every_block_selected_equals_the_mean_gate():
+    """topk >= blocks: the gate decides nothing, so both summaries give the same step."""
+    cu, q, k, v, q_new = _decode_inputs([300, 77, 0], 4, 1, 8, 9)
+    a = oracle.moba_decode(q_new, k, v, cu, 32, 16)
+    b = oracle.moba_decode(q_new, k, v, cu, 32, 16, gate="minmax")
+    assert np.array_equal(a["sel"], b["sel"])
+    np.testing.assert_array_equal(a["out"], b["out"])
+    np.testing.assert_array_equal(a["lse"], b["lse"])
