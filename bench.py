@@ -424,14 +424,21 @@ def run_decode(args, w, world, rank, local):
     chunk, topk = w.chunk_size, w.topk
     last = torch.tensor([c - 1 for c in w.cu_seqlens[1:]], device=dev)
     q_new = x["q"][last].contiguous()
-    means = moba.meanpool(k, cu, chunk)  # cache state, kept outside the timed step
+    # cache state, kept outside the timed step: the block means or the min/max summary
+    if args.gate == "minmax":
+        k_min, k_max = moba.minmaxpool(k, cu, chunk)
+    else:
+        means = moba.meanpool(k, cu, chunk)
     p = moba.make_params(B, w.total_tokens, hq, hkv, d, chunk, topk)
     ws = torch.empty(moba.load_library().moba_decode_workspace_size(p), dtype=torch.uint8, device=dev)
     out = torch.empty((B, hq, d), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((hq, B), dtype=torch.float32, device=dev)
 
     def step():
-        moba.decode_fwd(q_new, k, v, cu, means, chunk, topk, workspace=ws, out=out, lse=lse)
+        if args.gate == "minmax":
+            moba.decode_minmax_fwd(q_new, k, v, cu, k_min, k_max, chunk, topk, workspace=ws, out=out, lse=lse)
+        else:
+            moba.decode_fwd(q_new, k, v, cu, means, chunk, topk, workspace=ws, out=out, lse=lse)
 
     for _ in range(args.warmup):
         step()
@@ -493,10 +500,10 @@ def run_decode(args, w, world, rank, local):
         vh = v[:n0].double().cpu().numpy()
         qh1 = q_new[:1].double().cpu().numpy()
         t0 = time.time()
-        oracle.moba_decode(qh1, kh, vh, [0, n0], chunk, topk)
+        oracle.moba_decode(qh1, kh, vh, [0, n0], chunk, topk, gate=args.gate)
         dt = time.time() - t0
         cpu = {"value": 1.0 / dt, "unit": "sequences/s", "cores": os.cpu_count(), "kind": "oracle",
-               "sample": f"1 of {B} sequences (its whole {n0}-token cache: block means, gate, attention)"}
+               "sample": f"1 of {B} sequences (its whole {n0}-token cache: block summary, gate, attention)"}
 
     if rank == 0:
         line = {
@@ -515,7 +522,10 @@ def run_decode(args, w, world, rank, local):
             "config": {"workload": w.name, "description": w.description, "sequences": B,
                        "cache_tokens": w.total_tokens, "q_heads": hq, "kv_heads": hkv,
                        "head_dim": d, "chunk_size": chunk, "topk": topk,
-                       "means": "cached block means (moba_meanpool once, outside the step)",
+                       "gate": args.gate,
+                       "block_summary": ("cached bf16 block min/max (moba_minmaxpool once, outside the step)"
+                                         if args.gate == "minmax" else
+                                         "cached block means (moba_meanpool once, outside the step)"),
                        "l2": "caches larger than L2 (no flush)", "parallelism": f"dp{world}"},
             "roofline": {"bound": "hbm", "kernel": "decode step (gate, block attention, merge)",
                          "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -548,10 +558,10 @@ def run_decode_reference(args, w, world, rank):
     k = x["k"].double().numpy()
     v = x["v"].double().numpy()
     q1 = x["q"][n0 - 1:n0].double().numpy()
-    oracle.moba_decode(q1, k, v, [0, n0], w.chunk_size, w.topk)  # warm-up
+    oracle.moba_decode(q1, k, v, [0, n0], w.chunk_size, w.topk, gate=args.gate)  # warm-up
     t0 = time.time()
     for _ in range(args.steps):
-        oracle.moba_decode(q1, k, v, [0, n0], w.chunk_size, w.topk)
+        oracle.moba_decode(q1, k, v, [0, n0], w.chunk_size, w.topk, gate=args.gate)
     dt = (time.time() - t0) / args.steps
     value = 1.0 / dt
     print(json.dumps({
@@ -560,7 +570,7 @@ def run_decode_reference(args, w, world, rank):
         "value": value, "unit": "sequences/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-        "config": {"workload": w.name, "description": w.description},
+        "config": {"workload": w.name, "description": w.description, "gate": args.gate},
         "cpu_baseline": {"value": value, "unit": "sequences/s", "cores": os.cpu_count(),
                          "kind": "oracle", "sample": f"1 of {len(w.seqlens)} sequences per step"},
         "e2e": {"value": value, "unit": "sequences/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -646,6 +656,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--decode", action="store_true",
                     help="time the decode step (workloads.DECODE_WORKLOADS) instead of the prefill")
+    ap.add_argument("--gate", choices=["mean", "minmax"], default="mean",
+                    help="decode gate: block means, or the min/max (Quest-style) block summary")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -5,9 +5,11 @@
 // c = (L-1) / B is forced and attended whole (every cached token of it precedes or equals t),
 // the topk-1 best earlier blocks by q . mean_j are routed, and softmax attention runs over the
 // union; per-block partial results are merged by their log-sum-exp (§3.2).  The means are the
-// cached fp32 block means of moba_meanpool over the same caches.  There is one query row per
-// (sequence, head), so the step streams whole K/V blocks and is HBM-bound: it runs on the CUDA
-// cores.
+// cached fp32 block means of moba_meanpool over the same caches.  The gate may instead score
+// with the min/max block summary of moba_minmaxpool: the Quest variant the analysis names
+// (§1.3, §5.1 item 6), s_j = sum_i max(q_i kmin_ji, q_i kmax_ji), the largest q . x over the
+// block's bounding box.  There is one query row per (sequence, head), so the step streams
+// whole K/V blocks and is HBM-bound: it runs on the CUDA cores.
 //   decode_gate_kernel   one warp per (sequence, query head): fp32 scores, top-(k-1)
 //   decode_attn_kernel   one CTA per (slot, key range, query head, sequence): a selected
 //                        block's keys in tiles (a block is cut into several ranges when there
@@ -41,11 +43,60 @@ __device__ __forceinline__ int seq_block_base(const int* __restrict__ cu, int se
     return base;
 }
 
+// Gate score of one block summary row (global block x KV head) for the fp32 query qs[D].
+// Mean gate (analysis §2.2): q . mean, fp32 means.
+template <int D>
+struct MeanScore {
+    const float* means;
+    __device__ __forceinline__ float operator()(const float* qs, size_t row) const {
+        const float4* m = reinterpret_cast<const float4*>(means + row * D);
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 8
+        for (int e = 0; e < D / 4; ++e) {
+            const float4 mv = __ldg(m + e);
+            a0 = fmaf(qs[4 * e], mv.x, a0);
+            a1 = fmaf(qs[4 * e + 1], mv.y, a1);
+            a2 = fmaf(qs[4 * e + 2], mv.z, a2);
+            a3 = fmaf(qs[4 * e + 3], mv.w, a3);
+        }
+        return (a0 + a1) + (a2 + a3);
+    }
+};
+
+// Min/max gate (Quest): sum over channels of max(q_i kmin_i, q_i kmax_i).  q and the
+// summaries are bf16 values, so every product is exact in fp32; only the sum rounds.
+__device__ __forceinline__ float box_pair(float q0, float q1, uint32_t lo, uint32_t hi) {
+    const float t0 = fmaxf(q0 * __uint_as_float(lo << 16), q0 * __uint_as_float(hi << 16));
+    const float t1 = fmaxf(q1 * __uint_as_float(lo & 0xffff0000u), q1 * __uint_as_float(hi & 0xffff0000u));
+    return t0 + t1;
+}
+
+template <int D>
+struct MinMaxScore {
+    const __nv_bfloat16* kmin;
+    const __nv_bfloat16* kmax;
+    __device__ __forceinline__ float operator()(const float* qs, size_t row) const {
+        const uint4* lo = reinterpret_cast<const uint4*>(kmin + row * D);
+        const uint4* hi = reinterpret_cast<const uint4*>(kmax + row * D);
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 8
+        for (int e = 0; e < D / 8; ++e) {
+            const uint4 l = __ldg(lo + e), h = __ldg(hi + e);
+            const float* qe = qs + 8 * e;
+            a0 += box_pair(qe[0], qe[1], l.x, h.x);
+            a1 += box_pair(qe[2], qe[3], l.y, h.y);
+            a2 += box_pair(qe[4], qe[5], l.z, h.z);
+            a3 += box_pair(qe[6], qe[7], l.w, h.w);
+        }
+        return (a0 + a1) + (a2 + a3);
+    }
+};
+
 // sel row of (sequence, head) w: slot 0 = own block c, slots 1..n_route = routed past blocks
 // (best first), then -1; nsl[w] = 1 + n_route (0 for an empty sequence).
-template <int D, int K>
+template <int D, int K, class Score>
 __global__ void __launch_bounds__(kGateWarps * 32)
-decode_gate_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ means,
+decode_gate_kernel(const __nv_bfloat16* __restrict__ q, Score score,
                    const int* __restrict__ cu, Problem P, int* __restrict__ sel,
                    int* __restrict__ nsl) {
     __shared__ float qs[kGateWarps][D];
@@ -75,19 +126,8 @@ decode_gate_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict_
             val[i] = -INFINITY;
             idx[i] = INT_MAX;
         }
-        for (int j = lane; j < c; j += 32) {
-            const float4* m = reinterpret_cast<const float4*>(means + ((size_t)(b0 + j) * P.hkv + g) * D);
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 8
-            for (int e = 0; e < D / 4; ++e) {
-                const float4 mv = __ldg(m + e);
-                a0 = fmaf(qs[warp][4 * e], mv.x, a0);
-                a1 = fmaf(qs[warp][4 * e + 1], mv.y, a1);
-                a2 = fmaf(qs[warp][4 * e + 2], mv.z, a2);
-                a3 = fmaf(qs[warp][4 * e + 3], mv.w, a3);
-            }
-            insert_desc<K>(val, idx, (a0 + a1) + (a2 + a3), j, true);
-        }
+        for (int j = lane; j < c; j += 32)
+            insert_desc<K>(val, idx, score(qs[warp], (size_t)(b0 + j) * P.hkv + g), j, true);
         // n_route rounds of a warp argmax over the lists' heads, order (score desc, index asc)
         for (int r = 0; r < n_route; ++r) {
             float bv = val[0];
@@ -285,22 +325,32 @@ decode_merge_kernel(const int* __restrict__ nsl, const float* __restrict__ part_
     if (lane == 0) lse[(size_t)h * P.batch + seq] = mx + logf(L);
 }
 
+template <int D, class Score>
+void launch_decode_gate(const Problem& P, const __nv_bfloat16* q, Score score, const int* cu,
+                        const DecodeWorkspace& ws, cudaStream_t st) {
+    const int row_blocks = (P.batch * P.hq + kGateWarps - 1) / kGateWarps;
+    const int route = P.topk - 1;  // list size must hold every routed block of one lane
+    if (route <= 4)
+        decode_gate_kernel<D, 4><<<row_blocks, kGateWarps * 32, 0, st>>>(q, score, cu, P, ws.sel, ws.nsl);
+    else if (route <= 8)
+        decode_gate_kernel<D, 8><<<row_blocks, kGateWarps * 32, 0, st>>>(q, score, cu, P, ws.sel, ws.nsl);
+    else if (route <= 16)
+        decode_gate_kernel<D, 16><<<row_blocks, kGateWarps * 32, 0, st>>>(q, score, cu, P, ws.sel, ws.nsl);
+    else
+        decode_gate_kernel<D, 32><<<row_blocks, kGateWarps * 32, 0, st>>>(q, score, cu, P, ws.sel, ws.nsl);
+}
+
 template <int D>
 cudaError_t launch_decode_d(const Problem& P, const __nv_bfloat16* q, const __nv_bfloat16* k,
-                            const __nv_bfloat16* v, const int* cu, const float* means,
+                            const __nv_bfloat16* v, const int* cu, const DecodeGate& gate,
                             const DecodeWorkspace& ws, __nv_bfloat16* out, float* lse,
                             cudaStream_t st) {
     const int rows = P.batch * P.hq;
     const int row_blocks = (rows + kGateWarps - 1) / kGateWarps;
-    const int route = P.topk - 1;  // list size must hold every routed block of one lane
-    if (route <= 4)
-        decode_gate_kernel<D, 4><<<row_blocks, kGateWarps * 32, 0, st>>>(q, means, cu, P, ws.sel, ws.nsl);
-    else if (route <= 8)
-        decode_gate_kernel<D, 8><<<row_blocks, kGateWarps * 32, 0, st>>>(q, means, cu, P, ws.sel, ws.nsl);
-    else if (route <= 16)
-        decode_gate_kernel<D, 16><<<row_blocks, kGateWarps * 32, 0, st>>>(q, means, cu, P, ws.sel, ws.nsl);
+    if (gate.means)
+        launch_decode_gate<D>(P, q, MeanScore<D>{gate.means}, cu, ws, st);
     else
-        decode_gate_kernel<D, 32><<<row_blocks, kGateWarps * 32, 0, st>>>(q, means, cu, P, ws.sel, ws.nsl);
+        launch_decode_gate<D>(P, q, MinMaxScore<D>{gate.kmin, gate.kmax}, cu, ws, st);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     decode_attn_kernel<D><<<dim3(P.topk * ws.splits, P.hq, P.batch), kAttnThreads, 0, st>>>(
@@ -315,11 +365,11 @@ cudaError_t launch_decode_d(const Problem& P, const __nv_bfloat16* q, const __nv
 }  // namespace
 
 cudaError_t launch_decode(const Problem& P, const __nv_bfloat16* q, const __nv_bfloat16* k,
-                          const __nv_bfloat16* v, const int* cu_seqlens, const float* means,
+                          const __nv_bfloat16* v, const int* cu_seqlens, const DecodeGate& gate,
                           const DecodeWorkspace& ws, __nv_bfloat16* out, float* lse,
                           cudaStream_t st) {
-    if (P.d == 64) return launch_decode_d<64>(P, q, k, v, cu_seqlens, means, ws, out, lse, st);
-    return launch_decode_d<128>(P, q, k, v, cu_seqlens, means, ws, out, lse, st);
+    if (P.d == 64) return launch_decode_d<64>(P, q, k, v, cu_seqlens, gate, ws, out, lse, st);
+    return launch_decode_d<128>(P, q, k, v, cu_seqlens, gate, ws, out, lse, st);
 }
 
 }  // namespace moba

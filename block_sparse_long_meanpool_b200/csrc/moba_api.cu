@@ -187,6 +187,22 @@ moba_status moba_meanpool(const moba_params* p, const void* k, const int* cu_seq
     return MOBA_OK;
 }
 
+moba_status moba_minmaxpool(const moba_params* p, const void* k, const int* cu_seqlens,
+                            void* k_min, void* k_max, void* stream) {
+    moba_status s = check_params(p);
+    if (s != MOBA_OK) return s;
+    if (p->total_tokens == 0) return MOBA_OK;
+    if (!k || !cu_seqlens || !k_min || !k_max) return fail(MOBA_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned16(k) || !aligned16(k_min) || !aligned16(k_max))
+        return fail(MOBA_ERR_INVALID_ARG, "k, k_min and k_max must be 16-byte aligned");
+    const Problem P = make_problem(*p, blocks_bound(*p));
+    cudaError_t e = launch_minmaxpool(P, static_cast<const __nv_bfloat16*>(k), cu_seqlens,
+                                      static_cast<__nv_bfloat16*>(k_min), static_cast<__nv_bfloat16*>(k_max),
+                                      static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "minmaxpool launch");
+    return MOBA_OK;
+}
+
 moba_status moba_gate_topk(const moba_params* p, const void* q, const float* k_mean,
                            const int* cu_seqlens, int* sel, void* stream) {
     moba_status s = check_params(p);
@@ -340,18 +356,23 @@ size_t moba_decode_workspace_size(const moba_params* p) {
     return make_decode_layout(*p).total;
 }
 
-moba_status moba_decode_fwd(const moba_params* p, const void* q, const void* k, const void* v,
-                            const int* cu_seqlens, const float* k_mean, void* workspace,
-                            size_t ws_bytes, void* out, float* lse, void* stream) {
+namespace {
+
+// The decode step with either block summary (gate.means, or gate.kmin and gate.kmax).
+moba_status decode_fwd(const moba_params* p, const void* q, const void* k, const void* v,
+                       const int* cu_seqlens, const DecodeGate& gate, void* workspace,
+                       size_t ws_bytes, void* out, float* lse, void* stream) {
     moba_status s = check_params(p);
     if (s != MOBA_OK) return s;
     if (p->batch > 65535)
         return fail(MOBA_ERR_UNSUPPORTED, "decode batch %d unsupported (<= 65535)", p->batch);
-    if (!q || !cu_seqlens || !workspace || !out || !lse || (p->total_tokens > 0 && (!k || !v || !k_mean)))
+    const bool summary = gate.means || (gate.kmin && gate.kmax);
+    if (!q || !cu_seqlens || !workspace || !out || !lse || (p->total_tokens > 0 && (!k || !v || !summary)))
         return fail(MOBA_ERR_INVALID_ARG, "NULL pointer argument");
     if (!aligned16(q) || !aligned16(out) || !aligned16(workspace) ||
-        (p->total_tokens > 0 && (!aligned16(k) || !aligned16(v) || !aligned16(k_mean))))
-        return fail(MOBA_ERR_INVALID_ARG, "q, k, v, k_mean, out and workspace must be 16-byte aligned");
+        (p->total_tokens > 0 && (!aligned16(k) || !aligned16(v) || !aligned16(gate.means) ||
+                                 !aligned16(gate.kmin) || !aligned16(gate.kmax))))
+        return fail(MOBA_ERR_INVALID_ARG, "q, k, v, the block summary, out and workspace must be 16-byte aligned");
     const DecodeLayout L = make_decode_layout(*p);
     if (ws_bytes < L.total)
         return fail(MOBA_ERR_WORKSPACE, "decode workspace too small: %zu < %zu bytes", ws_bytes, L.total);
@@ -364,10 +385,29 @@ moba_status moba_decode_fwd(const moba_params* p, const void* q, const void* k, 
     ws.part_lse = reinterpret_cast<float*>(base + L.part_lse);
     ws.splits = decode_splits(p->batch, p->num_q_heads, p->topk, p->chunk_size);
     cudaError_t e = launch_decode(P, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                                  static_cast<const __nv_bfloat16*>(v), cu_seqlens, k_mean, ws,
+                                  static_cast<const __nv_bfloat16*>(v), cu_seqlens, gate, ws,
                                   static_cast<__nv_bfloat16*>(out), lse, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     return MOBA_OK;
+}
+
+}  // namespace
+
+moba_status moba_decode_fwd(const moba_params* p, const void* q, const void* k, const void* v,
+                            const int* cu_seqlens, const float* k_mean, void* workspace,
+                            size_t ws_bytes, void* out, float* lse, void* stream) {
+    return decode_fwd(p, q, k, v, cu_seqlens, DecodeGate{k_mean, nullptr, nullptr}, workspace, ws_bytes,
+                      out, lse, stream);
+}
+
+moba_status moba_decode_minmax_fwd(const moba_params* p, const void* q, const void* k, const void* v,
+                                   const int* cu_seqlens, const void* k_min, const void* k_max,
+                                   void* workspace, size_t ws_bytes, void* out, float* lse,
+                                   void* stream) {
+    return decode_fwd(p, q, k, v, cu_seqlens,
+                      DecodeGate{nullptr, static_cast<const __nv_bfloat16*>(k_min),
+                                 static_cast<const __nv_bfloat16*>(k_max)},
+                      workspace, ws_bytes, out, lse, stream);
 }
 
 moba_status moba_device_status(const moba_params* p, const void* workspace, void* stream) {

@@ -148,6 +148,8 @@ cudaError_t launch_plan_blocks(const Problem& P, const int* cu_seqlens, const Wo
                                cudaStream_t st);
 cudaError_t launch_meanpool(const Problem& P, const __nv_bfloat16* k, const int* cu_seqlens,
                             float* means, cudaStream_t st);
+cudaError_t launch_minmaxpool(const Problem& P, const __nv_bfloat16* k, const int* cu_seqlens,
+                              __nv_bfloat16* kmin, __nv_bfloat16* kmax, cudaStream_t st);
 cudaError_t launch_gate(const Problem& P, const __nv_bfloat16* q, const float* means,
                         const int* cu_seqlens, int* sel, cudaStream_t st);
 cudaError_t launch_gate_best(const Problem& P, const __nv_bfloat16* q, const float* means,
@@ -181,8 +183,15 @@ inline int decode_splits(int batch, int hq, int topk, int chunk) {
     while ((long long)batch * hq * topk * s < 1184 && topk * s * 2 <= 64 && chunk / (s * 2) >= 128) s *= 2;
     return s;
 }
+// Block summary the decode gate scores against: the fp32 means (kmin == kmax == nullptr) or
+// the bf16 min/max pair (means == nullptr), each [NB, Hkv, d].
+struct DecodeGate {
+    const float* means;
+    const __nv_bfloat16* kmin;
+    const __nv_bfloat16* kmax;
+};
 cudaError_t launch_decode(const Problem& P, const __nv_bfloat16* q, const __nv_bfloat16* k,
-                          const __nv_bfloat16* v, const int* cu_seqlens, const float* means,
+                          const __nv_bfloat16* v, const int* cu_seqlens, const DecodeGate& gate,
                           const DecodeWorkspace& ws, __nv_bfloat16* out, float* lse,
                           cudaStream_t st);
 

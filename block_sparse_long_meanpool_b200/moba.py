@@ -19,11 +19,13 @@ EXPORTS = (
     "moba_num_blocks_bound",
     "moba_workspace_size",
     "moba_meanpool",
+    "moba_minmaxpool",
     "moba_gate_topk",
     "moba_attn_fwd",
     "moba_attn_fwd_noalloc",
     "moba_decode_workspace_size",
     "moba_decode_fwd",
+    "moba_decode_minmax_fwd",
     "moba_device_status",
     "moba_selftest_timeout",
     "moba_status_string",
@@ -86,6 +88,8 @@ def load_library(path=LIB_PATH):
     lib.moba_workspace_size.restype = ctypes.c_size_t
     lib.moba_meanpool.argtypes = [P, vp, vp, vp, vp]
     lib.moba_meanpool.restype = ctypes.c_int
+    lib.moba_minmaxpool.argtypes = [P, vp, vp, vp, vp, vp]
+    lib.moba_minmaxpool.restype = ctypes.c_int
     lib.moba_gate_topk.argtypes = [P, vp, vp, vp, vp, vp]
     lib.moba_gate_topk.restype = ctypes.c_int
     lib.moba_attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp,
@@ -97,6 +101,8 @@ def load_library(path=LIB_PATH):
     lib.moba_decode_workspace_size.restype = ctypes.c_size_t
     lib.moba_decode_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp, vp]
     lib.moba_decode_fwd.restype = ctypes.c_int
+    lib.moba_decode_minmax_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp, vp]
+    lib.moba_decode_minmax_fwd.restype = ctypes.c_int
     lib.moba_device_status.argtypes = [P, vp, vp]
     lib.moba_device_status.restype = ctypes.c_int
     lib.moba_selftest_timeout.argtypes = [vp, ctypes.c_uint, vp]
@@ -179,6 +185,20 @@ def meanpool(k, cu_seqlens, chunk_size, num_blocks_out=None):
     return out[:nb]
 
 
+def minmaxpool(k, cu_seqlens, chunk_size, num_blocks_out=None):
+    """Min/max block summary (moba_minmaxpool): (k_min, k_max), bf16 [NB, Hkv, d] each."""
+    _check_qkv(None, k)
+    batch = cu_seqlens.numel() - 1
+    T, hkv, d = k.shape
+    p = make_params(batch, T, hkv, hkv, d, chunk_size, 1)
+    nb = num_blocks_out if num_blocks_out is not None else max(load_library().moba_num_blocks_bound(ctypes.byref(p)), 0)
+    k_min = torch.empty((max(nb, 1), hkv, d), dtype=torch.bfloat16, device=k.device)
+    k_max = torch.empty_like(k_min)
+    _check(load_library().moba_minmaxpool(ctypes.byref(p), _ptr(k), _ptr(cu_seqlens), _ptr(k_min),
+                                          _ptr(k_max), _stream(k.device)))
+    return k_min[:nb], k_max[:nb]
+
+
 def gate_topk(q, k_mean, cu_seqlens, chunk_size, topk, num_kv_heads=None):
     """Selections int32 [Hq, T, topk] (moba_gate_topk)."""
     _check_qkv(q, None)
@@ -193,22 +213,12 @@ def gate_topk(q, k_mean, cu_seqlens, chunk_size, topk, num_kv_heads=None):
     return sel
 
 
-def decode_fwd(q, k, v, cu_seqlens, k_mean, chunk_size, topk, softmax_scale=None,
-               workspace=None, out=None, lse=None):
-    """Decode step (moba_decode_fwd): one new query per sequence against its KV cache.
-
-    q bf16 [batch, Hq, d] (the new token's query of each sequence); k, v bf16 [T, Hkv, d]
-    packed caches whose last row per sequence is the new token; cu_seqlens int32 [batch + 1];
-    k_mean fp32 block means of these caches (``meanpool``).  Returns (out bf16 [batch, Hq, d],
-    lse fp32 [Hq, batch]).
-    """
+def _decode(fn, summary, q, k, v, cu_seqlens, chunk_size, topk, softmax_scale, workspace, out, lse):
     _check_qkv(q, k, v)
     batch, hq, d = q.shape
     T, hkv, _ = k.shape
     _require(cu_seqlens.is_cuda and cu_seqlens.dtype == torch.int32 and cu_seqlens.numel() == batch + 1,
              "cu_seqlens must be a CUDA int32 tensor of batch + 1 entries")
-    _require(k_mean.is_cuda and k_mean.dtype == torch.float32 and k_mean.is_contiguous(),
-             "k_mean must be a contiguous CUDA fp32 tensor")
     p = make_params(batch, T, hq, hkv, d, chunk_size, topk, softmax_scale)
     lib = load_library()
     n = lib.moba_decode_workspace_size(ctypes.byref(p))
@@ -220,10 +230,36 @@ def decode_fwd(q, k, v, cu_seqlens, k_mean, chunk_size, topk, softmax_scale=None
         out = torch.empty((batch, hq, d), dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty((hq, batch), dtype=torch.float32, device=q.device)
-    _check(lib.moba_decode_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens),
-                               _ptr(k_mean), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
-                               _ptr(out), _ptr(lse), _stream(q.device)))
+    _check(getattr(lib, fn)(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens),
+                            *[_ptr(t) for t in summary], _ptr(workspace),
+                            ctypes.c_size_t(workspace.numel()), _ptr(out), _ptr(lse), _stream(q.device)))
     return out, lse
+
+
+def decode_fwd(q, k, v, cu_seqlens, k_mean, chunk_size, topk, softmax_scale=None,
+               workspace=None, out=None, lse=None):
+    """Decode step (moba_decode_fwd): one new query per sequence against its KV cache.
+
+    q bf16 [batch, Hq, d] (the new token's query of each sequence); k, v bf16 [T, Hkv, d]
+    packed caches whose last row per sequence is the new token; cu_seqlens int32 [batch + 1];
+    k_mean fp32 block means of these caches (``meanpool``).  Returns (out bf16 [batch, Hq, d],
+    lse fp32 [Hq, batch]).
+    """
+    _require(k_mean.is_cuda and k_mean.dtype == torch.float32 and k_mean.is_contiguous(),
+             "k_mean must be a contiguous CUDA fp32 tensor")
+    return _decode("moba_decode_fwd", (k_mean,), q, k, v, cu_seqlens, chunk_size, topk,
+                   softmax_scale, workspace, out, lse)
+
+
+def decode_minmax_fwd(q, k, v, cu_seqlens, k_min, k_max, chunk_size, topk, softmax_scale=None,
+                      workspace=None, out=None, lse=None):
+    """Decode step with the min/max gate (moba_decode_minmax_fwd): as ``decode_fwd``, with the
+    bf16 block summary (k_min, k_max) of ``minmaxpool`` in place of the means."""
+    for t in (k_min, k_max):
+        _require(t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous(),
+                 "k_min and k_max must be contiguous CUDA bf16 tensors")
+    return _decode("moba_decode_minmax_fwd", (k_min, k_max), q, k, v, cu_seqlens, chunk_size, topk,
+                   softmax_scale, workspace, out, lse)
 
 
 def selftest_timeout(device=None, polls=4096):

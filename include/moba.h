@@ -108,6 +108,18 @@ size_t moba_workspace_size(const moba_params* p);
 moba_status moba_meanpool(const moba_params* p, const void* k, const int* cu_seqlens,
                           float* k_mean, void* stream);
 
+/* Min/max block summary, the Quest-style alternative to the mean (the analysis names Quest as
+ * the MoBA variant with min/max pooling, §1.3, and as the stronger summary, §5.1 item 6 and
+ * §6.3; the summary is Quest's): k_min[b, g, i] and k_max[b, g, i] = minimum and maximum of
+ * k[t, g, i] over the valid tokens t of block b.  Exact (the extrema of bf16 values are bf16).
+ *   k              bf16 [T, Hkv, d] device
+ *   cu_seqlens     int32 [batch + 1] device
+ *   k_min, k_max   bf16 [NB, Hkv, d] device each, NB as for moba_meanpool; rows past the true
+ *                  block count are left untouched
+ * Uses no workspace; asynchronous on `stream`; argument errors return before any launch. */
+moba_status moba_minmaxpool(const moba_params* p, const void* k, const int* cu_seqlens,
+                            void* k_min, void* k_max, void* stream);
+
 /* Steps 3-4 (analysis §2.2-§2.3): per query row, gate scores against the means of the past
  * blocks of its sequence (fp32), future blocks excluded, the own block forced, the best
  * topk-1 past blocks kept (ties to the lower block index).
@@ -165,6 +177,16 @@ size_t moba_decode_workspace_size(const moba_params* p);
 moba_status moba_decode_fwd(const moba_params* p, const void* q, const void* k, const void* v,
                             const int* cu_seqlens, const float* k_mean, void* workspace,
                             size_t ws_bytes, void* out, float* lse, void* stream);
+
+/* The decode step with the min/max gate: as moba_decode_fwd, except that an earlier block j
+ * is scored by s_j = sum_i max(q_i k_min[j, g, i], q_i k_max[j, g, i]) (fp32; Quest's bound of
+ * q . k over the block), from the summary moba_minmaxpool computes for these caches:
+ *   k_min, k_max   bf16 [moba_num_blocks_bound(p), Hkv, d] device each
+ * Same workspace (moba_decode_workspace_size), outputs, errors and limits. */
+moba_status moba_decode_minmax_fwd(const moba_params* p, const void* q, const void* k, const void* v,
+                                   const int* cu_seqlens, const void* k_min, const void* k_max,
+                                   void* workspace, size_t workspace_bytes, void* out, float* lse,
+                                   void* stream);
 
 /* ---- Self-test of the bounded device waits (no counterpart in the paper) ---------------
  *

@@ -171,6 +171,41 @@ def test_decode_checks_precede_any_launch(lib):
     assert rc == moba.ERR_UNSUPPORTED
 
 
+def test_minmax_argument_checks(lib):
+    p = params()
+    assert lib.moba_minmaxpool(None, None, None, None, None, None) == moba.ERR_INVALID_ARG
+    assert lib.moba_minmaxpool(ctypes.byref(p), None, None, None, None, None) == moba.ERR_INVALID_ARG
+    need = lib.moba_decode_workspace_size(ctypes.byref(p))
+    assert lib.moba_decode_minmax_fwd(None, None, None, None, None, None, None, None, 0, None, None,
+                                      None) == moba.ERR_INVALID_ARG
+    assert lib.moba_decode_minmax_fwd(ctypes.byref(p), None, None, None, None, None, None, None, need,
+                                      None, None, None) == moba.ERR_INVALID_ARG
+    bad = params(head_dim=96)
+    assert lib.moba_minmaxpool(ctypes.byref(bad), None, None, None, None, None) == moba.ERR_UNSUPPORTED
+
+
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="hands fake device addresses to the library: host-only check")
+def test_minmax_checks_precede_any_launch(lib):
+    p = params()
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    # k_max misaligned, k_min missing
+    assert lib.moba_minmaxpool(ctypes.byref(p), fake, fake, fake, odd, None) == moba.ERR_INVALID_ARG
+    assert lib.moba_minmaxpool(ctypes.byref(p), fake, fake, None, fake, None) == moba.ERR_INVALID_ARG
+    need = lib.moba_decode_workspace_size(ctypes.byref(p))
+    # only one half of the summary given
+    rc = lib.moba_decode_minmax_fwd(ctypes.byref(p), fake, fake, fake, fake, fake, None, fake, need,
+                                    fake, fake, None)
+    assert rc == moba.ERR_INVALID_ARG
+    rc = lib.moba_decode_minmax_fwd(ctypes.byref(p), fake, fake, fake, fake, fake, odd, fake, need,
+                                    fake, fake, None)
+    assert rc == moba.ERR_INVALID_ARG
+    rc = lib.moba_decode_minmax_fwd(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, need - 1,
+                                    fake, fake, None)
+    assert rc == moba.ERR_WORKSPACE
+
+
 def test_selftest_argument_checks(lib):
     assert lib.moba_selftest_timeout(None, 16, None) == moba.ERR_INVALID_ARG
     fake = ctypes.c_void_p(1 << 20)

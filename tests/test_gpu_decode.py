@@ -1,8 +1,11 @@
-"""Decode step on the GPU (moba_decode_fwd through the C ABI) against the float64 oracle.
+"""Decode step on the GPU (moba_decode_fwd and moba_decode_minmax_fwd through the C ABI)
+against the float64 oracle.
 
 The new query of each sequence sits at its cache's last row, so the reference is the oracle's
 row-wise selection and attention of those rows (oracle.moba_decode, pinned against the prefill
-forward's last rows on the CPU).  Tolerances as for the prefill path."""
+forward's last rows on the CPU; with gate="minmax", pinned by box-corner enumeration and
+brute-force selection).  Tolerances as for the prefill path; the min/max block summary
+(moba_minmaxpool) is exact."""
 
 import numpy as np
 import pytest
@@ -29,13 +32,18 @@ def decode_inputs(w):
     return q_new, q_full, k, v, cu_t
 
 
-def gpu_decode(w, q_new, k, v, cu_t, return_sel=False):
-    means = moba.meanpool(k, cu_t, w.chunk_size)
+def gpu_decode(w, q_new, k, v, cu_t, return_sel=False, gate="mean"):
     p = moba.make_params(len(w.seqlens), w.total_tokens, w.num_q_heads, w.num_kv_heads,
                          w.head_dim, w.chunk_size, w.topk)
     ws = torch.empty(moba.load_library().moba_decode_workspace_size(p), dtype=torch.uint8,
                      device="cuda")
-    out, lse = moba.decode_fwd(q_new, k, v, cu_t, means, w.chunk_size, w.topk, workspace=ws)
+    if gate == "mean":
+        means = moba.meanpool(k, cu_t, w.chunk_size)
+        out, lse = moba.decode_fwd(q_new, k, v, cu_t, means, w.chunk_size, w.topk, workspace=ws)
+    else:
+        k_min, k_max = moba.minmaxpool(k, cu_t, w.chunk_size)
+        out, lse = moba.decode_minmax_fwd(q_new, k, v, cu_t, k_min, k_max, w.chunk_size, w.topk,
+                                          workspace=ws)
     torch.cuda.synchronize()
     if not return_sel:
         return out, lse
@@ -45,9 +53,11 @@ def gpu_decode(w, q_new, k, v, cu_t, return_sel=False):
     return out, lse, sel.cpu().numpy()
 
 
-def near_tie_rows(w, q_new_np, k_np, ref):
+def near_tie_rows(w, q_new_np, k_np, ref, gate="mean"):
     """(b, h) rows whose last routed and first excluded past scores are within the band."""
     cu = np.asarray(w.cu_seqlens)
+    if gate == "minmax":
+        return near_tie_rows_minmax(w, q_new_np, k_np)
     means = oracle.block_means(k_np, cu, w.chunk_size)
     tab = oracle.block_table(cu, w.chunk_size)
     group = w.num_q_heads // w.num_kv_heads
@@ -64,6 +74,40 @@ def near_tie_rows(w, q_new_np, k_np, ref):
     return ties
 
 
+def near_tie_rows_minmax(w, q_new_np, k_np):
+    """Rows whose m-th and (m+1)-th best min/max scores could swap under the kernel's fp32
+    arithmetic.  Every term max(q_i kmin_i, q_i kmax_i) is exact (bf16 x bf16), so a score is
+    off only by its fp32 sum: 4 accumulators of d/8 pair sums, then two more adds, at most
+    (d/4 + 2) * 2^-24 * sum_i |t_i|.  Two scores may swap only when their gap is below the sum
+    of their bounds.  (The mean gate's 1e-3 relative band would cover every row here: a box
+    over thousands of N(0, 1) keys gives scores of a few hundred that differ by a few units.)"""
+    cu = np.asarray(w.cu_seqlens)
+    kmin, kmax = oracle.block_minmax(k_np, cu, w.chunk_size)
+    tab = oracle.block_table(cu, w.chunk_size)
+    group = w.num_q_heads // w.num_kv_heads
+    unit = (w.head_dim / 4 + 2) * 2.0 ** -24
+    ties = set()
+    for b in range(len(w.seqlens)):
+        n = w.seqlens[b]
+        if n == 0:
+            continue
+        c = (n - 1) // w.chunk_size
+        m = min(w.topk - 1, c)
+        if m == 0 or c <= m:
+            continue
+        b0 = int(tab["cu_blocks"][b])
+        for h in range(w.num_q_heads):
+            q = q_new_np[b, h]
+            lo, hi = kmin[b0:b0 + c, h // group], kmax[b0:b0 + c, h // group]
+            terms = np.maximum(q * lo, q * hi)
+            score, bound = terms.sum(axis=1), unit * np.abs(terms).sum(axis=1)
+            order = np.argsort(-score, kind="stable")
+            x, y = order[m - 1], order[m]
+            if score[x] - score[y] <= bound[x] + bound[y]:
+                ties.add((b, h))
+    return ties
+
+
 SMALL = [
     W.custom("dec_ragged_gqa", [700, 1337, 128, 1, 0, 390], 8, 2, 128, 128, 3, "k_offsets", 61),
     W.custom("dec_d64_mha", [3000, 1500], 4, 4, 64, 128, 5, "qk_offsets", 62),
@@ -74,13 +118,14 @@ SMALL = [
 ]
 
 
+@pytest.mark.parametrize("gate", ["mean", "minmax"])
 @pytest.mark.parametrize("w", SMALL, ids=[w.name for w in SMALL])
-def test_decode_small(w):
+def test_decode_small(w, gate):
     q_new, _, k, v, cu_t = decode_inputs(w)
-    out, lse, sel = gpu_decode(w, q_new, k, v, cu_t, return_sel=True)
+    out, lse, sel = gpu_decode(w, q_new, k, v, cu_t, return_sel=True, gate=gate)
     qn, kn, vn = PT.host(q_new), PT.host(k), PT.host(v)
-    ref = oracle.moba_decode(qn, kn, vn, np.asarray(w.cu_seqlens), w.chunk_size, w.topk)
-    ties = near_tie_rows(w, qn, kn, ref)
+    ref = oracle.moba_decode(qn, kn, vn, np.asarray(w.cu_seqlens), w.chunk_size, w.topk, gate=gate)
+    ties = near_tie_rows(w, qn, kn, ref, gate)
     B, hq = len(w.seqlens), w.num_q_heads
     keep = np.ones((B, hq), dtype=bool)
     for b in range(B):
@@ -117,15 +162,58 @@ def test_decode_matches_prefill_last_rows_on_gpu():
     assert np.abs(PT.host(lse) - PT.host(plse)[:, last]).max() <= PT.LSE_ABS
 
 
-def test_decode_long_cache():
+@pytest.mark.parametrize("gate", ["mean", "minmax"])
+def test_decode_long_cache(gate):
     """A 256K-token cache with the 1M workload's block size and top-k (64 blocks of 4096)."""
     w = W.custom("dec_256k", [1 << 18], 8, 2, 128, 4096, 12, "k_offsets", 68)
     q_new, _, k, v, cu_t = decode_inputs(w)
-    out, lse = gpu_decode(w, q_new, k, v, cu_t)
+    out, lse = gpu_decode(w, q_new, k, v, cu_t, gate=gate)
     qn, kn, vn = PT.host(q_new), PT.host(k), PT.host(v)
-    ref = oracle.moba_decode(qn, kn, vn, np.asarray(w.cu_seqlens), w.chunk_size, w.topk)
-    ties = near_tie_rows(w, qn, kn, ref)
+    ref = oracle.moba_decode(qn, kn, vn, np.asarray(w.cu_seqlens), w.chunk_size, w.topk, gate=gate)
+    ties = near_tie_rows(w, qn, kn, ref, gate)
     rows = [(0, h) for h in range(w.num_q_heads) if (0, h) not in ties]
     o, l = PT.host(out), PT.host(lse)
     PT.check_out(np.stack([o[b, h] for b, h in rows]), np.array([l[h, b] for b, h in rows]),
                  np.stack([ref["out"][b, h] for b, h in rows]), np.array([ref["lse"][h, b] for b, h in rows]))
+
+
+@pytest.mark.parametrize("w", [SMALL[0], SMALL[1], W.custom("mm_long", [1 << 17, 5000], 8, 8, 128, 4096, 4,
+                                                            "k_offsets", 69)],
+                         ids=["dec_ragged_gqa", "dec_d64_mha", "mm_long"])
+def test_minmaxpool_is_exact(w):
+    """The bf16 min/max summary equals the oracle's extrema bit for bit (extrema of bf16
+    values are bf16 values), partial blocks included."""
+    _, _, k, _, cu_t = decode_inputs(w)
+    nb = moba.num_blocks(w.seqlens, w.chunk_size)
+    k_min, k_max = moba.minmaxpool(k, cu_t, w.chunk_size, num_blocks_out=nb)
+    torch.cuda.synchronize()
+    rmin, rmax = oracle.block_minmax(PT.host(k), np.asarray(w.cu_seqlens), w.chunk_size)
+    assert k_min.shape == rmin.shape and k_max.shape == rmax.shape
+    np.testing.assert_array_equal(PT.host(k_min), rmin)
+    np.testing.assert_array_equal(PT.host(k_max), rmax)
+
+
+def test_minmax_gate_routes_the_single_matching_key_on_gpu():
+    """Block 1 holds one key aligned with q among zeros: its mean (4/128) loses to block 0's
+    uniform 0.5, its box maximum (4) wins.  The mean path routes block 0, the min/max path
+    block 1; both outputs match the oracle."""
+    d, chunk, L = 64, 128, 3 * 128 + 40
+    k = torch.zeros((L, 1, d), dtype=torch.float32)
+    k[0:128, 0, 0] = 0.5
+    k[128 + 77, 0, 0] = 4.0
+    k[256:384, 0, 0] = -1.0
+    k[384:, 0, 1] = 1.0
+    g = torch.Generator().manual_seed(70)
+    v = torch.randn((L, 1, d), generator=g)
+    q_new = torch.zeros((1, 1, d))
+    q_new[0, 0, 0] = 1.0
+    k, v, q_new = (t.to(torch.bfloat16).cuda().contiguous() for t in (k, v, q_new))
+    cu_t = torch.tensor([0, L], dtype=torch.int32, device="cuda")
+    w = W.custom("mm_spike", [L], 1, 1, d, chunk, 2, "k_offsets", 70)
+    qn, kn, vn = PT.host(q_new), PT.host(k), PT.host(v)
+    for gate, routed in (("mean", 0), ("minmax", 1)):
+        out, lse, sel = gpu_decode(w, q_new, k, v, cu_t, return_sel=True, gate=gate)
+        assert sorted(int(x) for x in sel[0, 0]) == sorted([routed, 3]), (gate, sel[0, 0])
+        ref = oracle.moba_decode(qn, kn, vn, np.array([0, L]), chunk, 2, gate=gate)
+        assert sorted(ref["sel"][0, 0]) == sorted([routed, 3])
+        PT.check_out(PT.host(out)[0], PT.host(lse)[:, 0], ref["out"][0], ref["lse"][:, 0])
