@@ -559,3 +559,24 @@ def test_minmax_decode_with_every_block_selected_equals_the_mean_gate():
     assert np.array_equal(a["sel"], b["sel"])
     np.testing.assert_array_equal(a["out"], b["out"])
     np.testing.assert_array_equal(a["lse"], b["lse"])
+
+
+def test_minmax_score_is_the_centre_radius_contraction():
+    """For either sign of q_i, max(q_i lo_i, q_i hi_i) = q_i (lo_i + hi_i)/2 + |q_i| (hi_i - lo_i)/2,
+    so the min/max score is the length-2d product of [q, |q|] with [centre; radius] (torch fp64
+    matmul over all blocks at once)."""
+    rng = np.random.default_rng(13)
+    k = rng.standard_normal((700, 3, 16)) + rng.standard_normal((1, 3, 16))
+    cu = np.array([0, 300, 700])
+    kmin, kmax = oracle.block_minmax(k, cu, 64)
+    q = rng.standard_normal((5, 16))
+    q[:, :3] = 0.0
+    for g in range(3):
+        centre = torch.from_numpy((kmin[:, g] + kmax[:, g]) / 2)
+        radius = torch.from_numpy((kmax[:, g] - kmin[:, g]) / 2)
+        lhs = torch.cat([torch.from_numpy(q), torch.from_numpy(np.abs(q))], dim=1)
+        rhs = torch.cat([centre, radius], dim=1)
+        want = (lhs @ rhs.T).numpy()
+        for r in range(q.shape[0]):
+            got = oracle.minmax_scores_row(q[r], np.stack([kmin[:, g], kmax[:, g]], axis=1))
+            np.testing.assert_allclose(got, want[r], rtol=1e-13, atol=1e-12)
