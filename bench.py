@@ -661,6 +661,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gate != "mean" and not args.decode:
+        ap.error("--gate applies to the decode step (--decode); the prefill gate is the mean gate")
     from block_sparse_long_meanpool_b200 import workloads as W
 
     if args.decode:

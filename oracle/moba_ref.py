@@ -1,4 +1,5 @@
-"""Plain float64 definition of the MoBA causal prefill forward (CPU, NumPy).
+"""Plain float64 definition of the MoBA causal prefill forward (CPU, NumPy), with its decode
+step, the min/max (Quest-style) gate variant and the backward pass.
 
 TEST INFRASTRUCTURE ONLY: see ``oracle/__init__.py``.  Slow on purpose; every
 step is written the way the pages define it so that it can be checked by eye.
@@ -342,6 +343,54 @@ def moba_forward(q, k, v, cu_seqlens, chunk, topk, scale=None, sel=None):
         sel = select_blocks(q, means, cu_seqlens, chunk, topk)
     out, lse = attention_masked_dense(q, k, v, cu_seqlens, chunk, sel, scale)
     return {"out": out, "lse": lse, "sel": sel, "means": means}
+
+
+def moba_backward(q, k, v, cu_seqlens, chunk, sel, d_out, d_lse=None, scale=None):
+    """Gradients of the forward's ``out`` and ``lse`` with respect to ``q``, ``k`` and ``v``.
+
+    Reading: the gate has no parameters (the analysis, §2.5) and routes by hard top-k (§2.2),
+    so the selection is piecewise constant in ``q`` and ``k``: its derivative is zero wherever
+    it exists, and the gradient reaches q, k and v only through the softmax attention over the
+    selected union (§2.2-§2.3).  ``sel`` is the selection the forward used.
+
+    Per row ``(t, h)`` with attended keys U (:func:`attended_keys`), logits
+    ``z_u = scale * <q, k_u>``, ``p = softmax(z)``, ``out = sum_u p_u v_u`` and
+    ``lse = log sum_u exp(z_u)``, the chain rule gives, with ``dp_u = <d_out, v_u>``:
+
+    * ``dv_u += p_u * d_out``
+    * ``dz_u = p_u * (dp_u - <d_out, out>) + p_u * d_lse``  (d lse / d z_u = p_u)
+    * ``dq = scale * sum_u dz_u k_u`` and ``dk_u += scale * dz_u * q``
+
+    A KV head collects the contributions of every query head that reads it (GQA).
+    ``d_out`` is ``[T, Hq, d]``, ``d_lse`` ``[Hq, T]`` or None (zero).  Returns
+    ``dq [T, Hq, d]``, ``dk`` and ``dv [T, Hkv, d]``, float64.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    d_out = np.asarray(d_out, dtype=np.float64)
+    T, Hq, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    group = Hq // k.shape[1]
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for t in range(T):
+        for h in range(Hq):
+            u = attended_keys(t, sel[h, t], cu_seqlens, chunk)
+            g = h // group
+            z = scale * (k[u, g] @ q[t, h])
+            p = np.exp(z - z.max())
+            p /= p.sum()
+            o = p @ v[u, g]
+            dp = v[u, g] @ d_out[t, h]
+            dz = p * (dp - d_out[t, h] @ o)
+            if d_lse is not None:
+                dz += p * float(d_lse[h, t])
+            dq[t, h] = scale * (dz @ k[u, g])
+            dk[u, g] += scale * np.outer(dz, q[t, h])
+            dv[u, g] += np.outer(p, d_out[t, h])
+    return dq, dk, dv
 
 
 class _LastRowQueries:

@@ -580,3 +580,116 @@ def test_minmax_score_is_the_centre_radius_contraction():
         for r in range(q.shape[0]):
             got = oracle.minmax_scores_row(q[r], np.stack([kmin[:, g], kmax[:, g]], axis=1))
             np.testing.assert_allclose(got, want[r], rtol=1e-13, atol=1e-12)
+
+
+# ---- backward: moba_backward (dq, dk, dv for the forward's selection)
+
+def _bw_case(seqlens, hq, hkv, d, chunk, topk, seed):
+    cu, q, k, v, _ = _decode_inputs(seqlens, hq, hkv, d, seed)
+    rng = np.random.default_rng(seed + 1000)
+    fwd = oracle.moba_forward(q, k, v, cu, chunk, topk)
+    d_out = rng.standard_normal(q.shape)
+    d_lse = rng.standard_normal((hq, q.shape[0]))
+    return cu, q, k, v, fwd, d_out, d_lse
+
+
+def _autograd_masked(q, k, v, cu, chunk, sel, d_out, d_lse, scale):
+    """torch fp64 autograd through the library's masked SDPA and logsumexp, with the mask
+    built from the attended key sets (KV heads repeated for GQA; autograd sums them back)."""
+    T, hq, d = q.shape
+    group = hq // k.shape[1]
+    allowed = torch.zeros((hq, T, T), dtype=torch.bool)
+    for h in range(hq):
+        for t in range(T):
+            allowed[h, t, torch.from_numpy(oracle.attended_keys(t, sel[h, t], cu, chunk))] = True
+    qt, kt, vt = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    kr = kt.repeat_interleave(group, dim=1).transpose(0, 1)
+    vr = vt.repeat_interleave(group, dim=1).transpose(0, 1)
+    qh = qt.transpose(0, 1)
+    out = torch.nn.functional.scaled_dot_product_attention(qh, kr, vr, attn_mask=allowed, scale=scale)
+    z = (qh @ kr.transpose(1, 2)) * scale
+    lse = torch.logsumexp(z.masked_fill(~allowed, float("-inf")), dim=-1)
+    loss = (out.transpose(0, 1) * torch.from_numpy(d_out)).sum() + (lse * torch.from_numpy(d_lse)).sum()
+    loss.backward()
+    return qt.grad.numpy(), kt.grad.numpy(), vt.grad.numpy()
+
+
+@pytest.mark.parametrize("seqlens,hq,hkv,d,chunk,topk", [
+    ([37, 0, 50, 1], 4, 2, 8, 8, 3),     # varlen GQA, empty and 1-token sequences, partial blocks
+    ([64], 2, 2, 16, 16, 2),             # MHA
+    ([45, 30], 6, 2, 4, 5, 4),           # odd group, chunk not a power of two
+])
+def test_backward_matches_autograd_of_masked_attention(seqlens, hq, hkv, d, chunk, topk):
+    cu, q, k, v, fwd, d_out, d_lse = _bw_case(seqlens, hq, hkv, d, chunk, topk, 21 + hq)
+    scale = 1.0 / math.sqrt(d)
+    got = oracle.moba_backward(q, k, v, cu, chunk, fwd["sel"], d_out, d_lse)
+    want = _autograd_masked(q, k, v, cu, chunk, fwd["sel"], d_out, d_lse, scale)
+    for g, w_ in zip(got, want):
+        np.testing.assert_allclose(g, w_, rtol=1e-10, atol=1e-12)
+
+
+def test_backward_with_every_block_selected_is_causal_attention_backward():
+    """topk >= blocks: the gradients of torch's fp64 causal SDPA (no mask built by the test)."""
+    seqlens, hq, d = [70], 2, 8
+    cu, q, k, v, fwd, d_out, _ = _bw_case(seqlens, hq, hq, d, 16, 8, 5)
+    dq, dk, dv = oracle.moba_backward(q, k, v, cu, 16, fwd["sel"], d_out)
+    qt, kt, vt = (torch.tensor(x.transpose(1, 0, 2), requires_grad=True) for x in (q, k, v))
+    out = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True)
+    (out * torch.from_numpy(d_out.transpose(1, 0, 2))).sum().backward()
+    np.testing.assert_allclose(dq, qt.grad.numpy().transpose(1, 0, 2), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dk, kt.grad.numpy().transpose(1, 0, 2), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dv, vt.grad.numpy().transpose(1, 0, 2), rtol=1e-10, atol=1e-12)
+
+
+def test_backward_matches_finite_differences_of_the_forward():
+    """Central differences of L = <d_out, out> + <d_lse, lse> through the oracle's own forward
+    with the selection held fixed."""
+    cu, q, k, v, fwd, d_out, d_lse = _bw_case([23, 17], 4, 2, 4, 4, 3, 8)
+    sel = fwd["sel"]
+    grads = oracle.moba_backward(q, k, v, cu, 4, sel, d_out, d_lse)
+
+    def loss(qq, kk, vv):
+        o, l = oracle.attention_masked_dense(qq, kk, vv, cu, 4, sel)
+        return float((o * d_out).sum() + (l * d_lse).sum())
+
+    rng = np.random.default_rng(9)
+    eps = 1e-6
+    for which, x in enumerate((q, k, v)):
+        for _ in range(12):
+            idx = tuple(int(rng.integers(0, n)) for n in x.shape)
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = [q, k, v]
+            args_m = [q, k, v]
+            args_p[which], args_m[which] = xp, xm
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            assert abs(fd - grads[which][idx]) < 1e-6 * max(1.0, abs(fd)), (which, idx, fd, grads[which][idx])
+
+
+def test_backward_closed_form_sums():
+    """Softmax weights sum to one, so per KV head the value gradients sum to the sum of d_out
+    over the rows that read it, and the key gradients sum to scale * sum of d_lse * q (zero
+    without d_lse)."""
+    seqlens, hq, hkv, d = [40, 25], 4, 2, 8
+    cu, q, k, v, fwd, d_out, d_lse = _bw_case(seqlens, hq, hkv, d, 8, 3, 12)
+    scale = 1.0 / math.sqrt(d)
+    group = hq // hkv
+    _, dk0, dv0 = oracle.moba_backward(q, k, v, cu, 8, fwd["sel"], d_out)
+    _, dk1, _ = oracle.moba_backward(q, k, v, cu, 8, fwd["sel"], d_out, d_lse)
+    for g in range(hkv):
+        hs = list(range(g * group, (g + 1) * group))
+        np.testing.assert_allclose(dv0[:, g].sum(axis=0), d_out[:, hs].sum(axis=(0, 1)), atol=1e-11)
+        np.testing.assert_allclose(dk0[:, g].sum(axis=0), 0.0, atol=1e-11)
+        want = scale * sum((d_lse[h][:, None] * q[:, h]).sum(axis=0) for h in hs)
+        np.testing.assert_allclose(dk1[:, g].sum(axis=0), want, atol=1e-11)
+
+
+def test_backward_gqa_equals_mha_with_repeated_kv_heads():
+    cu, q, k, v, fwd, d_out, d_lse = _bw_case([30, 21], 4, 2, 8, 8, 3, 14)
+    dq, dk, dv = oracle.moba_backward(q, k, v, cu, 8, fwd["sel"], d_out, d_lse)
+    kr, vr = np.repeat(k, 2, axis=1), np.repeat(v, 2, axis=1)
+    dq2, dk2, dv2 = oracle.moba_backward(q, kr, vr, cu, 8, fwd["sel"], d_out, d_lse)
+    np.testing.assert_allclose(dq, dq2, atol=1e-13)
+    np.testing.assert_allclose(dk, dk2.reshape(dk2.shape[0], 2, 2, -1).sum(axis=2), atol=1e-13)
+    np.testing.assert_allclose(dv, dv2.reshape(dv2.shape[0], 2, 2, -1).sum(axis=2), atol=1e-13)
