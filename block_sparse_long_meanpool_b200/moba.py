@@ -153,6 +153,56 @@ def _check_qkv(q, k, v=None):
         _require(t.dim() == 3 and t.is_contiguous(), f"{name} must be contiguous [T, H, d]")
 
 
+def _require_buffer(t, name, shape, dtype, device):
+    """A caller-supplied buffer the kernels read or write whole: exact shape, dtype, layout and
+    device (a wrong shape would be an out-of-bounds access on the device, not an error)."""
+    _require(tuple(t.shape) == tuple(shape), f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    _require(t.dtype == dtype, f"{name} must be {dtype}, got {t.dtype}")
+    _require(t.is_contiguous(), f"{name} must be contiguous")
+    _require(t.device == device, f"{name} must be on {device}, got {t.device}")
+
+
+def _rows_backed(t):
+    """Rows of t[0]'s size that the memory behind t.data_ptr() holds (a view such as
+    ``meanpool(..., num_blocks_out=n)`` keeps the block-count bound's rows behind it)."""
+    row = t.shape[1] * t.shape[2] * t.element_size()
+    avail = t.untyped_storage().nbytes() - t.storage_offset() * t.element_size()
+    return avail // row if row else 0
+
+
+def _require_summary(t, name, dtype, nb_bound, hkv, d, device):
+    """A per-block summary indexed by global block id [NB, Hkv, d].  The kernels index it by
+    block without knowing how many rows the caller has, so the memory behind it must hold the
+    block-count bound's rows (moba_num_blocks_bound; ``meanpool`` and ``minmaxpool`` always
+    allocate that many)."""
+    _require(t.dim() == 3 and tuple(t.shape[1:]) == (hkv, d),
+             f"{name} must be [NB, {hkv}, {d}], got {tuple(t.shape)}")
+    _require(t.dtype == dtype, f"{name} must be {dtype}, got {t.dtype}")
+    _require(t.is_contiguous(), f"{name} must be contiguous")
+    _require(t.device == device, f"{name} must be on {device}, got {t.device}")
+    _require(_rows_backed(t) >= nb_bound,
+             f"{name} must be backed by >= {nb_bound} block rows (moba_num_blocks_bound), has {_rows_backed(t)}")
+
+
+def _validate_decode(q, k, v, cu_seqlens, summary, out, lse, chunk_size, topk):
+    """Shapes, dtypes and devices of a decode call (host-only; no CUDA needed).  ``summary`` is
+    a list of (name, tensor, dtype) block summaries."""
+    batch, hq, d = q.shape
+    T, hkv, dk = k.shape
+    _require(dk == d, f"k head_dim {dk} differs from q head_dim {d}")
+    _require(tuple(v.shape) == tuple(k.shape), "v must have k's shape [T, Hkv, d]")
+    _require(v.device == q.device and k.device == q.device, "q, k and v must be on one device")
+    _require(cu_seqlens.dtype == torch.int32 and cu_seqlens.numel() == batch + 1,
+             "cu_seqlens must be an int32 tensor of batch + 1 entries")
+    bound = num_blocks_bound(make_params(batch, T, hq, hkv, d, chunk_size, topk))
+    for name, t, dtype in summary:
+        _require_summary(t, name, dtype, bound, hkv, d, q.device)
+    if out is not None:
+        _require_buffer(out, "out", (batch, hq, d), torch.bfloat16, q.device)
+    if lse is not None:
+        _require_buffer(lse, "lse", (hq, batch), torch.float32, q.device)
+
+
 def num_blocks(seqlens, chunk_size):
     """Exact block count sum(ceil(L_i / chunk)) from host-side sequence lengths."""
     return int(sum((int(n) + chunk_size - 1) // chunk_size for n in seqlens))
@@ -178,8 +228,10 @@ def meanpool(k, cu_seqlens, chunk_size, num_blocks_out=None):
     batch = cu_seqlens.numel() - 1
     T, hkv, d = k.shape
     p = make_params(batch, T, hkv, hkv, d, chunk_size, 1)
-    nb = num_blocks_out if num_blocks_out is not None else max(load_library().moba_num_blocks_bound(ctypes.byref(p)), 0)
-    out = torch.empty((max(nb, 1), hkv, d), dtype=torch.float32, device=k.device)
+    bound = max(load_library().moba_num_blocks_bound(ctypes.byref(p)), 0)
+    nb = bound if num_blocks_out is None else min(int(num_blocks_out), bound)
+    # the kernel writes every real block, so the buffer always has the bound's rows
+    out = torch.empty((max(bound, 1), hkv, d), dtype=torch.float32, device=k.device)
     _check(load_library().moba_meanpool(ctypes.byref(p), _ptr(k), _ptr(cu_seqlens), _ptr(out),
                                         _stream(k.device)))
     return out[:nb]
@@ -191,8 +243,10 @@ def minmaxpool(k, cu_seqlens, chunk_size, num_blocks_out=None):
     batch = cu_seqlens.numel() - 1
     T, hkv, d = k.shape
     p = make_params(batch, T, hkv, hkv, d, chunk_size, 1)
-    nb = num_blocks_out if num_blocks_out is not None else max(load_library().moba_num_blocks_bound(ctypes.byref(p)), 0)
-    k_min = torch.empty((max(nb, 1), hkv, d), dtype=torch.bfloat16, device=k.device)
+    bound = max(load_library().moba_num_blocks_bound(ctypes.byref(p)), 0)
+    nb = bound if num_blocks_out is None else min(int(num_blocks_out), bound)
+    # the kernel writes every real block, so the buffers always have the bound's rows
+    k_min = torch.empty((max(bound, 1), hkv, d), dtype=torch.bfloat16, device=k.device)
     k_max = torch.empty_like(k_min)
     _check(load_library().moba_minmaxpool(ctypes.byref(p), _ptr(k), _ptr(cu_seqlens), _ptr(k_min),
                                           _ptr(k_max), _stream(k.device)))
@@ -207,6 +261,7 @@ def gate_topk(q, k_mean, cu_seqlens, chunk_size, topk, num_kv_heads=None):
     T, hq, d = q.shape
     hkv = num_kv_heads or k_mean.shape[1]
     p = make_params(batch, T, hq, hkv, d, chunk_size, topk)
+    _require_summary(k_mean, "k_mean", torch.float32, num_blocks_bound(p), hkv, d, q.device)
     sel = torch.empty((hq, T, topk), dtype=torch.int32, device=q.device)
     _check(load_library().moba_gate_topk(ctypes.byref(p), _ptr(q), _ptr(k_mean), _ptr(cu_seqlens),
                                          _ptr(sel), _stream(q.device)))
@@ -215,10 +270,10 @@ def gate_topk(q, k_mean, cu_seqlens, chunk_size, topk, num_kv_heads=None):
 
 def _decode(fn, summary, q, k, v, cu_seqlens, chunk_size, topk, softmax_scale, workspace, out, lse):
     _check_qkv(q, k, v)
+    _require(cu_seqlens.is_cuda, "cu_seqlens must be a CUDA tensor")
+    _validate_decode(q, k, v, cu_seqlens, summary, out, lse, chunk_size, topk)
     batch, hq, d = q.shape
     T, hkv, _ = k.shape
-    _require(cu_seqlens.is_cuda and cu_seqlens.dtype == torch.int32 and cu_seqlens.numel() == batch + 1,
-             "cu_seqlens must be a CUDA int32 tensor of batch + 1 entries")
     p = make_params(batch, T, hq, hkv, d, chunk_size, topk, softmax_scale)
     lib = load_library()
     n = lib.moba_decode_workspace_size(ctypes.byref(p))
@@ -231,7 +286,7 @@ def _decode(fn, summary, q, k, v, cu_seqlens, chunk_size, topk, softmax_scale, w
     if lse is None:
         lse = torch.empty((hq, batch), dtype=torch.float32, device=q.device)
     _check(getattr(lib, fn)(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens),
-                            *[_ptr(t) for t in summary], _ptr(workspace),
+                            *[_ptr(t) for _, t, _ in summary], _ptr(workspace),
                             ctypes.c_size_t(workspace.numel()), _ptr(out), _ptr(lse), _stream(q.device)))
     return out, lse
 
@@ -245,9 +300,7 @@ def decode_fwd(q, k, v, cu_seqlens, k_mean, chunk_size, topk, softmax_scale=None
     k_mean fp32 block means of these caches (``meanpool``).  Returns (out bf16 [batch, Hq, d],
     lse fp32 [Hq, batch]).
     """
-    _require(k_mean.is_cuda and k_mean.dtype == torch.float32 and k_mean.is_contiguous(),
-             "k_mean must be a contiguous CUDA fp32 tensor")
-    return _decode("moba_decode_fwd", (k_mean,), q, k, v, cu_seqlens, chunk_size, topk,
+    return _decode("moba_decode_fwd", [("k_mean", k_mean, torch.float32)], q, k, v, cu_seqlens, chunk_size, topk,
                    softmax_scale, workspace, out, lse)
 
 
@@ -255,10 +308,8 @@ def decode_minmax_fwd(q, k, v, cu_seqlens, k_min, k_max, chunk_size, topk, softm
                       workspace=None, out=None, lse=None):
     """Decode step with the min/max gate (moba_decode_minmax_fwd): as ``decode_fwd``, with the
     bf16 block summary (k_min, k_max) of ``minmaxpool`` in place of the means."""
-    for t in (k_min, k_max):
-        _require(t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous(),
-                 "k_min and k_max must be contiguous CUDA bf16 tensors")
-    return _decode("moba_decode_minmax_fwd", (k_min, k_max), q, k, v, cu_seqlens, chunk_size, topk,
+    return _decode("moba_decode_minmax_fwd", [("k_min", k_min, torch.bfloat16), ("k_max", k_max, torch.bfloat16)],
+                   q, k, v, cu_seqlens, chunk_size, topk,
                    softmax_scale, workspace, out, lse)
 
 
@@ -316,12 +367,15 @@ def attn_fwd(q, k, v, cu_seqlens, chunk_size, topk, softmax_scale=None, sel=None
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
     if out is None:
         out = torch.empty((T, hq, d), dtype=torch.bfloat16, device=dev)
+    else:
+        _require_buffer(out, "out", (T, hq, d), torch.bfloat16, dev)
     if lse is None:
         lse = torch.empty((hq, T), dtype=torch.float32, device=dev)
+    else:
+        _require_buffer(lse, "lse", (hq, T), torch.float32, dev)
     sel_out = None
     if sel is not None:
-        _require(sel.dtype == torch.int32 and sel.is_contiguous() and tuple(sel.shape) == (hq, T, topk),
-                 "sel must be int32 [Hq, T, topk]")
+        _require_buffer(sel, "sel", (hq, T, topk), torch.int32, dev)
     elif return_sel:
         sel_out = torch.empty((hq, T, topk), dtype=torch.int32, device=dev)
     info = MobaRunInfo()

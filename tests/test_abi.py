@@ -211,3 +211,41 @@ def test_selftest_argument_checks(lib):
     fake = ctypes.c_void_p(1 << 20)
     assert lib.moba_selftest_timeout(fake, 0, None) == moba.ERR_INVALID_ARG
     assert lib.moba_selftest_timeout(fake, (1 << 20) + 1, None) == moba.ERR_INVALID_ARG
+
+
+def _meta(*shape, dtype=torch.bfloat16):
+    return torch.empty(shape, dtype=dtype, device="meta")
+
+
+def test_decode_binding_rejects_mismatched_buffers(lib):
+    """The binding checks every caller-supplied tensor's shape, dtype and backing memory before
+    any launch (host-only: meta tensors, no device memory)."""
+    B, T, hq, hkv, d, chunk, topk = 3, 1000, 4, 2, 64, 128, 3
+    bound = moba.num_blocks_bound(moba.make_params(B, T, hq, hkv, d, chunk, topk))
+    q, k, v = _meta(B, hq, d), _meta(T, hkv, d), _meta(T, hkv, d)
+    cu = _meta(B + 1, dtype=torch.int32)
+    means = _meta(bound, hkv, d, dtype=torch.float32)
+    kmin, kmax = _meta(bound, hkv, d), _meta(bound, hkv, d)
+    out, lse = _meta(B, hq, d), _meta(hq, B, dtype=torch.float32)
+    ok_mean = [("k_mean", means, torch.float32)]
+    ok_mm = [("k_min", kmin, torch.bfloat16), ("k_max", kmax, torch.bfloat16)]
+    moba._validate_decode(q, k, v, cu, ok_mean, out, lse, chunk, topk)
+    moba._validate_decode(q, k, v, cu, ok_mm, None, None, chunk, topk)
+    # a view of fewer rows is fine while its memory holds the bound's rows (as meanpool returns)
+    moba._validate_decode(q, k, v, cu, [("k_mean", means[:bound - 2], torch.float32)], out, lse, chunk, topk)
+    bad = [
+        (q, _meta(T, hkv, 128), _meta(T, hkv, 128), cu, ok_mean, out, lse),          # head_dim
+        (q, k, _meta(T - 1, hkv, d), cu, ok_mean, out, lse),                         # v shape
+        (q, k, v, _meta(B, dtype=torch.int32), ok_mean, out, lse),                   # cu entries
+        (q, k, v, cu, [("k_mean", _meta(bound - 1, hkv, d, dtype=torch.float32), torch.float32)], out, lse),
+        (q, k, v, cu, [("k_mean", means[1:], torch.float32)], out, lse),             # offset view
+        (q, k, v, cu, [("k_mean", _meta(bound, hkv, d), torch.float32)], out, lse),  # dtype
+        (q, k, v, cu, [("k_min", _meta(bound, 1, d), torch.bfloat16)], out, lse),    # kv heads
+        (q, k, v, cu, ok_mm, _meta(B, hq, d + 1), lse),                              # out shape
+        (q, k, v, cu, ok_mm, out.float(), lse),                                      # out dtype
+        (q, k, v, cu, ok_mm, out, _meta(B, hq, dtype=torch.float32)),                # lse layout
+    ]
+    for i, args in enumerate(bad):
+        with pytest.raises(ValueError):
+            moba._validate_decode(*args, chunk, topk)
+            pytest.fail(f"case {i} accepted")
