@@ -6,6 +6,8 @@
 #include <cstring>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "moba.h"
 #include "moba_internal.cuh"
 #include "ptx.cuh"
@@ -13,6 +15,17 @@
 using namespace moba;
 
 namespace {
+
+// Named NVTX range over a scope.  Without a profiler attached each push/pop is a no-op after a
+// one-time check; under nsys or ncu every launch is attributed to its entry point and stage,
+// e.g. `ncu --nvtx --nvtx-include "moba_attn_fwd/wave/attention/"` captures the attention
+// launches only.
+struct NvtxScope {
+    explicit NvtxScope(const char* name) { nvtxRangePushA(name); }
+    ~NvtxScope() { nvtxRangePop(); }
+    NvtxScope(const NvtxScope&) = delete;
+    NvtxScope& operator=(const NvtxScope&) = delete;
+};
 
 thread_local std::string g_last_error;
 
@@ -174,6 +187,7 @@ size_t moba_workspace_size(const moba_params* p) {
 
 moba_status moba_meanpool(const moba_params* p, const void* k, const int* cu_seqlens,
                           float* k_mean, void* stream) {
+    NvtxScope range("moba_meanpool");
     moba_status s = check_params(p);
     if (s != MOBA_OK) return s;
     if (p->total_tokens == 0) return MOBA_OK;
@@ -189,6 +203,7 @@ moba_status moba_meanpool(const moba_params* p, const void* k, const int* cu_seq
 
 moba_status moba_minmaxpool(const moba_params* p, const void* k, const int* cu_seqlens,
                             void* k_min, void* k_max, void* stream) {
+    NvtxScope range("moba_minmaxpool");
     moba_status s = check_params(p);
     if (s != MOBA_OK) return s;
     if (p->total_tokens == 0) return MOBA_OK;
@@ -205,6 +220,7 @@ moba_status moba_minmaxpool(const moba_params* p, const void* k, const int* cu_s
 
 moba_status moba_gate_topk(const moba_params* p, const void* q, const float* k_mean,
                            const int* cu_seqlens, int* sel, void* stream) {
+    NvtxScope range("moba_gate_topk");
     moba_status s = check_params(p);
     if (s != MOBA_OK) return s;
     if (p->total_tokens == 0) return MOBA_OK;
@@ -223,6 +239,7 @@ moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, co
                           const int* cu_seqlens, const int* sel_in, int* sel_out,
                           void* workspace, size_t workspace_bytes, void* out, float* lse,
                           moba_run_info* info, void* stream) {
+    NvtxScope range("moba_attn_fwd");
     moba_status s = check_params(p);
     if (s != MOBA_OK) return s;
     if (info) {
@@ -281,12 +298,16 @@ moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, co
     } while (0)
 
     MOBA_TRY(record(MOBA_EV_BEGIN), "event record");
-    MOBA_TRY(launch_plan_blocks(P, cu_seqlens, ws, st), "block table launch");
-    MOBA_TRY(launch_meanpool(P, kb, cu_seqlens, ws.means, st), "meanpool launch");
+    {
+        NvtxScope stage("means");
+        MOBA_TRY(launch_plan_blocks(P, cu_seqlens, ws, st), "block table launch");
+        MOBA_TRY(launch_meanpool(P, kb, cu_seqlens, ws.means, st), "meanpool launch");
+    }
     launches += 2;
     MOBA_TRY(record(MOBA_EV_MEANS_DONE), "event record");
     const int* sel_use = sel_in;
     if (!sel_use) {
+        NvtxScope stage("gate");
         int* dst = sel_out ? sel_out : ws.sel;
         MOBA_TRY(launch_gate_best(P, qb, ws.means, cu_seqlens, dst, &ws.hdr->status, st),
                  "gate launch");
@@ -301,17 +322,27 @@ moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, co
     for (int t0 = 0; t0 < T; t0 += L.wave, ++w) {
         const int t1 = (T - t0 > L.wave) ? t0 + L.wave : T;
         const int ev = MOBA_EV_WAVE0 + 4 * w;
+        NvtxScope wave("wave");
         MOBA_TRY(record(ev), "event record");
-        MOBA_TRY(cudaMemsetAsync(ws.counts, 0, 4ull * P.hkv * L.nb_cap, st), "memset");
-        MOBA_TRY(launch_route_count(P, cu_seqlens, sel_use, ws, t0, t1, st), "route count launch");
-        MOBA_TRY(launch_route_plan(P, ws, t0, t1, st), "route plan launch");
-        MOBA_TRY(launch_route_scatter(P, cu_seqlens, sel_use, ws, t0, t1, st), "route scatter launch");
+        {
+            NvtxScope stage("route");
+            MOBA_TRY(cudaMemsetAsync(ws.counts, 0, 4ull * P.hkv * L.nb_cap, st), "memset");
+            MOBA_TRY(launch_route_count(P, cu_seqlens, sel_use, ws, t0, t1, st), "route count launch");
+            MOBA_TRY(launch_route_plan(P, ws, t0, t1, st), "route plan launch");
+            MOBA_TRY(launch_route_scatter(P, cu_seqlens, sel_use, ws, t0, t1, st), "route scatter launch");
+        }
         MOBA_TRY(record(ev + 1), "event record");
-        MOBA_TRY(launch_attention(P, qb, kb, vb, ws, t0, t1, num_sms, st), "attention launch");
+        {
+            NvtxScope stage("attention");
+            MOBA_TRY(launch_attention(P, qb, kb, vb, ws, t0, t1, num_sms, st), "attention launch");
+        }
         MOBA_TRY(record(ev + 2), "event record");
-        MOBA_TRY(launch_merge(P, cu_seqlens, sel_use, ws, t0, t1,
-                              static_cast<__nv_bfloat16*>(out), lse, st),
-                 "merge launch");
+        {
+            NvtxScope stage("merge");
+            MOBA_TRY(launch_merge(P, cu_seqlens, sel_use, ws, t0, t1,
+                                  static_cast<__nv_bfloat16*>(out), lse, st),
+                     "merge launch");
+        }
         MOBA_TRY(record(ev + 3), "event record");
         launches += 5;
     }
@@ -396,6 +427,7 @@ moba_status decode_fwd(const moba_params* p, const void* q, const void* k, const
 moba_status moba_decode_fwd(const moba_params* p, const void* q, const void* k, const void* v,
                             const int* cu_seqlens, const float* k_mean, void* workspace,
                             size_t ws_bytes, void* out, float* lse, void* stream) {
+    NvtxScope range("moba_decode_fwd");
     return decode_fwd(p, q, k, v, cu_seqlens, DecodeGate{k_mean, nullptr, nullptr}, workspace, ws_bytes,
                       out, lse, stream);
 }
@@ -404,6 +436,7 @@ moba_status moba_decode_minmax_fwd(const moba_params* p, const void* q, const vo
                                    const int* cu_seqlens, const void* k_min, const void* k_max,
                                    void* workspace, size_t ws_bytes, void* out, float* lse,
                                    void* stream) {
+    NvtxScope range("moba_decode_minmax_fwd");
     return decode_fwd(p, q, k, v, cu_seqlens,
                       DecodeGate{nullptr, static_cast<const __nv_bfloat16*>(k_min),
                                  static_cast<const __nv_bfloat16*>(k_max)},
