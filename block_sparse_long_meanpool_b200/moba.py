@@ -323,19 +323,31 @@ def selftest_timeout(device=None, polls=4096):
 
 
 def choose_wave_tokens(T, hq, hkv, d, chunk_size, topk, batch, budget_bytes):
-    """Largest multiple of 128 query tokens per wave whose workspace fits in budget_bytes."""
+    """Query tokens per wave: 0 (one wave over all T tokens) when that workspace fits in
+    budget_bytes, else the largest multiple of 128 whose workspace fits, or 128 when even
+    that does not.  A wave also keeps wave * hq * topk below 2^31 (int32 partial indices).
+    The workspace size never decreases as the wave grows, so a bisection over multiples of
+    128 against moba_workspace_size finds the exact largest fit."""
     lib = load_library()
-    full = make_params(batch, T, hq, hkv, d, chunk_size, topk, None, 0)
-    if lib.moba_workspace_size(ctypes.byref(full)) <= budget_bytes and T * hq * topk < 2 ** 31:
+
+    def size(w):
+        return lib.moba_workspace_size(ctypes.byref(make_params(batch, T, hq, hkv, d, chunk_size, topk, None, w)))
+
+    if T * hq * topk < 2 ** 31 and size(0) <= budget_bytes:
         return 0
-    one = make_params(batch, T, hq, hkv, d, chunk_size, topk, None, 128)
-    base = lib.moba_workspace_size(ctypes.byref(one))
-    two = make_params(batch, T, hq, hkv, d, chunk_size, topk, None, 256)
-    per128 = max(lib.moba_workspace_size(ctypes.byref(two)) - base, 1)
-    n = max(1, int((budget_bytes - base) // per128) + 1)
-    n = min(n, (2 ** 31 - 1) // (hq * topk * 128))
-    w = 128 * max(n, 1)
-    return 0 if w >= T else w
+    hi = min((T - 1) // 128, (2 ** 31 - 1) // (hq * topk * 128))  # tiles of a wave shorter than T
+    if hi < 1:
+        return 0 if T <= 128 else 128
+    lo = 1
+    if size(128) > budget_bytes:
+        return 128
+    while lo < hi:
+        mid = (lo + hi + 1) // 2
+        if size(128 * mid) <= budget_bytes:
+            lo = mid
+        else:
+            hi = mid - 1
+    return 128 * lo
 
 
 def attn_fwd(q, k, v, cu_seqlens, chunk_size, topk, softmax_scale=None, sel=None,

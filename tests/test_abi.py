@@ -131,6 +131,43 @@ def test_workspace_grows_with_the_wave_and_block_bound(lib):
     assert lib.moba_num_blocks_bound(ctypes.byref(p)) == 4 + 2
 
 
+WAVE_CASES = [  # T, Hq, Hkv, d, chunk, topk, batch
+    (1 << 20, 32, 8, 128, 4096, 12, 1), (1 << 22, 32, 8, 128, 16384, 12, 1),
+    (10 << 20, 8, 2, 128, 40960, 12, 1), (63000, 32, 8, 128, 1024, 4, 4),
+    (32768, 32, 32, 128, 512, 3, 1), (32768, 32, 8, 128, 256, 32, 1), (2048, 4, 4, 64, 256, 3, 1),
+    (200000, 16, 16, 64, 128, 8, 50), (100, 4, 4, 64, 128, 3, 1),
+]
+
+
+def test_workspace_size_never_decreases_with_the_wave(lib):
+    for T, hq, hkv, d, chunk, topk, batch in WAVE_CASES:
+        waves = [128 * k for k in (1, 2, 3, 5, 8, 13, 100, 1000, 4000) if 128 * k < T] + [0]  # 0: one wave
+        sizes = [lib.moba_workspace_size(ctypes.byref(moba.make_params(batch, T, hq, hkv, d, chunk, topk, None, w)))
+                 for w in waves]
+        assert all(x > 0 for x in sizes) and sizes == sorted(sizes), (T, sizes)
+
+
+def test_wave_choice_is_the_largest_that_fits(lib):
+    """Every budget gets one wave when it fits, else the largest multiple of 128 whose
+    workspace fits (the next one does not), or 128 when nothing fits."""
+    for T, hq, hkv, d, chunk, topk, batch in WAVE_CASES:
+        def size(w):
+            return lib.moba_workspace_size(ctypes.byref(moba.make_params(batch, T, hq, hkv, d, chunk, topk, None, w)))
+        full = size(0)
+        for frac in (0.01, 0.05, 0.1, 0.3, 0.6, 0.9, 1.0, 1.1):
+            budget = int(full * frac)
+            w = moba.choose_wave_tokens(T, hq, hkv, d, chunk, topk, batch, budget)
+            if w == 0:
+                assert full <= budget or T <= 128
+                continue
+            assert w % 128 == 0 and 0 < w < T and w * hq * topk < 2 ** 31
+            if size(w) > budget:
+                assert w == 128, (T, frac, w)
+                continue
+            nxt = w + 128
+            assert nxt >= T or nxt * hq * topk >= 2 ** 31 or size(nxt) > budget, (T, frac, w)
+
+
 def test_wave_choice_respects_budget(lib):
     w = moba.choose_wave_tokens(1 << 20, 32, 8, 128, 4096, 12, 1, 8 << 30)
     assert w > 0 and w % 128 == 0
