@@ -167,8 +167,10 @@ moba_status moba_device_status(const moba_params* p, const void* workspace, void
  *   k, v             bf16 [T, Hkv, d] packed caches (cu_seqlens); each sequence's last row is
  *                    the new token's key / value
  *   cu_seqlens       int32 [batch + 1], device; an empty sequence yields out = 0, lse = -inf
- *   k_mean           fp32 [moba_num_blocks_bound(p), Hkv, d]: the block means moba_meanpool
- *                    computes for these caches (only complete earlier blocks are read)
+ *   k_mean           fp32 [NB, Hkv, d]: the block means moba_meanpool computes for these
+ *                    caches, NB >= the true block count (moba_num_blocks_bound(p) is always
+ *                    enough; only complete earlier blocks are read).  The Python binding,
+ *                    which cannot see the true count without a device sync, asks for the bound
  *   workspace        moba_decode_workspace_size(p) bytes, caller-owned device memory
  *   out              bf16 [batch, Hq, d]; lse fp32 [Hq, batch] (natural log, scale included)
  * Runs on the CUDA cores (HBM-bound: it streams the selected K/V blocks).  Asynchronous on
@@ -181,7 +183,7 @@ moba_status moba_decode_fwd(const moba_params* p, const void* q, const void* k, 
 /* The decode step with the min/max gate: as moba_decode_fwd, except that an earlier block j
  * is scored by s_j = sum_i max(q_i k_min[j, g, i], q_i k_max[j, g, i]) (fp32; Quest's bound of
  * q . k over the block), from the summary moba_minmaxpool computes for these caches:
- *   k_min, k_max   bf16 [moba_num_blocks_bound(p), Hkv, d] device each
+ *   k_min, k_max   bf16 [NB, Hkv, d] device each, NB as for k_mean
  * Same workspace (moba_decode_workspace_size), outputs, errors and limits. */
 moba_status moba_decode_minmax_fwd(const moba_params* p, const void* q, const void* k, const void* v,
                                    const int* cu_seqlens, const void* k_min, const void* k_max,
