@@ -286,3 +286,23 @@ def test_decode_binding_rejects_mismatched_buffers(lib):
         with pytest.raises(ValueError):
             moba._validate_decode(*args, chunk, topk)
             pytest.fail(f"case {i} accepted")
+
+
+def test_decode_workspace_follows_the_split_rule(lib):
+    """The decode workspace: selections and slot counts per (sequence, head) row, and fp32
+    partials for topk * splits key ranges per row.  splits doubles from 1 while the grid has
+    fewer than 1184 (row, block, range) tasks (8 per SM), every row's partials still fit one
+    warp's merge (topk * splits <= 64) and a range keeps at least 128 keys."""
+    def align(x):
+        return (x + 255) // 256 * 256
+
+    for batch, hq, d, chunk, topk in [(64, 32, 128, 512, 3), (16, 32, 128, 2048, 8), (1, 32, 128, 4096, 12),
+                                      (1, 4, 64, 128, 32), (3, 8, 64, 256, 1), (5000, 32, 128, 512, 3),
+                                      (2, 6, 128, 1024, 4)]:
+        s = 1
+        while batch * hq * topk * s < 1184 and topk * s * 2 <= 64 and chunk // (s * 2) >= 128:
+            s *= 2
+        rows, parts = batch * hq, topk * s
+        want = align(4 * rows * topk) + align(4 * rows) + align(4 * rows * parts * d) + align(4 * rows * parts)
+        p = moba.make_params(batch, 1 << 20, hq, hq // 2 if hq % 2 == 0 else hq, d, chunk, topk)
+        assert lib.moba_decode_workspace_size(ctypes.byref(p)) == want, (batch, hq, chunk, topk, s)
