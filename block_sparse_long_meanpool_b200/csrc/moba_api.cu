@@ -99,6 +99,14 @@ Layout make_layout(const moba_params& p) {
     L.nb_cap = blocks_bound(p);
     L.wave = (p.wave_tokens > 0 && p.wave_tokens < T) ? p.wave_tokens : (int)T;
     const long long W = L.wave;
+    // Work items of one wave (route_plan_kernel), bounded from above:
+    //  - history: a list of n routed rows gives ceil(n / 256) items <= n / 256 + 1, so all lists
+    //    give at most routed / 256 + min(lists, routed);
+    //  - current block: at most Hq items per 128-row query tile that overlaps the wave (head
+    //    pairs give Hkv * ceil(group / 2) <= Hq, MHA tile pairs fewer).  Blocks start on their
+    //    sequence's 128-token grid and only a sequence's last block is partial, so the tiles
+    //    overlapping W tokens number at most W / 128 + (partial blocks) + 2 (the blocks that
+    //    straddle the wave's ends), within W / 128 + min(NB, W) + 4.
     const long long lists = (long long)p.num_kv_heads * L.nb_cap;
     const long long routed = W * p.num_q_heads * (p.topk - 1);
     const long long past_items = routed / kTileM + (lists < routed ? lists : routed) + 1;
