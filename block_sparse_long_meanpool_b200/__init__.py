@@ -1,4 +1,5 @@
-"""B200-native MoBA (Mixture of Block Attention) causal prefill forward.
+"""B200-native MoBA (Mixture of Block Attention): the causal prefill forward, the decode step
+with the mean or the min/max block gate.
 
 The compute path is the C-ABI library ``libmoba.so`` (CUDA for sm_100a, headers in
 ``include/moba.h``); ``moba`` is its thin ctypes binding and ``workloads`` makes seeded
@@ -8,10 +9,13 @@ synthetic inputs.  Build the library with ``python -m block_sparse_long_meanpool
 from .moba import (  # noqa: F401
     MobaError,
     attn_fwd,
+    decode_fwd,
+    decode_minmax_fwd,
     gate_topk,
     load_library,
+    make_params,
     meanpool,
+    minmaxpool,
     num_blocks,
     workspace_size,
-    make_params,
 )

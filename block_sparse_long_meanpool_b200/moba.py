@@ -1,6 +1,7 @@
 """Thin ctypes binding of libmoba.so (include/moba.h).
 
-Argument marshalling only: every step of the forward runs in the library's CUDA kernels.
+Argument marshalling and shape checks only: every step of the forward and of the decode step
+runs in the library's CUDA kernels.
 PyTorch provides device memory, the current stream and events.  There is no fallback: if
 the library is missing or the tensors are not on a CUDA device, the calls raise.
 """
