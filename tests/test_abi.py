@@ -306,3 +306,19 @@ def test_decode_workspace_follows_the_split_rule(lib):
         want = align(4 * rows * topk) + align(4 * rows) + align(4 * rows * parts * d) + align(4 * rows * parts)
         p = moba.make_params(batch, 1 << 20, hq, hq // 2 if hq % 2 == 0 else hq, d, chunk, topk)
         assert lib.moba_decode_workspace_size(ctypes.byref(p)) == want, (batch, hq, chunk, topk, s)
+
+
+def test_product_package_never_touches_the_oracle():
+    """The oracle is test infrastructure: nothing under the package imports or names it."""
+    pkg = os.path.join(ROOT, "block_sparse_long_meanpool_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", text, flags=re.M), f
+                assert "oracle." not in text, f
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="build"):
+        moba.load_library(str(tmp_path / "libmoba.so"))
