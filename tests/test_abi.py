@@ -322,3 +322,59 @@ def test_product_package_never_touches_the_oracle():
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(RuntimeError, match="build"):
         moba.load_library(str(tmp_path / "libmoba.so"))
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "moba.h"
+
+/* A C99 client: every entry point linked, the host-side ones called, the compute ones on
+   their argument-error paths (nothing reaches a device). */
+int main(void) {
+    moba_params p;
+    memset(&p, 0, sizeof p);
+    p.batch = 1; p.total_tokens = 2048; p.num_q_heads = 4; p.num_kv_heads = 4;
+    p.head_dim = 64; p.chunk_size = 256; p.topk = 3;
+    printf("%d %zu %zu\n", moba_num_blocks_bound(&p), moba_workspace_size(&p), moba_decode_workspace_size(&p));
+    printf("%d %d %d %d %d %d %d %d %d %d\n",
+           (int)moba_meanpool(NULL, NULL, NULL, NULL, NULL),
+           (int)moba_minmaxpool(&p, NULL, NULL, NULL, NULL, NULL),
+           (int)moba_gate_topk(&p, NULL, NULL, NULL, NULL, NULL),
+           (int)moba_attn_fwd(&p, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL, NULL, NULL, NULL),
+           (int)moba_device_status(&p, NULL, NULL),
+           (int)moba_decode_fwd(&p, NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL, NULL, NULL),
+           (int)moba_decode_minmax_fwd(&p, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL, NULL, NULL),
+           (int)moba_selftest_timeout(NULL, 16, NULL),
+           (int)moba_attn_fwd_noalloc(NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL),
+           (int)MOBA_OK);
+    printf("%s|%s\n", moba_status_string(MOBA_ERR_WORKSPACE), moba_last_error());
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_every_entry_point_links(lib, tmp_path):
+    """include/moba.h compiles as C99 with warnings as errors, and a C program links and runs
+    against libmoba.so (C linkage of every declared entry point)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(moba.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), "-L", libdir, "-lmoba", "-Wl,-rpath," + libdir],
+                   check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60,
+                         env=dict(os.environ, CUDA_VISIBLE_DEVICES="")).stdout.splitlines()
+    nb, ws, dws = (int(x) for x in out[0].split())
+    assert nb == 8 and ws > 0 and dws > 0
+    codes = [int(x) for x in out[1].split()]
+    I, W = moba.ERR_INVALID_ARG, moba.ERR_WORKSPACE  # device_status with no workspace: WORKSPACE
+    assert codes == [I, I, I, I, W, I, I, I, I, moba.OK], codes
+    name, _ = out[2].split("|", 1)
+    assert name == lib.moba_status_string(moba.ERR_WORKSPACE).decode()
