@@ -8,6 +8,7 @@ GPU; it needs the NVIDIA driver only when a function is called.
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -38,19 +39,36 @@ def _stale():
     return any(os.path.getmtime(d) > t for d in deps if os.path.exists(d))
 
 
-def build(force=False, verbose=False):
-    """Compile every source into libmoba.so unless it is up to date.  Returns its path."""
-    if not force and not _stale():
-        return LIB
-    cmd = [nvcc()] + ARCH + FLAGS + ["-I", os.path.join(ROOT, "include"), "-I", CSRC]
-    if verbose:
-        cmd += ["-Xptxas", "-v"]
-    cmd += ["-shared", "-o", LIB + ".tmp"] + [os.path.join(CSRC, f) for f in SOURCES]
+def _run(cmd):
     proc = subprocess.run(cmd, capture_output=True, text=True)
     if proc.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + proc.stdout + proc.stderr)
+    return proc.stdout + proc.stderr
+
+
+def build(force=False, verbose=False):
+    """Compile every source into libmoba.so unless it is up to date.  Returns its path.
+
+    Each source is compiled to its own object in parallel (build/ beside the sources), then
+    the objects are linked into the shared library."""
+    if not force and not _stale():
+        return LIB
+    objdir = os.path.join(PKG, "build")
+    os.makedirs(objdir, exist_ok=True)
+    base = [nvcc()] + ARCH + FLAGS + ["-I", os.path.join(ROOT, "include"), "-I", CSRC]
     if verbose:
-        sys.stderr.write(proc.stdout + proc.stderr)
+        base += ["-Xptxas", "-v"]
+    objs, cmds = [], []
+    for f in SOURCES:
+        obj = os.path.join(objdir, f.replace(".cu", ".o"))
+        objs.append(obj)
+        cmds.append(base + ["-c", "-o", obj, os.path.join(CSRC, f)])
+    workers = max(1, min(len(cmds), os.cpu_count() or 1))
+    with ThreadPoolExecutor(workers) as pool:
+        logs = list(pool.map(_run, cmds))
+    if verbose:
+        sys.stderr.write("".join(logs))
+    _run([nvcc()] + ARCH + ["-cudart", "static", "-shared", "-o", LIB + ".tmp"] + objs)
     os.replace(LIB + ".tmp", LIB)
     return LIB
 

@@ -45,7 +45,8 @@ struct GateSmem {
 template <int D, int KMAX>
 __global__ void __launch_bounds__(kThreads, 1)
 gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restrict__ means,
-               const int* __restrict__ cu, Problem P, int* __restrict__ sel, int* status) {
+               const int* __restrict__ cu, Problem P, int* __restrict__ sel, int* status,
+               int n_cap) {
     using L = GateSmem<D>;
     constexpr int kHalfBytesQ = kTileM * 128;
     extern __shared__ uint8_t smem_raw[];
@@ -76,8 +77,11 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
     const int qtiles = (len + kTileM - 1) / kTileM;
     const int ntiles = qtiles * P.group;
 
-    if (n_route == 0) {
-        // nothing to score: every row takes its own block only
+    if (n_route == 0 || c > n_cap) {
+        // nothing to score: every row takes its own block only.  c > n_cap means the sequence
+        // is longer than the caller's max_seqlen promised: its rows keep the own block only
+        // and the call's status word (when there is one) records the broken promise.
+        if (c > n_cap && threadIdx.x == 0 && status) atomicExch(status, 1 /* INVALID_ARG */);
         for (int e = threadIdx.x; e < len * P.group; e += kThreads) {
             const int h = g * P.group + e / len;
             const int t = start + e % len;
@@ -299,7 +303,7 @@ cudaError_t launch_tc(const Problem& P, const __nv_bfloat16* q, const float* mea
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid(P.nb_cap, P.hkv);
-    gate_tc_kernel<D, KMAX><<<grid, kThreads, smem, st>>>(mq, means, cu, P, sel, status);
+    gate_tc_kernel<D, KMAX><<<grid, kThreads, smem, st>>>(mq, means, cu, P, sel, status, n_max);
     return cudaGetLastError();
 }
 
@@ -317,13 +321,17 @@ cudaError_t launch_tc_k(const Problem& P, const __nv_bfloat16* q, const float* m
 
 }  // namespace
 
-// Tensor-core gate when every sequence has at most kMaxPast + 1 blocks (bounded through the
-// block-count bound), else the fp32 CUDA-core gate.
+// Tensor-core gate when every sequence has at most kMaxPast + 1 blocks (P.max_blocks, from the
+// caller's max_seqlen, else the block-count bound of the whole call), else the fp32 CUDA-core
+// gate.  Shared memory and the MMA's N are sized for the longest sequence's past blocks.
 cudaError_t launch_gate_best(const Problem& P, const __nv_bfloat16* q, const float* means,
-                             const int* cu_seqlens, int* sel, int* status, cudaStream_t st) {
+                             const int* cu_seqlens, int* sel, int* status, cudaStream_t st,
+                             int* path) {
     if (P.nb_cap == 0) return cudaSuccess;
-    if (P.nb_cap > kMaxPast + 1) return launch_gate(P, q, means, cu_seqlens, sel, st);
-    const int n_max = ((P.nb_cap - 1) + 15) & ~15;  // largest c is nb_cap - 1
+    const bool cuda_cores = P.max_blocks > kMaxPast + 1;
+    if (path) *path = cuda_cores ? 2 : 1;
+    if (cuda_cores) return launch_gate(P, q, means, cu_seqlens, sel, st);
+    const int n_max = ((P.max_blocks - 1) + 15) & ~15;  // largest c is max_blocks - 1
     const int n_alloc = n_max < 16 ? 16 : n_max;
     if (P.d == 64) return launch_tc_k<64>(P, q, means, cu_seqlens, sel, status, n_alloc, st);
     return launch_tc_k<128>(P, q, means, cu_seqlens, sel, status, n_alloc, st);

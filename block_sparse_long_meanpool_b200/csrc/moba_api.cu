@@ -18,7 +18,7 @@ namespace {
 
 // Named NVTX range over a scope.  Without a profiler attached each push/pop is a no-op after a
 // one-time check; under nsys or ncu every launch is attributed to its entry point and stage,
-// e.g. `ncu --nvtx --nvtx-include "moba_attn_fwd/wave/attention/"` captures the attention
+// e.g. `ncu --clock-control none --nvtx --nvtx-include "moba_attn_fwd/wave/attention/"` captures the attention
 // launches only.
 struct NvtxScope {
     explicit NvtxScope(const char* name) { nvtxRangePushA(name); }
@@ -64,6 +64,13 @@ moba_status check_params(const moba_params* p) {
         return fail(MOBA_ERR_INVALID_ARG, "chunk_size must be >= 1 (got %d)", p->chunk_size);
     if (p->head_dim < 1) return fail(MOBA_ERR_INVALID_ARG, "head_dim must be >= 1");
     if (p->wave_tokens < 0) return fail(MOBA_ERR_INVALID_ARG, "wave_tokens must be >= 0");
+    if (p->max_seqlen < 0)
+        return fail(MOBA_ERR_INVALID_ARG, "max_seqlen must be >= 0 (got %d)", p->max_seqlen);
+    if (p->max_seqlen > 0 &&
+        (p->max_seqlen > p->total_tokens || (long long)p->batch * p->max_seqlen < p->total_tokens))
+        return fail(MOBA_ERR_INVALID_ARG,
+                    "max_seqlen %d inconsistent with %d tokens in %d sequences", p->max_seqlen,
+                    p->total_tokens, p->batch);
     if (!(p->softmax_scale == p->softmax_scale) || std::isinf(p->softmax_scale))
         return fail(MOBA_ERR_INVALID_ARG, "softmax_scale must be finite");
     if (p->head_dim != 64 && p->head_dim != 128)
@@ -150,6 +157,11 @@ Problem make_problem(const moba_params& p, long long nb_cap) {
     P.topk = p.topk;
     P.group = p.num_q_heads / p.num_kv_heads;
     P.nb_cap = (int)nb_cap;
+    P.max_blocks = (int)nb_cap;
+    if (p.max_seqlen > 0) {
+        const long long mb = (p.max_seqlen + (long long)p.chunk_size - 1) / p.chunk_size;
+        if (mb < nb_cap) P.max_blocks = (int)mb;
+    }
     P.scale = p.softmax_scale > 0.f ? p.softmax_scale : 1.0f / sqrtf((float)p.head_dim);
     P.scale_log2 = P.scale * 1.4426950408889634f;
     return P;
@@ -253,6 +265,7 @@ moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, co
     if (info) {
         info->launches = 0;
         info->waves = 0;
+        info->gate_path = MOBA_GATE_PATH_NONE;
     }
     if (p->total_tokens == 0) return MOBA_OK;
     if (!q || !k || !v || !cu_seqlens || !out || !lse)
@@ -317,8 +330,10 @@ moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, co
     if (!sel_use) {
         NvtxScope stage("gate");
         int* dst = sel_out ? sel_out : ws.sel;
-        MOBA_TRY(launch_gate_best(P, qb, ws.means, cu_seqlens, dst, &ws.hdr->status, st),
+        int path = MOBA_GATE_PATH_NONE;
+        MOBA_TRY(launch_gate_best(P, qb, ws.means, cu_seqlens, dst, &ws.hdr->status, st, &path),
                  "gate launch");
+        if (info) info->gate_path = path;
         ++launches;
         sel_use = dst;
     }

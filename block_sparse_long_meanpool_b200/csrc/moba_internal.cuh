@@ -38,6 +38,7 @@ struct Problem {
     int batch, T, hq, hkv, d, chunk, topk;
     int group;       // hq / hkv
     int nb_cap;      // capacity of per-block arrays (upper bound of the block count)
+    int max_blocks;  // most blocks one sequence may have (from max_seqlen), <= nb_cap
     float scale;     // softmax scale (natural units)
     float scale_log2;  // scale * log2(e)
 };
@@ -152,8 +153,11 @@ cudaError_t launch_minmaxpool(const Problem& P, const __nv_bfloat16* k, const in
                               __nv_bfloat16* kmin, __nv_bfloat16* kmax, cudaStream_t st);
 cudaError_t launch_gate(const Problem& P, const __nv_bfloat16* q, const float* means,
                         const int* cu_seqlens, int* sel, cudaStream_t st);
+// Runs the tensor-core gate when every sequence fits it, else the CUDA-core gate; *path (when
+// non-null) receives MOBA_GATE_PATH_TENSOR_CORES (1) or MOBA_GATE_PATH_CUDA_CORES (2).
 cudaError_t launch_gate_best(const Problem& P, const __nv_bfloat16* q, const float* means,
-                             const int* cu_seqlens, int* sel, int* status, cudaStream_t st);
+                             const int* cu_seqlens, int* sel, int* status, cudaStream_t st,
+                             int* path = nullptr);
 cudaError_t launch_route_count(const Problem& P, const int* cu_seqlens, const int* sel,
                                const Workspace& ws, int t0, int t1, cudaStream_t st);
 cudaError_t launch_route_plan(const Problem& P, const Workspace& ws, int t0, int t1,

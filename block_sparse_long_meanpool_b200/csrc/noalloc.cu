@@ -16,8 +16,11 @@
 //     counters, work cursor) at the start of each call and wave.  Calls whose work overlaps
 //     on the GPU (different streams, or different host threads) race on the array.
 //   - The first call on each device looks up the array's device address with
-//     cudaGetSymbolAddress while that device is current; that first call should come before
-//     any stream capture.
+//     cudaGetSymbolAddress while that device is current, and the address is kept for the
+//     life of the process; that first call should come before any stream capture, and
+//     destroying the device's primary context (cudaDeviceReset) invalidates the kept address.
+//   - The forward's status word (MOBA_ERR_DEVICE_TIMEOUT when a bounded device wait gives up)
+//     lives in the array; moba_device_status_noalloc reads it from the kept address.
 //   - The call allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
 #include <cuda_runtime.h>
 
@@ -25,6 +28,7 @@
 #include <mutex>
 
 #include "moba.h"
+#include "moba_internal.cuh"
 
 namespace moba {
 void set_error_message(const char* msg);
@@ -56,7 +60,45 @@ int fitting_wave(moba_params pp) {
     return 128 * lo;  // 0 when even one 128-token wave does not fit
 }
 
+// Kept scratch address of the current device, or nullptr when this process has not run an
+// allocation-free forward there.  Sets *dev.
+cudaError_t kept_scratch(int* dev, void** ptr) {
+    *ptr = nullptr;
+    const cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess) return e;
+    if (*dev < 0 || *dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    *ptr = g_scratch_ptr[*dev];
+    return cudaSuccess;
+}
+
 }  // namespace
+
+extern "C" moba_status moba_device_status_noalloc(void* stream) {
+    int dev = 0;
+    void* scratch = nullptr;
+    cudaError_t e = kept_scratch(&dev, &scratch);
+    if (e != cudaSuccess) {
+        moba::set_error_message(cudaGetErrorString(e));
+        return MOBA_ERR_CUDA;
+    }
+    if (!scratch) return MOBA_OK;  // no allocation-free forward ran on this device
+    // the workspace header sits at the start of the array
+    const moba::WsHeader* hdr = static_cast<const moba::WsHeader*>(scratch);
+    int word = 0;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    e = cudaMemcpyAsync(&word, &hdr->status, sizeof(int), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) {
+        moba::set_error_message(cudaGetErrorString(e));
+        return MOBA_ERR_CUDA;
+    }
+    if (word == 0) return MOBA_OK;
+    char msg[64];
+    snprintf(msg, sizeof(msg), "device status word %d", word);
+    moba::set_error_message(msg);
+    return (moba_status)word;
+}
 
 extern "C" moba_status moba_attn_fwd_noalloc(const moba_params* p, const void* q, const void* k,
                                             const void* v, const int* cu_seqlens, void* out,

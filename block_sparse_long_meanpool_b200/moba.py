@@ -28,6 +28,7 @@ EXPORTS = (
     "moba_decode_fwd",
     "moba_decode_minmax_fwd",
     "moba_device_status",
+    "moba_device_status_noalloc",
     "moba_selftest_timeout",
     "moba_status_string",
     "moba_last_error",
@@ -38,12 +39,15 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOU
 
 # moba_run_info event slots
 EV_BEGIN, EV_MEANS_DONE, EV_GATE_DONE, EV_WAVE0 = 0, 1, 2, 3
+# moba_run_info.gate_path
+GATE_PATH_NONE, GATE_PATH_TENSOR_CORES, GATE_PATH_CUDA_CORES = 0, 1, 2
 
 
 class MobaParams(ctypes.Structure):
     _fields_ = [
         ("batch", ctypes.c_int),
         ("total_tokens", ctypes.c_int),
+        ("max_seqlen", ctypes.c_int),
         ("num_q_heads", ctypes.c_int),
         ("num_kv_heads", ctypes.c_int),
         ("head_dim", ctypes.c_int),
@@ -60,6 +64,7 @@ class MobaRunInfo(ctypes.Structure):
         ("n_events", ctypes.c_int),
         ("launches", ctypes.c_int),
         ("waves", ctypes.c_int),
+        ("gate_path", ctypes.c_int),
     ]
 
 
@@ -106,6 +111,8 @@ def load_library(path=LIB_PATH):
     lib.moba_decode_minmax_fwd.restype = ctypes.c_int
     lib.moba_device_status.argtypes = [P, vp, vp]
     lib.moba_device_status.restype = ctypes.c_int
+    lib.moba_device_status_noalloc.argtypes = [vp]
+    lib.moba_device_status_noalloc.restype = ctypes.c_int
     lib.moba_selftest_timeout.argtypes = [vp, ctypes.c_uint, vp]
     lib.moba_selftest_timeout.restype = ctypes.c_int
     lib.moba_status_string.argtypes = [ctypes.c_int]
@@ -126,9 +133,9 @@ def _check(status):
 
 
 def make_params(batch, total_tokens, num_q_heads, num_kv_heads, head_dim, chunk_size, topk,
-                softmax_scale=None, wave_tokens=0):
-    return MobaParams(int(batch), int(total_tokens), int(num_q_heads), int(num_kv_heads),
-                      int(head_dim), int(chunk_size), int(topk),
+                softmax_scale=None, wave_tokens=0, max_seqlen=0):
+    return MobaParams(int(batch), int(total_tokens), int(max_seqlen or 0), int(num_q_heads),
+                      int(num_kv_heads), int(head_dim), int(chunk_size), int(topk),
                       float(softmax_scale) if softmax_scale else 0.0, int(wave_tokens))
 
 
@@ -254,14 +261,15 @@ def minmaxpool(k, cu_seqlens, chunk_size, num_blocks_out=None):
     return k_min[:nb], k_max[:nb]
 
 
-def gate_topk(q, k_mean, cu_seqlens, chunk_size, topk, num_kv_heads=None):
-    """Selections int32 [Hq, T, topk] (moba_gate_topk)."""
+def gate_topk(q, k_mean, cu_seqlens, chunk_size, topk, num_kv_heads=None, max_seqlen=None):
+    """Selections int32 [Hq, T, topk] (moba_gate_topk).  ``max_seqlen``: the longest sequence,
+    when known (sizes the gate per sequence rather than by the whole call's block count)."""
     _check_qkv(q, None)
     _require(k_mean.dtype == torch.float32 and k_mean.is_contiguous(), "k_mean must be fp32")
     batch = cu_seqlens.numel() - 1
     T, hq, d = q.shape
     hkv = num_kv_heads or k_mean.shape[1]
-    p = make_params(batch, T, hq, hkv, d, chunk_size, topk)
+    p = make_params(batch, T, hq, hkv, d, chunk_size, topk, max_seqlen=max_seqlen)
     _require_summary(k_mean, "k_mean", torch.float32, num_blocks_bound(p), hkv, d, q.device)
     sel = torch.empty((hq, T, topk), dtype=torch.int32, device=q.device)
     _check(load_library().moba_gate_topk(ctypes.byref(p), _ptr(q), _ptr(k_mean), _ptr(cu_seqlens),
@@ -314,6 +322,23 @@ def decode_minmax_fwd(q, k, v, cu_seqlens, k_min, k_max, chunk_size, topk, softm
                    softmax_scale, workspace, out, lse)
 
 
+def device_status(params, workspace):
+    """moba_device_status: raises MobaError when the status word a previous moba_attn_fwd left
+    in ``workspace`` is not MOBA_OK (waits for the current stream)."""
+    _check(load_library().moba_device_status(ctypes.byref(params), _ptr(workspace),
+                                             _stream(workspace.device)))
+
+
+def device_status_noalloc(device=None):
+    """moba_device_status_noalloc: raises MobaError when the most recent allocation-free forward
+    on ``device`` left an error in its status word (waits for the current stream)."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    _check(load_library().moba_device_status_noalloc(_stream(dev)))
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20  # MOBA_NOALLOC_SCRATCH_BYTES of include/moba.h
+
+
 def selftest_timeout(device=None, polls=4096):
     """moba_selftest_timeout: runs the bounded-wait self-test on `device` and returns the status
     word it left (MOBA_ERR_DEVICE_TIMEOUT when the wait expired as it must)."""
@@ -353,11 +378,12 @@ def choose_wave_tokens(T, hq, hkv, d, chunk_size, topk, batch, budget_bytes):
 
 def attn_fwd(q, k, v, cu_seqlens, chunk_size, topk, softmax_scale=None, sel=None,
              return_sel=False, wave_tokens=None, workspace=None, events=None,
-             workspace_budget=None, out=None, lse=None):
+             workspace_budget=None, out=None, lse=None, max_seqlen=None):
     """MoBA causal prefill forward (moba_attn_fwd).
 
     q bf16 [T, Hq, d], k/v bf16 [T, Hkv, d], cu_seqlens int32 [batch + 1] on the device.
     sel: optional int32 [Hq, T, topk] selection to use instead of the gate.
+    max_seqlen: the longest sequence's length when known on the host (0 / None: unknown).
     Returns (out bf16 [T, Hq, d], lse fp32 [Hq, T]) and, with return_sel, the gate's
     selection.  ``events`` may be a list of torch.cuda.Event recorded at the library's stage
     boundaries; the call's moba_run_info is returned in ``attn_fwd.last_info``.
@@ -374,7 +400,7 @@ def attn_fwd(q, k, v, cu_seqlens, chunk_size, topk, softmax_scale=None, sel=None
             free, _ = torch.cuda.mem_get_info(dev)
             workspace_budget = min(int(free * 0.45), 48 << 30)
         wave_tokens = choose_wave_tokens(T, hq, hkv, d, chunk_size, topk, batch, workspace_budget)
-    p = make_params(batch, T, hq, hkv, d, chunk_size, topk, softmax_scale, wave_tokens)
+    p = make_params(batch, T, hq, hkv, d, chunk_size, topk, softmax_scale, wave_tokens, max_seqlen)
     need = workspace_size(p)
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
@@ -407,7 +433,8 @@ def attn_fwd(q, k, v, cu_seqlens, chunk_size, topk, softmax_scale=None, sel=None
         ctypes.byref(info), _stream(dev))
     _check(status)
     attn_fwd.last_info = {"launches": info.launches, "waves": info.waves,
-                          "wave_tokens": wave_tokens, "workspace_bytes": need}
+                          "gate_path": info.gate_path, "wave_tokens": wave_tokens,
+                          "workspace_bytes": need}
     if return_sel and sel is None:
         return out, lse, sel_out
     return out, lse

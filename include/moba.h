@@ -59,6 +59,16 @@ typedef enum {
 typedef struct {
     int batch;            /* number of packed sequences, >= 1 */
     int total_tokens;     /* T = cu_seqlens[batch], >= 0 */
+    int max_seqlen;       /* length of the longest sequence, or 0 when not known on the host.
+                             When given it must satisfy max_seqlen <= T <= batch * max_seqlen
+                             (else MOBA_ERR_INVALID_ARG) and the caller guarantees that no
+                             sequence is longer; it sizes the gate by the most blocks one
+                             sequence has (ceil(max_seqlen / chunk_size)) instead of by the
+                             block count of the whole batch.  A sequence longer than a given
+                             max_seqlen never causes an out-of-bounds access: rows of its
+                             blocks past the bound may select their own block only, and
+                             moba_attn_fwd then records MOBA_ERR_INVALID_ARG in its status
+                             word (moba_device_status). */
     int num_q_heads;      /* Hq >= 1 */
     int num_kv_heads;     /* Hkv >= 1, Hq % Hkv == 0 */
     int head_dim;         /* d */
@@ -79,7 +89,15 @@ typedef struct {
     int n_events;
     int launches;    /* out: number of kernel launches the call queued */
     int waves;       /* out: number of query waves */
+    int gate_path;   /* out: which gate kernel ran, MOBA_GATE_PATH_* */
 } moba_run_info;
+
+enum {
+    MOBA_GATE_PATH_NONE = 0,         /* no gate (the selection came in through sel_in) */
+    MOBA_GATE_PATH_TENSOR_CORES = 1, /* tcgen05 gate: every sequence has <= 257 blocks (the
+                                        longest by max_seqlen, else the whole call's bound) */
+    MOBA_GATE_PATH_CUDA_CORES = 2    /* fp32 CUDA-core gate: a sequence may have more */
+};
 
 enum {
     MOBA_EV_BEGIN = 0,      /* before the first launch */
@@ -218,16 +236,27 @@ moba_status moba_selftest_timeout(int* status_dev, unsigned polls, void* stream)
  *     the bytes it would need.  Other arguments are checked as in moba_attn_fwd.
  *   - The caller still owns and passes q, k, v, cu_seqlens, out and lse (same layouts).
  *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call before any
- *     stream capture.
+ *     (cudaGetSymbolAddress) with that device current and keeps it for the life of the
+ *     process; make that first call before any stream capture.  cudaDeviceReset (or anything
+ *     else that destroys the device's primary context) invalidates the kept address: do not
+ *     call this entry point on that device afterwards.
  *   - All calls on a device share the array and it keeps the previous call's contents; the
  *     forward re-initialises everything it reads.  Calls whose GPU work overlaps (other
  *     streams or host threads on the same device) race on the array and must be serialised
- *     by the caller. */
+ *     by the caller.
+ *   - A bounded device-side wait that gives up records MOBA_ERR_DEVICE_TIMEOUT in the array;
+ *     read it with moba_device_status_noalloc. */
 #define MOBA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 moba_status moba_attn_fwd_noalloc(const moba_params* p, const void* q, const void* k,
                                   const void* v, const int* cu_seqlens, void* out, float* lse,
                                   void* stream);
+
+/* The device status word of the most recent moba_attn_fwd_noalloc on the current device:
+ * MOBA_OK, or MOBA_ERR_DEVICE_TIMEOUT when one of its bounded device-side waits gave up.
+ * Waits for `stream` (enqueue it on the stream the forward ran on).  Returns MOBA_OK without
+ * touching the device when no allocation-free forward has run on the current device in this
+ * process, and MOBA_ERR_CUDA when the device cannot be queried or read.  Allocates nothing. */
+moba_status moba_device_status_noalloc(void* stream);
 
 /* Static description of a status code. */
 const char* moba_status_string(moba_status s);

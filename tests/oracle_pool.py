@@ -1,0 +1,193 @@
+"""The float64 oracle on many host cores, for the full-size GPU parity tests.
+
+Test infrastructure only.  Nothing here computes any part of the method: every function
+below calls an ``oracle`` function unchanged on an independent piece of the problem (one
+query head, or one group of sampled rows of one KV head) and the pieces are spread over
+worker processes.  Rows of different heads are independent in the definition (the analysis
+page of the MoBA paper, §2.2-§2.3: the gate and the attention are per query row and per
+query head), so the pieces together are exactly the oracle's result.
+
+The pool is started with the ``spawn`` method: the test process has already initialised CUDA,
+and a child forked from it can hang.  Inputs travel as bf16 bit patterns (uint16) and are
+widened exactly inside the worker.  Each worker runs one BLAS thread.
+"""
+
+import math
+import multiprocessing as mp
+import os
+from concurrent.futures import ProcessPoolExecutor
+
+import numpy as np
+
+import oracle
+import parity as PT
+
+
+def n_workers():
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        n = os.cpu_count() or 1
+    return max(1, min(n, int(os.environ.get("MOBA_ORACLE_WORKERS", "32"))))
+
+
+def _init_worker():
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(1)
+    except Exception:  # pragma: no cover
+        pass
+
+
+def pool():
+    """A spawn-started process pool (use as a context manager)."""
+    return ProcessPoolExecutor(n_workers(), mp_context=mp.get_context("spawn"),
+                               initializer=_init_worker)
+
+
+# ---- worker tasks (top level, so that they pickle) ------------------------------------------
+
+def _dense_head(q16, k16, v16, cu, chunk, sel_h, scale):
+    """oracle.attention_masked_dense for one query head: q16 [T, d], k16 / v16 [T, d] of its
+    KV head, sel_h [T, topk].  Returns out [T, d], lse [T]."""
+    q = PT.from_bits(q16)[:, None, :]
+    k = PT.from_bits(k16)[:, None, :]
+    v = PT.from_bits(v16)[:, None, :]
+    out, lse = oracle.attention_masked_dense(q, k, v, cu, chunk, sel_h[None], scale)
+    return out[:, 0, :], lse[0]
+
+
+def _select_head(q16, means_g, cu, chunk, topk):
+    """oracle.select_blocks for one query head against its KV head's block summary.
+    Returns [T, topk] int16."""
+    q = PT.from_bits(q16)[:, None, :]
+    sel = oracle.select_blocks(q, means_g[:, None, :], cu, chunk, topk)
+    return sel[0].astype(np.int16)
+
+
+def _compare_head(gsel_h, osel_h, q16, means_g, cu, chunk, topk):
+    """Rows of one head whose GPU selection differs from the oracle's: returns (tokens of the
+    rows that are valid near-tie alternatives, list of the other rows)."""
+    diff = np.nonzero((gsel_h != osel_h).any(axis=1))[0]
+    ties, bad = [], []
+    for t in diff:
+        t = int(t)
+        _, b0, c = PT.row_block(cu, chunk, t)
+        sc = oracle.gate_scores_row(PT.from_bits(q16[t]).astype(np.float64), means_g[b0:b0 + c])
+        if PT.near_tie_alternative(gsel_h[t], osel_h[t], sc, c, topk):
+            ties.append(t)
+        else:
+            bad.append((t, [int(x) for x in gsel_h[t]], [int(x) for x in osel_h[t]]))
+    return np.asarray(ties, dtype=np.int64), bad
+
+
+def _select_rows(q_rows16, ts, means_g, cu, chunk, topk):
+    """oracle.select_blocks_rows for sampled tokens of one query head."""
+    return oracle.select_blocks_rows(_RowsView(q_rows16, ts), means_g[:, None, :], cu, chunk, topk,
+                                     [(int(t), i) for i, t in enumerate(ts)])
+
+
+def _attend(q_rows16, ts, k16, v16, cu, chunk, sel_rows, scale):
+    """oracle.attend_rows for sampled tokens of query heads of one KV head: q_rows16 [n, d]
+    (each row's own query), ts [n], k16 / v16 [T, d], sel_rows [n, topk]."""
+    k = PT.from_bits(k16)[:, None, :]
+    v = PT.from_bits(v16)[:, None, :]
+    return oracle.attend_rows(_RowsView(q_rows16, ts), k, v, cu, chunk, sel_rows,
+                              [(int(t), i) for i, t in enumerate(ts)], scale)
+
+
+class _RowsView:
+    """q stand-in for oracle.attend_rows / select_blocks_rows over n sampled rows that all read
+    one KV head: row (t, i) is the i-th sampled row's query.  With n "heads" against one KV
+    head, the oracle's GQA mapping sends every row to that KV head."""
+
+    def __init__(self, q_rows16, ts):
+        self.q = q_rows16
+        self.ts = np.asarray(ts)
+        self.shape = (None, len(ts), q_rows16.shape[1])
+
+    def __getitem__(self, idx):
+        t, i = idx
+        assert int(self.ts[i]) == int(t)
+        return PT.from_bits(self.q[i])
+
+
+# ---- drivers used by the tests -----------------------------------------------------------------
+
+def dense_all_heads(ex, q16, k16, v16, cu, chunk, sel, scale=None):
+    """oracle.attention_masked_dense over all heads: q16 [T, Hq, d], k16 / v16 [T, Hkv, d]
+    (bf16 bits), sel [Hq, T, topk].  Returns out [T, Hq, d], lse [Hq, T] (float64)."""
+    T, hq, d = q16.shape
+    group = hq // k16.shape[1]
+    futs = [ex.submit(_dense_head, np.ascontiguousarray(q16[:, h]), np.ascontiguousarray(k16[:, h // group]),
+                      np.ascontiguousarray(v16[:, h // group]), cu, chunk, np.ascontiguousarray(sel[h]), scale)
+            for h in range(hq)]
+    out = np.zeros((T, hq, d))
+    lse = np.zeros((hq, T))
+    for h, f in enumerate(futs):
+        out[:, h], lse[h] = f.result()
+    return out, lse
+
+
+def select_and_compare_heads(ex, q_head16, means, gsel, cu, chunk, topk, group, heads):
+    """oracle.select_blocks per listed head, compared with the GPU's selection of that head.
+    q_head16(h) returns that head's q bits [T, d]; gsel(h) its GPU selection [T, topk].
+    Returns {h: (oracle selection [T, topk] int16, tie tokens)}; fails on any row that is not
+    a valid near-tie alternative."""
+    sel_f = {h: ex.submit(_select_head, q_head16(h), np.ascontiguousarray(means[:, h // group]), cu,
+                          chunk, topk) for h in heads}
+    res, cmp_f = {}, {}
+    for h in heads:
+        osel = sel_f[h].result()
+        g = gsel(h)
+        res[h] = osel
+        cmp_f[h] = ex.submit(_compare_head, g, osel, q_head16(h), np.ascontiguousarray(means[:, h // group]),
+                             cu, chunk, topk)
+    out = {}
+    bad = []
+    for h in heads:
+        ties, b = cmp_f[h].result()
+        bad += [(h,) + x for x in b]
+        out[h] = (res[h], ties)
+    assert not bad, f"{len(bad)} selection mismatches outside the near-tie band: {bad[:5]}"
+    return out
+
+
+def attend_rows_par(ex, rows, q_row16, k16, v16, cu, chunk, sel_rows, group, scale=None):
+    """oracle.attend_rows for sampled (t, h) rows, grouped by KV head.  q_row16 [n, d] holds
+    each row's query bits, sel_rows [n, topk] its selection, k16 / v16 [T, Hkv, d] the keys
+    and values (bf16 bits).  Returns out [n, d], lse [n] in the order of ``rows``.  About one
+    task per worker, so that each KV head's keys and values travel to few workers."""
+    n = len(rows)
+    rows_per_task = max(256, math.ceil(n / n_workers()))
+    g_of = np.array([h // group for _, h in rows])
+    ts = np.array([t for t, _ in rows])
+    futs = []
+    for g in np.unique(g_of):
+        idx = np.nonzero(g_of == g)[0]
+        kg = np.ascontiguousarray(k16[:, g])
+        vg = np.ascontiguousarray(v16[:, g])
+        n_tasks = max(1, math.ceil(len(idx) / rows_per_task))
+        for part in np.array_split(idx, n_tasks):
+            futs.append((part, ex.submit(_attend, q_row16[part], ts[part], kg, vg, cu, chunk,
+                                         sel_rows[part], scale)))
+    out = np.zeros((n, q_row16.shape[1]))
+    lse = np.zeros(n)
+    for part, f in futs:
+        out[part], lse[part] = f.result()
+    return out, lse
+
+
+def select_rows_par(ex, rows, q_row16, means, cu, chunk, topk, group):
+    """oracle.select_blocks_rows for sampled (t, h) rows, one task per head."""
+    hs = np.array([h for _, h in rows])
+    ts = np.array([t for t, _ in rows])
+    res = np.zeros((len(rows), topk), dtype=np.int64)
+    futs = []
+    for h in np.unique(hs):
+        idx = np.nonzero(hs == h)[0]
+        futs.append((idx, ex.submit(_select_rows, q_row16[idx], ts[idx],
+                                    np.ascontiguousarray(means[:, h // group]), cu, chunk, topk)))
+    for idx, f in futs:
+        res[idx] = f.result()
+    return res

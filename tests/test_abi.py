@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def params(**kw):
     base = dict(batch=1, total_tokens=2048, num_q_heads=4, num_kv_heads=4, head_dim=64,
-                chunk_size=256, topk=3, softmax_scale=None, wave_tokens=0)
+                chunk_size=256, topk=3, softmax_scale=None, wave_tokens=0, max_seqlen=0)
     base.update(kw)
     return moba.make_params(**base)
 
@@ -53,6 +53,9 @@ def params(**kw):
     (dict(chunk_size=100), moba.ERR_UNSUPPORTED),
     (dict(topk=33), moba.ERR_UNSUPPORTED),
     (dict(wave_tokens=100), moba.ERR_UNSUPPORTED),
+    (dict(max_seqlen=-1), moba.ERR_INVALID_ARG),
+    (dict(max_seqlen=4096), moba.ERR_INVALID_ARG),             # longer than all tokens
+    (dict(batch=2, max_seqlen=1000), moba.ERR_INVALID_ARG),    # 2 x 1000 < 2048 tokens
 ])
 def test_invalid_params_are_rejected(lib, kw, status):
     p = params(**kw)
@@ -115,6 +118,20 @@ def test_workspace_and_alignment_checks_precede_any_launch(lib):
     rc = lib.moba_attn_fwd(ctypes.byref(big), fake, fake, fake, fake, None, None, fake,
                            need_big, fake, fake, None, None)
     assert rc == moba.ERR_UNSUPPORTED
+
+
+def test_max_seqlen_is_accepted_when_consistent(lib):
+    for kw in (dict(max_seqlen=2048), dict(batch=2, max_seqlen=1024), dict(batch=3, max_seqlen=1500)):
+        assert lib.moba_workspace_size(ctypes.byref(params(**kw))) > 0, kw
+
+
+def test_noalloc_status_read_without_a_forward(lib):
+    """With no allocation-free forward run in this process there is nothing to read: OK, or a
+    CUDA error when no device can be queried (this host has none); never a device access."""
+    rc = lib.moba_device_status_noalloc(None)
+    assert rc in (moba.OK, moba.ERR_CUDA), rc
+    if rc == moba.ERR_CUDA:
+        assert lib.moba_last_error()
 
 
 def test_status_strings(lib):
@@ -348,6 +365,7 @@ int main(void) {
            (int)moba_selftest_timeout(NULL, 16, NULL),
            (int)moba_attn_fwd_noalloc(NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL),
            (int)MOBA_OK);
+    printf("%d\n", (int)moba_device_status_noalloc(NULL));
     printf("%s|%s\n", moba_status_string(MOBA_ERR_WORKSPACE), moba_last_error());
     return 0;
 }
@@ -376,5 +394,6 @@ def test_header_is_plain_c_and_every_entry_point_links(lib, tmp_path):
     codes = [int(x) for x in out[1].split()]
     I, W = moba.ERR_INVALID_ARG, moba.ERR_WORKSPACE  # device_status with no workspace: WORKSPACE
     assert codes == [I, I, I, I, W, I, I, I, I, moba.OK], codes
-    name, _ = out[2].split("|", 1)
+    assert int(out[2]) in (moba.OK, moba.ERR_CUDA)
+    name, _ = out[3].split("|", 1)
     assert name == lib.moba_status_string(moba.ERR_WORKSPACE).decode()

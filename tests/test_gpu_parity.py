@@ -1,17 +1,22 @@
 """GPU parity: the CUDA path, called through the C ABI, against the float64 oracle.
 
-Every case feeds the same seeded bf16 inputs to both sides.  Small cases are checked on all
-rows; the full-size workloads on all means, all selections (or whole heads at 1M) and
-sampled output rows.  Tolerances are in ``parity.py``.
+Every case feeds the same seeded bf16 inputs to both sides.  Selections are compared in full
+(every row of every head) except on the length sweep, where whole heads and sampled rows are
+compared; a row may differ only as a valid near-tie alternative (``parity.check_selection``),
+and such a row's output is checked against the oracle's attention over the GPU's own
+selection.  Outputs are compared on all rows for the small cases and the scaling, long and
+varlen workloads, and on sampled rows (4096 per head at 1M) for the larger ones; then the
+oracle's selection is fed back (``sel_in``) and the outputs must match with no exception.
+The full-size checks run the oracle on the host cores through ``oracle_pool``.  Tolerances
+are in ``parity.py``.
 """
-
-import os
 
 import numpy as np
 import pytest
 import torch
 
 import oracle
+import oracle_pool as OP
 import parity as PT
 from block_sparse_long_meanpool_b200 import build, moba
 from block_sparse_long_meanpool_b200 import workloads as W
@@ -23,6 +28,12 @@ pytestmark = pytest.mark.gpu
 def library():
     build.build()
     moba.load_library()
+
+
+@pytest.fixture(scope="module")
+def ex():
+    with OP.pool() as e:
+        yield e
 
 
 SMALL = [
@@ -51,15 +62,31 @@ def gpu_inputs(w):
 
 
 def full_sel_check(gsel, osel, q_np, om, cu, chunk, topk, group):
-    """Compare [Hq, T, topk] selections; returns a boolean [Hq, T] mask of near-tie rows."""
+    """Compare [Hq, T, topk] selections; returns the (t, h) rows whose GPU selection is a valid
+    near-tie alternative to the oracle's (any other difference fails)."""
     diff = np.nonzero((gsel != osel).any(axis=2))
     rows = [(int(t), int(h)) for h, t in zip(*diff)]
     ties = PT.check_selection(gsel[diff], osel[diff], rows, q_np, om, cu, chunk, topk, group)
-    mask = np.zeros(gsel.shape[:2], dtype=bool)
-    for r in ties:
-        t, h = rows[r]
-        mask[h, t] = True
-    return mask
+    return [rows[r] for r in sorted(ties)]
+
+
+def with_tie_rows(ref_o, ref_l, ties, gsel, q_np, k_np, v_np, cu, chunk, scale=None):
+    """Copies of the oracle's out [T, Hq, d] / lse [Hq, T] in which every near-tie row holds the
+    oracle's attention over the GPU's selection of that row."""
+    ref_o, ref_l = ref_o.copy(), ref_l.copy()
+    if ties:
+        sel_rows = np.stack([gsel[h, t] for t, h in ties])
+        o, l = oracle.attend_rows(q_np, k_np, v_np, cu, chunk, sel_rows, ties, scale)
+        for i, (t, h) in enumerate(ties):
+            ref_o[t, h] = o[i]
+            ref_l[h, t] = l[i]
+    return ref_o, ref_l
+
+
+def check_all_rows(out, lse, ref_o, ref_l):
+    T, hq = out.shape[0], out.shape[1]
+    return PT.check_out(PT.host(out).reshape(T * hq, -1), PT.host(lse).T.reshape(-1),
+                        ref_o.reshape(T * hq, -1), ref_l.T.reshape(-1))
 
 
 @pytest.mark.parametrize("w", SMALL, ids=[w.name for w in SMALL])
@@ -70,28 +97,23 @@ def test_small_all_rows(w):
     nb = moba.num_blocks(w.seqlens, chunk)
     means = moba.meanpool(k, cu_t, chunk, num_blocks_out=nb)
     sel_gate = moba.gate_topk(q, means, cu_t, chunk, topk)
-    out, lse, sel = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True)
+    out, lse, sel = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True, max_seqlen=w.max_seqlen)
     torch.cuda.synchronize()
     q_np, k_np, v_np = PT.host(q), PT.host(k), PT.host(v)
     ref = oracle.moba_forward(q_np, k_np, v_np, cu, chunk, topk)
 
     PT.check_means(PT.host(means), k_np, cu, chunk, ref["means"])
     gsel = PT.host(sel, np.int64)
+    # the gate sized by the batch's block bound and by max_seqlen select the same blocks
     np.testing.assert_array_equal(gsel, PT.host(sel_gate, np.int64))
     ties = full_sel_check(gsel, ref["sel"], q_np, ref["means"], cu, chunk, topk, group)
-
-    T, hq = q.shape[0], q.shape[1]
-    rows = [(t, h) for t in range(T) for h in range(hq)]
-    keep_skip = [i for i, (t, h) in enumerate(rows) if ties[h, t]]
-    out_np, lse_np = PT.host(out), PT.host(lse)
-    PT.check_out(out_np.reshape(T * hq, -1), lse_np.T.reshape(-1),
-                 ref["out"].reshape(T * hq, -1), ref["lse"].T.reshape(-1), skip=keep_skip)
+    ref_o, ref_l = with_tie_rows(ref["out"], ref["lse"], ties, gsel, q_np, k_np, v_np, cu, chunk)
+    check_all_rows(out, lse, ref_o, ref_l)
 
     # oracle-feed mode: the oracle's selection, no exceptions
     fed = torch.from_numpy(ref["sel"].astype(np.int32)).cuda()
     out2, lse2 = moba.attn_fwd(q, k, v, cu_t, chunk, topk, sel=fed)
-    PT.check_out(PT.host(out2).reshape(T * hq, -1), PT.host(lse2).T.reshape(-1),
-                 ref["out"].reshape(T * hq, -1), ref["lse"].T.reshape(-1))
+    check_all_rows(out2, lse2, ref["out"], ref["lse"])
 
 
 def test_waves_give_bitwise_identical_results():
@@ -120,8 +142,7 @@ def test_forced_selections_window_and_sink():
                 sel[:, t, :len(js)] = js
         ref_o, ref_l = oracle.attention_masked_dense(q_np, k_np, v_np, cu, 128, sel)
         out, lse = moba.attn_fwd(q, k, v, cu_t, 128, 3, sel=torch.from_numpy(sel.astype(np.int32)).cuda())
-        PT.check_out(PT.host(out).reshape(T * hq, -1), PT.host(lse).T.reshape(-1),
-                     ref_o.reshape(T * hq, -1), ref_l.T.reshape(-1))
+        check_all_rows(out, lse, ref_o, ref_l)
 
 
 def test_fed_selection_rule_ignores_invalid_entries():
@@ -154,20 +175,22 @@ def test_empty_input():
 def test_softmax_scale_parameter():
     w = W.custom("scaled", [777], 2, 2, 128, 128, 2, "k_offsets", 23)
     q, k, v, cu_t = gpu_inputs(w)
-    out, lse = moba.attn_fwd(q, k, v, cu_t, 128, 2, softmax_scale=0.05)
+    out, lse, sel = moba.attn_fwd(q, k, v, cu_t, 128, 2, softmax_scale=0.05, return_sel=True)
     cu = np.asarray(w.cu_seqlens)
-    ref = oracle.moba_forward(PT.host(q), PT.host(k), PT.host(v), cu, 128, 2, scale=0.05)
-    T = q.shape[0]
-    PT.check_out(PT.host(out).reshape(T * 2, -1), PT.host(lse).T.reshape(-1),
-                 ref["out"].reshape(T * 2, -1), ref["lse"].T.reshape(-1))
+    q_np, k_np, v_np = PT.host(q), PT.host(k), PT.host(v)
+    ref = oracle.moba_forward(q_np, k_np, v_np, cu, 128, 2, scale=0.05)
+    gsel = PT.host(sel, np.int64)
+    ties = full_sel_check(gsel, ref["sel"], q_np, ref["means"], cu, 128, 2, 1)
+    ref_o, ref_l = with_tie_rows(ref["out"], ref["lse"], ties, gsel, q_np, k_np, v_np, cu, 128, 0.05)
+    check_all_rows(out, lse, ref_o, ref_l)
 
 
-FULL = ["scaling_8k", "long_32k", "varlen_gqa", "fine_32k_8_2", "fine_32k_128_32"]
+# ---- full-size workloads ------------------------------------------------------------------
 
-
-@pytest.mark.parametrize("name", FULL)
-def test_full_size_workload(name):
-    """All means, all selections, sampled output rows; then the oracle-feed mode."""
+@pytest.mark.parametrize("name", ["scaling_8k", "long_32k", "varlen_gqa"])
+def test_full_size_all_rows(name, ex):
+    """All means, all selections and all output rows (masked-dense oracle over every head),
+    then the oracle-feed mode on all rows."""
     w = W.ALL_WORKLOADS[name]
     q, k, v, cu_t = gpu_inputs(w)
     cu = np.asarray(w.cu_seqlens)
@@ -175,123 +198,239 @@ def test_full_size_workload(name):
     group = hq // w.num_kv_heads
     nb = moba.num_blocks(w.seqlens, chunk)
     means = moba.meanpool(k, cu_t, chunk, num_blocks_out=nb)
-    out, lse, sel = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True)
+    out, lse, sel = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True, max_seqlen=w.max_seqlen)
     torch.cuda.synchronize()
-    q_np, k_np, v_np = PT.host(q, np.float32), PT.host(k, np.float32), PT.host(v, np.float32)
+    q16, k16, v16 = PT.bf16_bits(q), PT.bf16_bits(k), PT.bf16_bits(v)
+    q_np, k_np, v_np = PT.from_bits(q16), PT.from_bits(k16), PT.from_bits(v16)
     om = oracle.block_means(k_np, cu, chunk)
     PT.check_means(PT.host(means), k_np, cu, chunk, om)
     osel = oracle.select_blocks(q_np, om, cu, chunk, topk)
     gsel = PT.host(sel, np.int64)
     ties = full_sel_check(gsel, osel, q_np, om, cu, chunk, topk, group)
-    assert ties.mean() < 1e-3
+    assert len(ties) < 1e-3 * gsel.shape[0] * gsel.shape[1]
 
-    rows = PT.sample_rows(cu, chunk, hq, topk, 768, 256, seed=31)
-    ref_o, ref_l = oracle.attend_rows(q_np, k_np, v_np, cu, chunk, osel, rows)
-    out_np, lse_np = PT.host(out, np.float32), PT.host(lse)
-    g_o = np.stack([out_np[t, h] for t, h in rows])
-    g_l = np.array([lse_np[h, t] for t, h in rows])
-    skip = [i for i, (t, h) in enumerate(rows) if ties[h, t]]
-    PT.check_out(g_o, g_l, ref_o, ref_l, skip=skip)
+    ref_o, ref_l = OP.dense_all_heads(ex, q16, k16, v16, cu, chunk, osel)
+    t_o, t_l = with_tie_rows(ref_o, ref_l, ties, gsel, q_np, k_np, v_np, cu, chunk)
+    check_all_rows(out, lse, t_o, t_l)
 
     fed = torch.from_numpy(osel.astype(np.int32)).cuda()
     out2, lse2 = moba.attn_fwd(q, k, v, cu_t, chunk, topk, sel=fed)
-    out2_np, lse2_np = PT.host(out2, np.float32), PT.host(lse2)
-    PT.check_out(np.stack([out2_np[t, h] for t, h in rows]),
-                 np.array([lse2_np[h, t] for t, h in rows]), ref_o, ref_l)
+    check_all_rows(out2, lse2, ref_o, ref_l)
 
 
-def test_prefill_1m_sampled():
-    """1,048,576 tokens, 32 q / 8 kv heads, chunk 4096, top-12, in the wave configuration the
-    bench uses: all block means, whole-head selections for four heads (one per two KV
-    heads) plus sampled rows of every head, sampled output rows, and a fed selection."""
-    w = W.WORKLOADS["prefill_1m"]
+@pytest.mark.parametrize("name", ["fine_32k_8_2", "fine_32k_128_32"])
+def test_granularity_sweep_sampled(name, ex):
+    """Block granularity at 75% sparsity (8 blocks / top-2 and 128 blocks / top-32 at 32K):
+    all means and selections, sampled output rows, and the oracle-feed mode."""
+    w = W.ALL_WORKLOADS[name]
+    q, k, v, cu_t = gpu_inputs(w)
+    cu = np.asarray(w.cu_seqlens)
+    chunk, topk, hq = w.chunk_size, w.topk, w.num_q_heads
+    group = hq // w.num_kv_heads
+    nb = moba.num_blocks(w.seqlens, chunk)
+    means = moba.meanpool(k, cu_t, chunk, num_blocks_out=nb)
+    out, lse, sel = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True, max_seqlen=w.max_seqlen)
+    torch.cuda.synchronize()
+    q16, k16, v16 = PT.bf16_bits(q), PT.bf16_bits(k), PT.bf16_bits(v)
+    q_np, k_np = PT.from_bits(q16), PT.from_bits(k16)
+    om = oracle.block_means(k_np, cu, chunk)
+    PT.check_means(PT.host(means), k_np, cu, chunk, om)
+    osel = oracle.select_blocks(q_np, om, cu, chunk, topk)
+    gsel = PT.host(sel, np.int64)
+    ties = full_sel_check(gsel, osel, q_np, om, cu, chunk, topk, group)
+    assert len(ties) < 1e-3 * gsel.shape[0] * gsel.shape[1]
+
+    rows = sorted(set(PT.sample_rows(cu, chunk, hq, topk, 768, 256, seed=31)) | set(ties))
+    ts = np.array([t for t, _ in rows])
+    hs = np.array([h for _, h in rows])
+    q_rows = q16[ts, hs]
+    g_rows, o_rows = gsel[hs, ts], osel[hs, ts]
+    ref_g = OP.attend_rows_par(ex, rows, q_rows, k16, v16, cu, chunk, g_rows, group)
+    ref_f = OP.attend_rows_par(ex, rows, q_rows, k16, v16, cu, chunk, o_rows, group)
+    PT.check_out(PT.host(out[ts, hs]), PT.host(lse[hs, ts]), *ref_g)
+
+    fed = torch.from_numpy(osel.astype(np.int32)).cuda()
+    out2, lse2 = moba.attn_fwd(q, k, v, cu_t, chunk, topk, sel=fed)
+    PT.check_out(PT.host(out2[ts, hs]), PT.host(lse2[hs, ts]), *ref_f)
+
+
+class _Bf16Rows:
+    """Slices of a [T, ...] array of bf16 bits, widened on access (check_means reads the keys
+    block by block)."""
+
+    def __init__(self, u16):
+        self.u16 = u16
+
+    def __getitem__(self, sl):
+        return PT.from_bits(self.u16[sl])
+
+
+def _block_means_by_block(k16, w):
+    """The oracle's block means of a single-sequence workload, one block at a time (blocks
+    are independent), so that the keys are never widened all at once."""
+    chunk = w.chunk_size
+    nb = moba.num_blocks(w.seqlens, chunk)
+    return np.concatenate([oracle.block_means(PT.from_bits(k16[b * chunk:(b + 1) * chunk]),
+                                              [0, min(chunk, w.total_tokens - b * chunk)], chunk)
+                           for b in range(nb)])
+
+
+def _long_prefill_check(ex, w, sel_heads, n_uniform, n_strat, seed):
+    """The checks of a long single-sequence prefill in the bench's wave configuration:
+    - all block means;
+    - the full selection of every head in ``sel_heads`` against oracle.select_blocks;
+    - n_uniform + n_strat sampled rows of every head (plus every near-tie row found): their
+      selections against the oracle's and their outputs against oracle.attend_rows over the
+      GPU's selection;
+    - the oracle-feed mode: the oracle's selections (whole heads where computed, the sampled
+      rows elsewhere) fed back, the sampled rows' outputs compared with no exception."""
     q, k, v, cu_t = gpu_inputs(w)
     cu = np.asarray(w.cu_seqlens)
     chunk, topk, hq, hkv = w.chunk_size, w.topk, w.num_q_heads, w.num_kv_heads
     group = hq // hkv
-    n_rows = int(os.environ.get("MOBA_1M_SAMPLED_ROWS_PER_HEAD", "24"))
-    out, lse, sel = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True)
+    T = w.total_tokens
+    out, lse, sel = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True, max_seqlen=w.max_seqlen)
     nb = moba.num_blocks(w.seqlens, chunk)
     means = moba.meanpool(k, cu_t, chunk, num_blocks_out=nb)
     torch.cuda.synchronize()
     assert moba.attn_fwd.last_info["waves"] >= 1
-    k_np, v_np = PT.host(k, np.float32), PT.host(v, np.float32)
-    # means, per block through the oracle (blocks are independent)
-    om = np.concatenate([oracle.block_means(k_np[b * chunk:(b + 1) * chunk], [0, chunk], chunk)
-                         for b in range(nb)])
-    PT.check_means(PT.host(means), k_np, cu, chunk, om)
-    gsel = PT.host(sel, np.int64)
-    heads = [0, 9, 18, 27]
-    for h in heads:
-        qh = PT.host(q[:, h:h + 1], np.float32)
-        osel_h = oracle.select_blocks(qh, om[:, h // group:h // group + 1], cu, chunk, topk)
-        full_sel_check(gsel[h:h + 1], osel_h, qh, om[:, h // group:h // group + 1], cu, chunk,
-                       topk, 1)
-    rows = PT.sample_rows(cu, chunk, hq, topk, n_rows * hq * 3 // 4, n_rows * hq // 4, seed=41)
-    q_rows = {}
-    for t, h in rows:
-        if t not in q_rows:
-            q_rows[t] = PT.host(q[t], np.float32)
-    ref_sel = np.stack([
-        oracle.select_blocks_rows(_QView(q_rows), om, cu, chunk, topk, [(t, h)])[0] for t, h in rows])
-    g_rows = np.stack([gsel[h, t] for t, h in rows])
-    ties = PT.check_selection(g_rows, ref_sel, rows, _QView(q_rows), om, cu, chunk, topk, group)
-    ref_o, ref_l = oracle.attend_rows(_QView(q_rows), k_np, v_np, cu, chunk, ref_sel, rows)
-    out_np = {t: PT.host(out[t], np.float32) for t, _ in rows}
-    lse_rows = np.array([float(lse[h, t]) for t, h in rows])
-    g_o = np.stack([out_np[t][h] for t, h in rows])
-    PT.check_out(g_o, lse_rows, ref_o, ref_l, skip=sorted(ties))
+    k16, v16 = PT.bf16_bits(k), PT.bf16_bits(v)
+    om = _block_means_by_block(k16, w)
+    PT.check_means(PT.host(means), _Bf16Rows(k16), cu, chunk, om)
 
-    # fed selection defined here: own block, the previous block, block 0 and a
-    # pseudo-random far block, all rows; checked on the sampled rows
-    T = q.shape[0]
-    tt = torch.arange(T, device="cuda", dtype=torch.int64)
-    c = tt // chunk
-    fed = torch.full((hq, T, topk), -1, dtype=torch.int32, device="cuda")
-    hh = torch.arange(hq, device="cuda", dtype=torch.int64)[:, None]
-    far = (c[None, :] * 7 + hh * 13) % torch.clamp(c[None, :], min=1)
-    cand = torch.stack([torch.zeros_like(far), far, (c - 1).expand_as(far), c.expand_as(far)], dim=2)
-    fed[:, :, :4] = cand.to(torch.int32)
-    out3, lse3 = moba.attn_fwd(q, k, v, cu_t, chunk, topk, sel=fed)
-    fed_rows = PT.host(fed[:, :, :4], np.int64)
-    ref_sel3 = []
-    for t, h in rows:
-        cc = t // chunk
-        ref_sel3.append(sorted({int(j) for j in fed_rows[h, t] if 0 <= j <= cc}))
-    ref_sel3 = np.array([r + [-1] * (topk - len(r)) for r in ref_sel3])
-    ref_o3, ref_l3 = oracle.attend_rows(_QView(q_rows), k_np, v_np, cu, chunk, ref_sel3, rows)
-    g_o3 = np.stack([PT.host(out3[t, h], np.float32) for t, h in rows])
-    g_l3 = np.array([float(lse3[h, t]) for t, h in rows])
-    PT.check_out(g_o3, g_l3, ref_o3, ref_l3)
+    # whole heads
+    full = OP.select_and_compare_heads(
+        ex, lambda h: PT.bf16_bits(q[:, h]), om, lambda h: sel[h].cpu().numpy().astype(np.int16),
+        cu, chunk, topk, group, sel_heads)
+    ties = {(int(t), h) for h, (_, tt) in full.items() for t in tt}
+    assert len(ties) < 1e-3 * T * len(sel_heads)
+
+    # sampled rows of every head, plus the near-tie rows
+    rows = sorted(set(PT.sample_rows_per_head(cu, chunk, hq, topk, n_uniform, n_strat, seed)) | ties)
+    ts_t = torch.tensor([t for t, _ in rows], device="cuda")
+    hs_t = torch.tensor([h for _, h in rows], device="cuda")
+    ts, hs = ts_t.cpu().numpy(), hs_t.cpu().numpy()
+    q_rows = PT.bf16_bits(q[ts_t, hs_t])
+    g_rows = sel[hs_t, ts_t].cpu().numpy().astype(np.int64)
+    o_rows = np.zeros_like(g_rows)
+    in_full = np.isin(hs, list(sel_heads))
+    for h, (osel_h, _) in full.items():
+        m = hs == h
+        o_rows[m] = osel_h[ts[m]]
+    rest = np.nonzero(~in_full)[0]
+    if len(rest):
+        o_rows[rest] = OP.select_rows_par(ex, [rows[i] for i in rest], q_rows[rest], om, cu, chunk, topk, group)
+        ties_rest = PT.check_selection(g_rows[rest], o_rows[rest], [rows[i] for i in rest],
+                                       _RowQ(rows, q_rows), om, cu, chunk, topk, group)
+        assert len(ties_rest) < max(3, 1e-2 * len(rest))
+
+    ref_g = OP.attend_rows_par(ex, rows, q_rows, k16, v16, cu, chunk, g_rows, group)
+    PT.check_out(PT.host(out[ts_t, hs_t]), PT.host(lse[hs_t, ts_t]), *ref_g)
+
+    # oracle-feed mode (the output buffers are reused)
+    fed = sel.clone()
+    for h, (osel_h, _) in full.items():
+        fed[h] = torch.from_numpy(osel_h.astype(np.int32)).cuda()
+    fed[hs_t, ts_t] = torch.from_numpy(o_rows.astype(np.int32)).cuda()
+    moba.attn_fwd(q, k, v, cu_t, chunk, topk, sel=fed, out=out, lse=lse)
+    torch.cuda.synchronize()
+    diff = np.nonzero((g_rows != o_rows).any(axis=1))[0]
+    ref_o, ref_l = ref_g[0].copy(), ref_g[1].copy()
+    if len(diff):
+        o2, l2 = OP.attend_rows_par(ex, [rows[i] for i in diff], q_rows[diff], k16, v16, cu, chunk,
+                                    o_rows[diff], group)
+        ref_o[diff], ref_l[diff] = o2, l2
+    PT.check_out(PT.host(out[ts_t, hs_t]), PT.host(lse[hs_t, ts_t]), ref_o, ref_l)
 
 
-class _QView:
-    """Row-indexable stand-in for q [T, Hq, d] holding only the sampled tokens."""
+class _RowQ:
+    """q[t, h] of the sampled rows only (parity.check_selection reads the rows it checks)."""
 
-    def __init__(self, rows_by_t):
-        self.rows = rows_by_t
-        first = next(iter(rows_by_t.values()))
-        self.shape = (None, first.shape[0], first.shape[1])
+    def __init__(self, rows, q_rows16):
+        self.idx = {r: i for i, r in enumerate(rows)}
+        self.q = q_rows16
 
-    def __getitem__(self, idx):
-        t, h = idx
-        return self.rows[int(t)][h]
+    def __getitem__(self, th):
+        return PT.from_bits(self.q[self.idx[(int(th[0]), int(th[1]))]])
+
+
+def test_prefill_1m(ex):
+    """1,048,576 tokens, 32 q / 8 kv heads, chunk 4096, top-12: all block means, the full
+    selection of all 32 heads, 4096 sampled rows per head (3584 uniform + 512 stratified),
+    the oracle-feed mode with the oracle's whole selection."""
+    w = W.WORKLOADS["prefill_1m"]
+    _long_prefill_check(ex, w, list(range(w.num_q_heads)), 3584, 512, seed=41)
+
+
+def test_prefill_2m_length_sweep(ex):
+    """Length sweep, 2,097,152 tokens in 256 blocks of 8192, top-12: full selections of four
+    heads (one per two KV heads), 192 sampled rows per head, the oracle-feed mode."""
+    w = W.ALL_WORKLOADS["prefill_2m"]
+    _long_prefill_check(ex, w, [0, 9, 18, 27], 160, 32, seed=42)
+
+
+def test_prefill_10m_length_sweep(ex):
+    """Length sweep, 10,485,760 tokens in 256 blocks of 40,960 (the 8 q / 2 kv head-group
+    share), top-12: the full selection of one head, 64 sampled rows per head, the
+    oracle-feed mode."""
+    w = W.ALL_WORKLOADS["prefill_10m"]
+    _long_prefill_check(ex, w, [5], 48, 16, seed=43)
 
 
 def test_cuda_core_gate_above_257_blocks():
-    """More than 257 blocks in one call select the CUDA-core gate (csrc/gate.cu) instead of the
-    tensor-core one: its selections against the oracle's, outside the near-tie band."""
-    w = W.custom("gate_267_blocks", [20000, 14000], 2, 1, 64, 128, 4, "k_offsets", 25)
-    q, k, _, cu_t = gpu_inputs(w)
+    """A sequence of more than 257 blocks selects the CUDA-core gate (csrc/gate.cu) instead of
+    the tensor-core one: its selections against the oracle's (valid near ties allowed)."""
+    w = W.custom("gate_313_blocks", [40000, 3000], 2, 1, 64, 128, 4, "k_offsets", 25)
+    q, k, v, cu_t = gpu_inputs(w)
     cu = np.asarray(w.cu_seqlens)
     chunk, topk, group = w.chunk_size, w.topk, w.num_q_heads // w.num_kv_heads
-    p = moba.make_params(len(w.seqlens), w.total_tokens, w.num_q_heads, w.num_kv_heads,
-                         w.head_dim, chunk, topk)
-    assert moba.num_blocks_bound(p) > 257
     means = moba.meanpool(k, cu_t, chunk)
-    sel = moba.gate_topk(q, means, cu_t, chunk, topk)
+    sel = moba.gate_topk(q, means, cu_t, chunk, topk, max_seqlen=w.max_seqlen)
+    _, _, sel2 = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True, max_seqlen=w.max_seqlen)
+    assert moba.attn_fwd.last_info["gate_path"] == moba.GATE_PATH_CUDA_CORES
     torch.cuda.synchronize()
+    assert torch.equal(sel, sel2)
     q_np, k_np = PT.host(q), PT.host(k)
     om = oracle.block_means(k_np, cu, chunk)
     osel = oracle.select_blocks(q_np, om, cu, chunk, topk)
     full_sel_check(PT.host(sel, np.int64), osel, q_np, om, cu, chunk, topk, group)
+
+
+def test_packed_batch_uses_the_tensor_core_gate():
+    """A packed batch of 40 sequences of 2048 tokens (640 blocks in all, 16 per sequence):
+    with max_seqlen the tensor-core gate runs (sized for 16 blocks); without it the batch-wide
+    block bound sends the call to the CUDA-core gate.  Both selections match the oracle's,
+    and the outputs match on all rows."""
+    w = W.custom("packed_40x2k", [2048] * 40, 4, 2, 128, 128, 3, "k_offsets", 26)
+    q, k, v, cu_t = gpu_inputs(w)
+    cu = np.asarray(w.cu_seqlens)
+    chunk, topk, group = w.chunk_size, w.topk, w.num_q_heads // w.num_kv_heads
+    out, lse, sel = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True, max_seqlen=2048)
+    assert moba.attn_fwd.last_info["gate_path"] == moba.GATE_PATH_TENSOR_CORES
+    _, _, sel_cc = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True)
+    assert moba.attn_fwd.last_info["gate_path"] == moba.GATE_PATH_CUDA_CORES
+    torch.cuda.synchronize()
+    q_np, k_np, v_np = PT.host(q), PT.host(k), PT.host(v)
+    ref = oracle.moba_forward(q_np, k_np, v_np, cu, chunk, topk)
+    gsel = PT.host(sel, np.int64)
+    ties = full_sel_check(gsel, ref["sel"], q_np, ref["means"], cu, chunk, topk, group)
+    full_sel_check(PT.host(sel_cc, np.int64), ref["sel"], q_np, ref["means"], cu, chunk, topk, group)
+    ref_o, ref_l = with_tie_rows(ref["out"], ref["lse"], ties, gsel, q_np, k_np, v_np, cu, chunk)
+    check_all_rows(out, lse, ref_o, ref_l)
+
+
+def test_max_seqlen_too_small_is_reported_not_faulted():
+    """A max_seqlen shorter than a real sequence: no out-of-bounds access, the status word
+    reads MOBA_ERR_INVALID_ARG, and the next call with the right bound is correct again."""
+    w = W.custom("short_promise", [3000, 500], 2, 1, 64, 128, 3, "k_offsets", 27)
+    q, k, v, cu_t = gpu_inputs(w)
+    p = moba.make_params(len(w.seqlens), w.total_tokens, 2, 1, 64, 128, 3, max_seqlen=1750)
+    ws = torch.empty(moba.workspace_size(p), dtype=torch.uint8, device="cuda")
+    moba.attn_fwd(q, k, v, cu_t, 128, 3, workspace=ws, max_seqlen=1750)
+    with pytest.raises(moba.MobaError) as e:
+        moba.device_status(p, ws)
+    assert e.value.status == moba.ERR_INVALID_ARG
+    out, lse = moba.attn_fwd(q, k, v, cu_t, 128, 3, workspace=ws, max_seqlen=3000)
+    moba.device_status(p, ws)
+    ref_o, ref_l = moba.attn_fwd(q, k, v, cu_t, 128, 3)
+    assert torch.equal(out, ref_o) and torch.equal(lse, ref_l)

@@ -1,0 +1,50 @@
+"""CPU checks of the GPU parity helpers themselves (tests/parity.py): the selection rule that
+decides which GPU rows count as valid near-tie alternatives must reject every other kind of
+difference."""
+
+import numpy as np
+
+import parity as PT
+
+
+def test_near_tie_rule_rejects_planted_mistakes():
+    """The near-tie rule of the selection check, on hand-made rows: a swap inside the band
+    passes; a swap outside it, a duplicated block, a missing own block, an unsorted row, a
+    future block and bad padding fail."""
+    scores = np.array([5.0, 1.0, 3.0, 2.9999, 0.5])   # blocks 0..4 of a row with c = 5
+    ref = [0, 2, 5]                                    # topk 3: the best 2 routed + own block
+    assert PT.near_tie_alternative([0, 3, 5], ref, scores, 5, 3)   # 3 for 2: within 1e-3
+    for bad in ([0, 1, 5],        # 1 for 2: far outside the band
+                [2, 2, 5],        # duplicate
+                [0, 2, 4],        # own block missing
+                [2, 0, 5],        # not ascending
+                [0, 6, 5]):       # a future block
+        assert not PT.near_tie_alternative(bad, ref, scores, 5, 3), bad
+    # c = 2 with topk 4: both past blocks routed, then the own block, then -1
+    sc2 = np.array([1.0, 2.0])
+    assert PT.near_tie_alternative([0, 1, 2, -1], [0, 1, 2, -1], sc2, 2, 4)
+    assert not PT.near_tie_alternative([0, 1, 2, 3], [0, 1, 2, -1], sc2, 2, 4)
+
+
+def test_well_formed_rows():
+    assert PT.well_formed([1, 3, 4], 4, 3)
+    assert PT.well_formed([0, -1, -1], 0, 3)           # block 0: own block only
+    assert not PT.well_formed([0, 4, -1, -1], 4, 4)    # too few routed blocks for c = 4
+    assert not PT.well_formed([1, 3, 4, 4], 4, 3)      # own block repeated
+
+
+def test_check_selection_counts_ties_and_fails_otherwise():
+    """check_selection on two rows of a tiny problem: an equal-score swap is a tie; a swap of
+    a clearly better block fails."""
+    import pytest
+    q = np.zeros((3000, 1, 2))
+    q[:, 0, 0] = 1.0
+    means = np.zeros((4, 1, 2))
+    means[:, 0, 0] = [1.0, 1.0, 0.5, 0.0]              # blocks 0 and 1 tie, 2 is worse
+    cu = [0, 3000]
+    rows = [(2500, 0)]                                  # c = 3 with chunk 800 (blocks 0, 1, 2 past)
+    ref = np.array([[0, 3, -1]])                        # topk 3: one routed block + own
+    ties = PT.check_selection(np.array([[1, 3, -1]]), ref, rows, q, means, cu, 800, 2, 1)
+    assert ties == {0}
+    with pytest.raises(AssertionError):
+        PT.check_selection(np.array([[2, 3, -1]]), ref, rows, q, means, cu, 800, 2, 1)
