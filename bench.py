@@ -148,62 +148,109 @@ def job_value(tokens_per_rank, world, ms_max):
     return world * tokens_per_rank / (ms_max * 1e-3)
 
 
-def cpu_oracle_sample(w, budget_s, seed=0, inputs=None):
-    """Times the float64 oracle on sampled query rows of workload w (bounded CPU work).
+def _cpu_facts():
+    """Host cores this process may use and the CPU model (for the baseline records)."""
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_count": os.cpu_count(), "cores_usable": cores, "cpu_model": model}
 
-    Per sampled row (t, h): gate selection (against the block means) and attention over its
-    selected blocks.  The block means of the whole input are computed once and charged to
-    the sample in proportion (rows sampled / all rows).  Returns (tokens/s, detail).
-    """
+
+def cpu_oracle_baseline(w, budget_s, seed=0, inputs=None, dense=False):
+    """Times the float64 oracle, as it stands, on the host cores, on a bounded sample of
+    workload w, and extrapolates the whole forward's time on those cores.
+
+    Three measured parts, on a spawn pool of one process per usable core (the oracle's own
+    functions on independent pieces, tests/oracle_pool.py):
+      * the block means of the whole input (one process, measured in full);
+      * the gate selection of one whole query head (oracle.select_blocks), times Hq;
+      * sampled (token, head) rows' gate selection and attention (oracle.select_blocks_rows and
+        oracle.attend_rows), for about budget_s of wall time, scaled to all T * Hq rows.
+    The estimate is means + (gate + rows CPU-seconds) / cores.  With dense=True the dense
+    causal fp64 attention of the same shape (the oracle with every block selected) is timed on
+    one head and reported beside it.  Returns (tokens/s, detail)."""
     import numpy as np
     import torch
 
     import oracle
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import oracle_pool as OP
+    import parity as PT
     from block_sparse_long_meanpool_b200 import workloads as W
 
     x = inputs if inputs is not None else W.make_inputs(w, device="cpu")
-    k = x["k"].float().numpy()
-    v = x["v"].float().numpy()
-    qt = x["q"]
+    bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    q16, k16, v16 = bits(x["q"]), bits(x["k"]), bits(x["v"])
     cu = np.asarray(w.cu_seqlens)
-    T, hq = w.total_tokens, w.num_q_heads
+    T, hq, hkv = w.total_tokens, w.num_q_heads, w.num_kv_heads
+    group = hq // hkv
+    chunk, topk = w.chunk_size, w.topk
+    facts = _cpu_facts()
+    workers = OP.n_workers()
     t0 = time.perf_counter()
-    means = oracle.block_means(k, cu, w.chunk_size)
+    means = np.concatenate([oracle.block_means(PT.from_bits(k16[cu[i]:cu[i + 1]]), [0, cu[i + 1] - cu[i]], chunk)
+                            for i in range(len(cu) - 1)])
     t_means = time.perf_counter() - t0
     rng = np.random.default_rng(seed)
-
-    class QRows:
-        shape = (T, hq, w.head_dim)
-
-        def __getitem__(self, idx):
-            t, h = idx
-            return qt[int(t), int(h)].float().numpy()
-
-    qv = QRows()
-    done, t_rows = 0, 0.0
-    while t_rows < budget_s:
-        rows = [(int(rng.integers(0, T)), int(rng.integers(0, hq))) for _ in range(8)]
+    with OP.pool() as ex:
+        # warm the workers up (process start, imports) outside the timed parts
+        list(ex.map(int, range(workers)))
+        h = int(rng.integers(0, hq))
         a = time.perf_counter()
-        sel = oracle.select_blocks_rows(qv, means, cu, w.chunk_size, w.topk, rows)
-        oracle.attend_rows(qv, k, v, cu, w.chunk_size, sel, rows)
-        t_rows += time.perf_counter() - a
-        done += len(rows)
-    frac = done / float(T * hq)
-    seconds = t_rows + t_means * frac
-    tokens = done / hq
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
-    except Exception:
-        threads = 1
-    del torch
-    detail = {"rows": done, "row_seconds": t_rows, "means_seconds_full": t_means,
-              "cores": threads,
-              "sample": (f"{done} uniformly sampled (token, head) rows of {w.name} "
-                         f"({T} tokens x {hq} heads): per-row gate + top-k + attention, plus "
-                         f"the full-input block means charged at {frac:.2e} of their "
-                         f"{t_means:.1f} s")}
-    return tokens / seconds, detail
+        ex.submit(OP._select_head, np.ascontiguousarray(q16[:, h]),
+                  np.ascontiguousarray(means[:, h // group]), cu, chunk, topk).result()
+        t_gate_head = time.perf_counter() - a
+        done, cpu_rows = 0, 0.0
+        wall0 = time.perf_counter()
+        while time.perf_counter() - wall0 < budget_s:
+            rows = sorted({(int(rng.integers(0, T)), int(rng.integers(0, hq))) for _ in range(4 * workers)})
+            ts = np.array([t for t, _ in rows])
+            hs = np.array([hh for _, hh in rows])
+            a = time.perf_counter()
+            sel = OP.select_rows_par(ex, rows, q16[ts, hs], means, cu, chunk, topk, group)
+            OP.attend_rows_par(ex, rows, q16[ts, hs], k16, v16, cu, chunk, sel, group)
+            cpu_rows += (time.perf_counter() - a) * workers
+            done += len(rows)
+        dense_s = None
+        if dense:
+            # every block selected: dense causal attention, one query head
+            nbs = [(cu[i + 1] - cu[i] + chunk - 1) // chunk for i in range(len(cu) - 1)]
+            all_sel = np.full((1, T, max(nbs)), -1, dtype=np.int64)
+            for i in range(len(cu) - 1):
+                for t in range(cu[i], cu[i + 1]):
+                    c = (t - cu[i]) // chunk
+                    all_sel[0, t, :c + 1] = np.arange(c + 1)
+            a = time.perf_counter()
+            ex.submit(OP._dense_head, np.ascontiguousarray(q16[:, 0]), np.ascontiguousarray(k16[:, 0]),
+                      np.ascontiguousarray(v16[:, 0]), cu, chunk, all_sel[0], None).result()
+            dense_s = (time.perf_counter() - a) * hq
+    rows_all = float(T * hq)
+    cpu_total = t_gate_head * hq + cpu_rows * rows_all / max(done, 1)
+    seconds = t_means + cpu_total / workers
+    detail = dict(facts)
+    detail.update({
+        "cores": workers, "rows": done, "row_cpu_seconds": cpu_rows, "means_seconds": t_means,
+        "gate_seconds_per_head": t_gate_head,
+        "extrapolated": True,
+        "sample": (f"{w.name} ({T} tokens x {hq} heads) on {workers} host processes: block means of the "
+                   f"whole input ({t_means:.1f} s), the full gate selection of one head ({t_gate_head:.1f} s, "
+                   f"x {hq} heads), {done} uniformly sampled rows' gate + attention ({cpu_rows:.0f} "
+                   f"CPU-s), extrapolated to all rows as means + CPU-seconds / processes")})
+    if dense_s is not None:
+        detail["dense_causal_fp64_tokens_per_s"] = T / (dense_s / workers)
+        detail["dense_causal_fp64_note"] = ("the oracle with every block selected (dense causal attention), "
+                                            "one head timed, x heads / processes")
+    return T / seconds, detail
 
 
 def run_reference(args, w, world, rank):
@@ -225,7 +272,7 @@ def run_reference(args, w, world, rank):
     per_step = float(os.environ.get("MOBA_REF_STEP_SECONDS", "8"))
     vals, details = [], []
     for i in range(args.warmup + args.steps):
-        val, det = cpu_oracle_sample(w, per_step, seed=100 + i, inputs=inputs)
+        val, det = cpu_oracle_baseline(w, per_step, seed=100 + i, inputs=inputs)
         if i >= args.warmup:
             vals.append(val)
             details.append(det)
@@ -240,11 +287,221 @@ def run_reference(args, w, world, rank):
                    "global_batch": len(w.seqlens) * args.gpus, "seq_len": w.max_seqlen,
                    "parallelism": f"dp{args.gpus}", "l2": "n/a (CPU)"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": details[-1]["cores"],
-                         "kind": "oracle", "sample": details[-1]["sample"]},
+                         "kind": "oracle", "sample": details[-1]["sample"],
+                         "cpu_model": details[-1]["cpu_model"], "cpu_count": details[-1]["cpu_count"],
+                         "extrapolated": details[-1]["extrapolated"]},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def _time_forward(moba, w, x, steps, warmup, gate="mean", budget=None, wave_tokens=None,
+                  max_seqlen=None):
+    """CUDA-event timing of the whole forward (one moba_attn_fwd per step, inputs resident) with
+    the library's per-stage events.  Returns a dict with ms per step, the stage split, the wave
+    plan, launches and gate path, and the output buffers."""
+    import torch
+
+    q, k, v, cu = x["q"], x["k"], x["v"], x["cu_seqlens"]
+    T, hq, d = q.shape
+    chunk, topk = w.chunk_size, w.topk
+    dev = q.device
+    out = torch.empty((T, hq, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((hq, T), dtype=torch.float32, device=dev)
+    # first call fixes the wave size and the workspace
+    moba.attn_fwd(q, k, v, cu, chunk, topk, out=out, lse=lse, workspace_budget=budget,
+                  wave_tokens=wave_tokens, gate=gate, max_seqlen=max_seqlen)
+    info0 = dict(moba.attn_fwd.last_info)
+    wt = info0["wave_tokens"]
+    ws = torch.empty(info0["workspace_bytes"], dtype=torch.uint8, device=dev)
+    waves = info0["waves"]
+    n_ev = moba.EV_WAVE0 + 4 * waves
+
+    def step(events=None):
+        moba.attn_fwd(q, k, v, cu, chunk, topk, out=out, lse=lse, workspace=ws, wave_tokens=wt,
+                      events=events, gate=gate, max_seqlen=max_seqlen)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(steps)]
+    return {"step": step, "events": events, "waves": waves, "wave_tokens": wt or T, "ws": ws,
+            "out": out, "lse": lse, "info": info0}
+
+
+def _stage_split(moba, events, waves, steps):
+    def span(i, a, b):
+        return events[i][a].elapsed_time(events[i][b])
+    st = {"meanpool": 0.0, "gate": 0.0, "route": 0.0, "attention": 0.0, "merge": 0.0}
+    for i in range(steps):
+        st["meanpool"] += span(i, moba.EV_BEGIN, moba.EV_MEANS_DONE)
+        st["gate"] += span(i, moba.EV_MEANS_DONE, moba.EV_GATE_DONE)
+        for wv in range(waves):
+            b = moba.EV_WAVE0 + 4 * wv
+            st["route"] += span(i, b, b + 1)
+            st["attention"] += span(i, b + 1, b + 2)
+            st["merge"] += span(i, b + 2, b + 3)
+    return {kk: vv / steps for kk, vv in st.items()}
+
+
+def _run_timed(fwd, steps):
+    """Runs the prepared forward `steps` times between two events; returns ms per step."""
+    import torch
+
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(steps):
+        fwd["step"](fwd["events"][i])
+    end.record()
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / steps
+
+
+def _sub_forward(moba, W, w, dev, steps, warmup, peaks, gate="mean", max_seqlen=None, seed=None):
+    """A forward sub-record on workload w (inputs larger than L2): ms per step, the stage
+    split, attention TF/s against the burst peak (steps well under a second) and the gate's
+    and merge's HBM rates."""
+    import torch
+
+    x = W.make_inputs(w, device=dev, seed=seed)
+    fwd = _time_forward(moba, w, x, steps, warmup, gate=gate, max_seqlen=max_seqlen)
+    ms = _run_timed(fwd, steps)
+    st = _stage_split(moba, fwd["events"], fwd["waves"], steps)
+    f_sel = W.selected_block_flops(w.seqlens, w.num_q_heads, w.head_dim, w.chunk_size, w.topk)
+    peak = peaks["bf16_tflops_sustained"] if ms > 200.0 else peaks["bf16_tflops"]
+    att = f_sel / (st["attention"] * 1e-3) / 1e12
+    rec = {"workload": w.name, "gate": gate, "max_seqlen": max_seqlen, "steps": steps,
+           "ms_per_step": ms, "tokens_per_s": w.total_tokens / (ms * 1e-3), "stage_ms": st,
+           "attention_tflops": att, "attention_frac": att / peak,
+           "peak_kind": "bf16 sustained" if ms > 200.0 else "bf16 burst",
+           "gate_path": {1: "tensor cores", 2: "cuda cores"}.get(fwd["info"]["gate_path"], "none"),
+           "hbm_stages": _hbm_stage_rates(w, st, peaks, gate)}
+    del x, fwd
+    torch.cuda.empty_cache()
+    return rec
+
+
+def _sub_backward(moba, W, w, x, dev, peaks, steps=3, warmup=3):
+    """A backward sub-record on workload w: the forward runs once (outside the timing) for
+    out, lse and its selection; then moba_attn_bwd is timed.  TF/s counts the algorithmic
+    backward work as 2.5 x the forward's selected-block FLOPs (QK^T, dP, dV, dK, dQ); the
+    kernels execute 3.5 x (S and dP are recomputed for dQ)."""
+    import torch
+
+    q, k, v, cu = x["q"], x["k"], x["v"], x["cu_seqlens"]
+    out, lse, sel = moba.attn_fwd(q, k, v, cu, w.chunk_size, w.topk, return_sel=True,
+                                  max_seqlen=w.max_seqlen)
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed + 77)
+    d_out = torch.randn(out.shape, generator=g, device=dev).to(torch.bfloat16)
+    d_lse = torch.randn(lse.shape, generator=g, device=dev)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    moba.attn_bwd(q, k, v, out, lse, d_out, cu, w.chunk_size, w.topk, sel, d_lse=d_lse,
+                  dq=dq, dk=dk, dv=dv)
+    wsb = torch.empty(moba.attn_bwd.last_info["workspace_bytes"], dtype=torch.uint8, device=dev)
+
+    def step():
+        moba.attn_bwd(q, k, v, out, lse, d_out, cu, w.chunk_size, w.topk, sel, d_lse=d_lse,
+                      workspace=wsb, dq=dq, dk=dk, dv=dv)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    f_sel = W.selected_block_flops(w.seqlens, w.num_q_heads, w.head_dim, w.chunk_size, w.topk)
+    peak = peaks["bf16_tflops_sustained"] if ms > 200.0 else peaks["bf16_tflops"]
+    alg = 2.5 * f_sel / (ms * 1e-3) / 1e12
+    rec = {"workload": w.name, "steps": steps, "warmup": warmup, "ms_per_step": ms,
+           "tokens_per_s": w.total_tokens / (ms * 1e-3),
+           "algorithmic_tflops": alg, "frac": alg / peak,
+           "executed_tflops": 3.5 * f_sel / (ms * 1e-3) / 1e12,
+           "peak_kind": "bf16 sustained" if ms > 200.0 else "bf16 burst",
+           "note": "dq, dk, dv for the forward's selection; algorithmic work 2.5 x the forward's "
+                   "selected-block FLOPs, executed 3.5 x"}
+    del out, lse, sel, d_out, d_lse, dq, dk, dv, wsb
+    torch.cuda.empty_cache()
+    return rec
+
+
+def _e2e_pipelined(moba, w, x, fwd, steps, world):
+    """End to end through the public API with pinned host buffers: every step copies its inputs
+    host -> device, runs moba_attn_fwd and reads out and lse back.  Steps are pipelined over two
+    device buffer sets and two streams for the copies: step i+1's upload and step i-1's
+    download run while step i computes.  Every copy of every timed step is inside the timed
+    region (events on the compute stream after waiting for the copy streams)."""
+    import torch
+
+    q, k, v, cu = x["q"], x["k"], x["v"], x["cu_seqlens"]
+    out, lse, ws = fwd["out"], fwd["lse"], fwd["ws"]
+    chunk, topk, wt = w.chunk_size, w.topk, fwd["info"]["wave_tokens"]
+    host = {n: t.cpu().pin_memory() for n, t in (("q", q), ("k", k), ("v", v), ("cu", cu))}
+    outh = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    lseh = [torch.empty(lse.shape, dtype=lse.dtype).pin_memory() for _ in range(2)]
+    dev_in = [{"q": q, "k": k, "v": v, "cu": cu},
+              {n: torch.empty_like(t) for n, t in (("q", q), ("k", k), ("v", v), ("cu", cu))}]
+    dev_out = [(out, lse), (torch.empty_like(out), torch.empty_like(lse))]
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
+    main = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    in_ready = [ev(), ev()]
+    computed = [ev(), ev()]
+    out_read = [ev(), ev()]
+
+    def run(n):
+        for i in range(n):
+            bsel = i % 2
+            s_in.wait_event(computed[bsel]) if i >= 2 else None
+            with torch.cuda.stream(s_in):
+                for name in ("q", "k", "v", "cu"):
+                    dev_in[bsel][name].copy_(host[name], non_blocking=True)
+                in_ready[bsel].record(s_in)
+            main.wait_event(in_ready[bsel])
+            if i >= 2:
+                main.wait_event(out_read[bsel])
+            di = dev_in[bsel]
+            o, l = dev_out[bsel]
+            moba.attn_fwd(di["q"], di["k"], di["v"], di["cu"], chunk, topk, out=o, lse=l,
+                          workspace=ws, wave_tokens=wt)
+            computed[bsel].record(main)
+            s_out.wait_event(computed[bsel])
+            with torch.cuda.stream(s_out):
+                outh[bsel].copy_(o, non_blocking=True)
+                lseh[bsel].copy_(l, non_blocking=True)
+                out_read[bsel].record(s_out)
+        main.wait_event(out_read[(n - 1) % 2])
+        if n >= 2:
+            main.wait_event(out_read[(n - 2) % 2])
+
+    run(2)
+    torch.cuda.synchronize()
+    barrier(world)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(main)
+    run(steps)
+    b.record(main)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / steps, world)
+    del dev_in[1], dev_out[1]
+    torch.cuda.empty_cache()
+    return {"value": job_value(w.total_tokens, world, e2e_ms), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+            "steps": steps,
+            "pipelining": "two device buffer sets; uploads and downloads on their own streams "
+                          "overlap the neighbouring steps' compute"}
 
 
 def run_ours(args, w, world, rank, local):
@@ -257,68 +514,30 @@ def run_ours(args, w, world, rank, local):
     if rank == 0:
         _build.build()
     barrier(world)
-    lib = moba.load_library()
-    del lib
+    moba.load_library()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     x = W.make_inputs(w, device=dev, seed=rank_seed(w, rank))
-    q, k, v, cu = x["q"], x["k"], x["v"], x["cu_seqlens"]
+    q, k = x["q"], x["k"]
     T, hq, d = q.shape
     hkv = k.shape[1]
     chunk, topk = w.chunk_size, w.topk
-    budget = None
-    if args.workspace_gb:
-        budget = int(args.workspace_gb * (1 << 30))
-    out = torch.empty((T, hq, d), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((hq, T), dtype=torch.float32, device=dev)
-    # first call fixes the wave size and the workspace
-    moba.attn_fwd(q, k, v, cu, chunk, topk, out=out, lse=lse, workspace_budget=budget,
-                  wave_tokens=args.wave_tokens)
-    info0 = dict(moba.attn_fwd.last_info)
-    wave_tokens = info0["wave_tokens"]
-    ws = torch.empty(info0["workspace_bytes"], dtype=torch.uint8, device=dev)
-    waves = info0["waves"]
-    n_ev = moba.EV_WAVE0 + 4 * waves
-
-    def step(events=None):
-        moba.attn_fwd(q, k, v, cu, chunk, topk, out=out, lse=lse, workspace=ws,
-                      wave_tokens=wave_tokens, events=events)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    budget = int(args.workspace_gb * (1 << 30)) if args.workspace_gb else None
+    max_seqlen = w.max_seqlen
+    fwd = _time_forward(moba, w, x, args.steps, args.warmup, gate=args.gate, budget=budget,
+                        wave_tokens=args.wave_tokens, max_seqlen=max_seqlen)
+    waves, wave_tokens = fwd["waves"], fwd["wave_tokens"]
     sampler = ClockSampler(_gpu_id(dev))
     barrier(world)
     torch.cuda.synchronize()
     sampler.start()
     time.sleep(0.3)
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    start.record()
-    for i in range(args.steps):
-        step(events[i])
-    end.record()
-    torch.cuda.synchronize()
+    ms_local = _run_timed(fwd, args.steps)
     clocks = sampler.stop()
     barrier(world)
-    ms_local = start.elapsed_time(end) / args.steps
     ms = max_over_ranks(ms_local, world)
     launches = moba.attn_fwd.last_info["launches"]
-
-    # per-stage device times (ms per step, mean over steps)
-    def span(i, a, b):
-        return events[i][a].elapsed_time(events[i][b])
-    st = {"meanpool": 0.0, "gate": 0.0, "route": 0.0, "attention": 0.0, "merge": 0.0}
-    for i in range(args.steps):
-        st["meanpool"] += span(i, moba.EV_BEGIN, moba.EV_MEANS_DONE)
-        st["gate"] += span(i, moba.EV_MEANS_DONE, moba.EV_GATE_DONE)
-        for wv in range(waves):
-            b = moba.EV_WAVE0 + 4 * wv
-            st["route"] += span(i, b, b + 1)
-            st["attention"] += span(i, b + 1, b + 2)
-            st["merge"] += span(i, b + 2, b + 3)
-    st = {kk: vv / args.steps for kk, vv in st.items()}
+    st = _stage_split(moba, fwd["events"], waves, args.steps)
 
     peaks = read_peaks()
     f_sel = W.selected_block_flops(w.seqlens, hq, d, chunk, topk)
@@ -329,49 +548,39 @@ def run_ours(args, w, world, rank, local):
     traffic = _read_traffic(w.name)
     value = job_value(T, world, ms)
 
-    # end to end through the public API: pinned host inputs -> H2D -> forward -> D2H
     e2e = None
     if not args.no_e2e:
-        qh = q.cpu().pin_memory()
-        kh = k.cpu().pin_memory()
-        vh = v.cpu().pin_memory()
-        cuh = cu.cpu().pin_memory()
-        outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        lseh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-        h2d = qh.numel() * 2 + kh.numel() * 2 + vh.numel() * 2 + cuh.numel() * 4
-        d2h = outh.numel() * 2 + lseh.numel() * 4
-        n_e2e = max(1, min(args.steps, 3))
+        e2e = _e2e_pipelined(moba, w, x, fwd, max(1, min(args.steps, 4)), world)
 
-        def e2e_step():
-            q.copy_(qh, non_blocking=True)
-            k.copy_(kh, non_blocking=True)
-            v.copy_(vh, non_blocking=True)
-            cu.copy_(cuh, non_blocking=True)
-            step()
-            outh.copy_(out, non_blocking=True)
-            lseh.copy_(lse, non_blocking=True)
-
-        e2e_step()
-        torch.cuda.synchronize()
-        barrier(world)
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(n_e2e):
-            e2e_step()
-        b.record()
-        torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, world)
-        e2e = {"value": job_value(T, world, e2e_ms), "unit": "tokens/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-               "steps": n_e2e}
+    # sub-records, measured in this same run (rank 0 of a one-GPU run only)
+    subs = {}
+    if rank == 0 and world == 1 and not args.no_sub_records:
+        del fwd
+        torch.cuda.empty_cache()
+        if w.name != "long_32k":
+            subs["long_32k"] = _sub_forward(moba, W, W.WORKLOADS["long_32k"], dev, 20, 5, peaks,
+                                            max_seqlen=W.WORKLOADS["long_32k"].max_seqlen)
+        subs["packed_64x8k"] = _sub_forward(moba, W, W.ALL_WORKLOADS["packed_64x8k"], dev, 10, 3, peaks,
+                                            max_seqlen=8192)
+        if args.gate == "mean":
+            subs["minmax_gate"] = _sub_forward(moba, W, w, dev, 3, 3, peaks, gate="minmax",
+                                               max_seqlen=max_seqlen, seed=rank_seed(w, rank))
+        subs["backward"] = _sub_backward(moba, W, w, x, dev, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         x_cpu = {kk: vv.cpu() for kk, vv in x.items()}
-        val, det = cpu_oracle_sample(w, args.cpu_seconds, seed=7, inputs=x_cpu)
+        del x
+        torch.cuda.empty_cache()
+        val, det = cpu_oracle_baseline(w, args.cpu_seconds, seed=7, inputs=x_cpu,
+                                       dense=w.total_tokens <= (1 << 16))
         cpu = {"value": val, "unit": "tokens/s", "cores": det["cores"], "kind": "oracle",
-               "sample": det["sample"]}
+               "sample": det["sample"], "cpu_model": det["cpu_model"], "cpu_count": det["cpu_count"],
+               "extrapolated": det["extrapolated"], "gate_seconds_per_head": det["gate_seconds_per_head"],
+               "means_seconds": det["means_seconds"], "rows_sampled": det["rows"]}
+        if "dense_causal_fp64_tokens_per_s" in det:
+            cpu["dense_causal_fp64_tokens_per_s"] = det["dense_causal_fp64_tokens_per_s"]
+            cpu["dense_causal_fp64_note"] = det["dense_causal_fp64_note"]
 
     if rank == 0:
         line = {
@@ -382,8 +591,8 @@ def run_ours(args, w, world, rank, local):
             "config": {"workload": w.name, "description": w.description,
                        "global_batch": len(w.seqlens) * world, "seq_len": w.max_seqlen,
                        "tokens_per_gpu": T, "q_heads": hq, "kv_heads": hkv, "head_dim": d,
-                       "chunk_size": chunk, "topk": topk, "parallelism": f"dp{world}",
-                       "wave_tokens": wave_tokens or T, "waves": waves,
+                       "chunk_size": chunk, "topk": topk, "gate": args.gate,
+                       "parallelism": f"dp{world}", "wave_tokens": wave_tokens, "waves": waves,
                        "l2": "inputs larger than L2 (no flush)"},
             "selected_block_tflops": achieved,
             "selected_block_tflops_over_step": f_sel / (ms * 1e-3) / 1e12,
@@ -395,12 +604,13 @@ def run_ours(args, w, world, rank, local):
                          "peak_kind": ("bf16 sustained" if long_step else "bf16 burst")
                                       + f" ({peaks['source']})",
                          "traffic": traffic},
-            "hbm_stages": _hbm_stage_rates(w, st, peaks),
+            "hbm_stages": _hbm_stage_rates(w, st, peaks, args.gate),
             "clocks": clocks,
             "gpu_launches": launches * args.steps,
             "e2e": e2e,
             "cpu_baseline": cpu,
         }
+        line.update(subs)
         print(json.dumps(line), flush=True)
 
 
@@ -577,8 +787,9 @@ def run_decode_reference(args, w, world, rank):
     }), flush=True)
 
 
-def _hbm_stage_rates(w, st, peaks):
-    """Achieved GB/s of the HBM-bound stages from their algorithmic bytes."""
+def _hbm_stage_rates(w, st, peaks, gate="mean"):
+    """Achieved GB/s of the HBM-bound stages from their algorithmic bytes (the block summary:
+    fp32 means, or the bf16 min and max, the same bytes)."""
     T, hq, hkv, d = w.total_tokens, w.num_q_heads, w.num_kv_heads, w.head_dim
     nb = sum((n + w.chunk_size - 1) // w.chunk_size for n in w.seqlens)
     mean_bytes = T * hkv * d * 2 + nb * hkv * d * 4
@@ -657,12 +868,12 @@ def main():
     ap.add_argument("--decode", action="store_true",
                     help="time the decode step (workloads.DECODE_WORKLOADS) instead of the prefill")
     ap.add_argument("--gate", choices=["mean", "minmax"], default="mean",
-                    help="decode gate: block means, or the min/max (Quest-style) block summary")
+                    help="gate: block means, or the min/max (Quest-style) block summary")
+    ap.add_argument("--no-sub-records", action="store_true",
+                    help="skip the long_32k, packed-batch, min/max-gate and backward sub-records")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.gate != "mean" and not args.decode:
-        ap.error("--gate applies to the decode step (--decode); the prefill gate is the mean gate")
     from block_sparse_long_meanpool_b200 import workloads as W
 
     if args.decode:

@@ -1,5 +1,5 @@
-"""B200-native MoBA (Mixture of Block Attention): the causal prefill forward, the decode step
-with the mean or the min/max block gate.
+"""B200-native MoBA (Mixture of Block Attention): the causal prefill forward and its backward
+pass, the decode step with the mean or the min/max block gate.
 
 The compute path is the C-ABI library ``libmoba.so`` (CUDA for sm_100a, headers in
 ``include/moba.h``); ``moba`` is its thin ctypes binding and ``workloads`` makes seeded
@@ -8,6 +8,7 @@ synthetic inputs.  Build the library with ``python -m block_sparse_long_meanpool
 
 from .moba import (  # noqa: F401
     MobaError,
+    attn_bwd,
     attn_fwd,
     decode_fwd,
     decode_minmax_fwd,

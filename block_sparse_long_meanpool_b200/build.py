@@ -14,7 +14,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmoba.so")
-SOURCES = ["moba_api.cu", "meanpool.cu", "gate.cu", "gate_tc.cu", "route.cu", "attn_tc.cu", "merge.cu", "decode.cu", "minmaxpool.cu", "noalloc.cu"]
+SOURCES = ["moba_api.cu", "meanpool.cu", "gate.cu", "gate_tc.cu", "route.cu", "attn_tc.cu", "merge.cu", "decode.cu", "minmaxpool.cu", "noalloc.cu", "attn_bwd.cu"]
 HEADERS = ["moba_internal.cuh", "ptx.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

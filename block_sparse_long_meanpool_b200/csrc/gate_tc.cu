@@ -1,24 +1,35 @@
 // Steps 3-4 of the forward on the tensor cores: gate scores of 128-row query tiles against the
-// block means by tcgen05 MMA, then the future-block mask, the forced own block and the hard
-// top-k in registers.
+// block summaries by tcgen05 MMA, then the future-block mask, the forced own block and the
+// hard top-k on the CUDA cores.
 //
 // The analysis page of the MoBA paper (§2.2-§2.3): s_j = <q, mean_j>; blocks after the row's
 // own block c are masked to -inf, block c is always taken, the best topk-1 past blocks
-// (j < c) are routed.  Ties keep the lower block index.
+// (j < c) are routed.  Ties keep the lower block index.  The same kernel runs the min/max
+// (Quest-style) gate the analysis names as the stronger summary (§1.3, §5.1 item 6, §6.3):
+// s_j = sum_i max(q_i kmin_ji, q_i kmax_ji).
 //
-// Precision: each fp32 mean is split exactly into three bf16 parts, m = hi + mid + lo
-// (|m - hi - mid - lo| <= 2^-24 |m|), and the three products with the bf16 query row are
-// accumulated in fp32 by three MMAs into the same TMEM accumulator.  The score is therefore
-// the fp32-accurate dot product (about 1e-6 absolute here), far inside the 1e-3 relative
-// near-tie band, unlike a single bf16 rounding of the means (about 2e-3 relative).
+// Both scores are contractions with exact bf16 operands and fp32 accumulation:
+//   mean:    each fp32 mean is split exactly into three bf16 parts, m = hi + mid + lo
+//            (|m - hi - mid - lo| <= 2^-24 |m|), and s = q.hi + q.mid + q.lo: three MMAs of
+//            K = d into one accumulator, so the score is the fp32-accurate dot product (about
+//            1e-6 absolute here), far inside the 1e-3 relative near-tie band, unlike a single
+//            bf16 rounding of the means (about 2e-3 relative);
+//   min/max: max(q_i lo_i, q_i hi_i) = q+_i hi_i + q-_i lo_i with q+ = max(q, 0) and
+//            q- = min(q, 0), so s = q+.kmax + q-.kmin: two MMAs of K = d whose products are
+//            exact (bf16 x bf16 in fp32); only the fp32 accumulation rounds.
 //
-// One CTA per (query block b, KV head g): it stages the split means of the c past blocks of
-// b's sequence in shared memory once (SWIZZLE_128B, K-major), then runs the 128-row tiles of
-// block b for the query heads of g.  Warp 4 loads each Q tile by TMA and issues the MMAs
-// (N = c rounded up to 16) into one of two TMEM accumulators; warps 0-3 (one thread per row)
-// read the scores with tcgen05.ld and keep a sorted top-(topk-1) list in registers.  Rows
-// with fewer than topk-1 past blocks take all of them.  Sequences longer than 256 blocks use
-// the fp32 CUDA-core gate instead (gate.cu).
+// One CTA per (query block b, KV head g): it stages the summaries of the c past blocks of b's
+// sequence in shared memory once (SWIZZLE_128B, K-major), then runs the 128-row tiles of block
+// b for the query heads of g.  The last warp loads each Q tile by TMA (and, for the min/max
+// gate, splits it into q+ and q-) and issues the MMAs (N = c rounded up to 16) into TMEM.  Four
+// warpgroups (two for long lists; thread = row, TMEM lane) select the top-(topk-1): the
+// 64-column slices of a tile's scores are split over 1, 2 or 4 warpgroups, each keeps
+// a sorted list of its slice in registers, and the lists are merged pairwise through TMEM
+// (the merging warpgroup reads its partner's list from the columns the partner has finished
+// with, after a bounded mbarrier handshake) under the (score descending, index ascending)
+// order.  Rows with at most topk-1 past
+// blocks take all of them without scoring.  Sequences longer than 257 blocks use the fp32
+// CUDA-core gate instead (gate.cu).
 #include <climits>
 
 #include "moba_internal.cuh"
@@ -31,24 +42,71 @@ namespace {
 using namespace ptx;
 
 constexpr int kMaxPast = 256;   // past blocks scored in one MMA (N <= 256)
-constexpr int kThreads = 160;   // warps 0-3 top-k, warp 4 TMA + MMA
-constexpr int kWarpMMA = 4;
+constexpr int kSliceCols = 64;  // score columns per warpgroup slice
 
-template <int D>
-struct GateSmem {
-    static constexpr int kQ = 0;                         // Q tile [128 x D] bf16, swizzled
-    static constexpr int kMeans = kTileM * D * 2;        // 3 splits x [N x D] bf16
-    static constexpr int kBars(int n) { return kMeans + 3 * n * D * 2; }
-    static constexpr int kBytes(int n) { return kBars(n) + 8 * 8 + 16 + 1024; }
+// Top-k warpgroups: four, or two when the lists are long (topk - 1 > 11), so that each
+// thread keeps its list, a 32-score load and a partner's list in registers.
+template <int KMAX>
+struct GateWarps {
+    static constexpr int kNumWG = KMAX > 11 ? 2 : 4;
+    static constexpr int kThreads = kNumWG * 128 + 32;  // + the TMA / MMA warp
+    static constexpr int kWarpMMA = kNumWG * 4;
 };
 
-template <int D, int KMAX>
-__global__ void __launch_bounds__(kThreads, 1)
+__host__ __device__ constexpr int pow2_at_least(int x) {
+    int p = 32;
+    while (p < x) p *= 2;
+    return p;
+}
+
+// TMEM plan of one launch (the same in every CTA): NC columns per score buffer (a power of two
+// >= the largest N), WPT warpgroups per tile (one per 64-column slice), NGRP = NWG / WPT tile
+// groups taking tiles in turn, NB buffers per group (two when one group takes every tile).
+struct GatePlan {
+    int nc, wpt, ngrp, nb, cols;
+};
+__host__ __device__ inline GatePlan gate_plan(int n_alloc, int nwg) {
+    GatePlan g;
+    g.nc = pow2_at_least(n_alloc);
+    g.wpt = g.nc / kSliceCols;
+    if (g.wpt < 1) g.wpt = 1;
+    if (g.wpt > nwg) g.wpt = nwg;
+    g.ngrp = nwg / g.wpt;
+    g.nb = g.ngrp == 1 ? 2 : 1;
+    g.cols = g.ngrp * g.nb * g.nc;
+    return g;
+}
+
+template <int D, bool MINMAX>
+struct GateCfg {
+    static constexpr int kPairs = MINMAX ? 2 : 3;     // (A, B) products accumulated per score
+    static constexpr int kARegions = MINMAX ? 2 : 1;  // q (mean) or q+, q- (min/max)
+    static constexpr int kTile = kTileM * D * 2;      // one [128 x D] bf16 tile
+    // shared memory: NQ Q buffers, then kPairs B regions of [N x D] bf16, then barriers
+    static constexpr int kQBytes(int nq) { return nq * kARegions * kTile; }
+    static constexpr int kBars(int nq, int n) { return kQBytes(nq) + kPairs * n * D * 2; }
+    static constexpr int kNumBars = 24;
+    static constexpr int kBytes(int nq, int n) { return kBars(nq, n) + kNumBars * 8 + 16 + 1024; }
+};
+
+// q -> (q+, q-) in place: per bf16, q+ keeps positive values (and +0), q- negative ones.
+__device__ __forceinline__ void split_sign(uint32_t x, uint32_t& pos, uint32_t& neg) {
+    const uint32_t m = ((x >> 15) & 0x00010001u) * 0xFFFFu;  // 0xFFFF per negative half
+    pos = x & ~m;
+    neg = x & m;
+}
+
+template <int D, int KMAX, bool MINMAX>
+__global__ void __launch_bounds__(GateWarps<KMAX>::kThreads, 1)
 gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restrict__ means,
-               const int* __restrict__ cu, Problem P, int* __restrict__ sel, int* status,
-               int n_cap) {
-    using L = GateSmem<D>;
+               const __nv_bfloat16* __restrict__ kmin, const __nv_bfloat16* __restrict__ kmax,
+               const int* __restrict__ cu, Problem P, int* __restrict__ sel, int* status, int n_cap,
+               int nq) {
+    using C = GateCfg<D, MINMAX>;
+    constexpr int kThreads = GateWarps<KMAX>::kThreads;
+    constexpr int kWarpMMA = GateWarps<KMAX>::kWarpMMA;
     constexpr int kHalfBytesQ = kTileM * 128;
+    constexpr bool kTwoLists = KMAX <= 16;  // a second list for instruction-level parallelism
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
@@ -77,78 +135,100 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
     const int qtiles = (len + kTileM - 1) / kTileM;
     const int ntiles = qtiles * P.group;
 
-    if (n_route == 0 || c > n_cap) {
-        // nothing to score: every row takes its own block only.  c > n_cap means the sequence
-        // is longer than the caller's max_seqlen promised: its rows keep the own block only
-        // and the call's status word (when there is one) records the broken promise.
-        if (c > n_cap && threadIdx.x == 0 && status) atomicExch(status, 1 /* INVALID_ARG */);
+    if (n_route == c || c > n_cap) {
+        // nothing to choose: every past block is routed (c <= topk - 1).  c > n_cap means the
+        // sequence is longer than the caller's max_seqlen promised: its rows keep the own block
+        // only and the call's status word (when there is one) records the broken promise.
+        const bool broken = c > n_cap;
+        if (broken && threadIdx.x == 0 && status) atomicExch(status, 1 /* INVALID_ARG */);
         for (int e = threadIdx.x; e < len * P.group; e += kThreads) {
             const int h = g * P.group + e / len;
             const int t = start + e % len;
             int* dst = sel + ((size_t)h * P.T + t) * P.topk;
-            for (int i = 0; i < P.topk; ++i) dst[i] = (i == 0) ? c : -1;
+            const int nr = broken ? 0 : c;
+            for (int i = 0; i < P.topk; ++i) dst[i] = (i < nr) ? i : (i == nr ? c : -1);
         }
         return;
     }
-    const int N = (c + 15) & ~15;  // MMA N: past blocks rounded up to 16 (c <= kMaxPast)
+    const int N = (c + 15) & ~15;  // MMA N: past blocks rounded up to 16 (c <= n_cap)
     const int split_bytes = N * D * 2;
+    const GatePlan plan = gate_plan(n_cap, GateWarps<KMAX>::kNumWG);
     const uint32_t sm_base = smem_u32(smem);
-    const uint32_t m_base = sm_base + L::kMeans;
-    const uint32_t bar0 = sm_base + L::kBars(N);
+    const uint32_t b_base = sm_base + C::kQBytes(nq);
+    const uint32_t bar0 = sm_base + C::kBars(nq, N);
     auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-    const int B_QFULL = 0, B_QEMPTY = 1, B_SFULL = 2, B_SEMPTY = 4, B_FINAL = 6;
+    // B_XFER + 3 grp + k: a partner's list is in TMEM (k = 0: part 1 -> 0, 1: part 3 -> 2,
+    // 2: part 2 -> 0)
+    const int B_QFULL = 0, B_QEMPTY = 2, B_SFULL = 4, B_SEMPTY = 8, B_FINAL = 12, B_XFER = 13;
 
-    // stage the split means of past blocks 0..c-1 (rows c..N-1 are zero)
+    // stage the summaries of past blocks 0..c-1 as K-major SW128 rows (rows c..N-1 are zero)
     {
-        const float* mg = means + ((size_t)s_first * P.hkv + g) * D;
         const size_t mstride = (size_t)P.hkv * D;
-        for (int e = threadIdx.x; e < N * (D / 4); e += kThreads) {
-            const int j = e / (D / 4), d0 = (e % (D / 4)) * 4;
-            float4 m4 = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (j < c) m4 = __ldg(reinterpret_cast<const float4*>(mg + (size_t)j * mstride + d0));
-            const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
-            uint32_t part[3][2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                float r0 = mv[2 * u], r1 = mv[2 * u + 1];
-                __nv_bfloat16 h0[3], h1[3];
-#pragma unroll
-                for (int k = 0; k < 3; ++k) {
-                    h0[k] = __float2bfloat16_rn(r0);
-                    h1[k] = __float2bfloat16_rn(r1);
-                    r0 -= __bfloat162float(h0[k]);
-                    r1 -= __bfloat162float(h1[k]);
-                    __nv_bfloat162 pr;
-                    pr.x = h0[k];
-                    pr.y = h1[k];
-                    part[k][u] = *reinterpret_cast<uint32_t*>(&pr);
-                }
-            }
-            // byte offset of (row j, column d0) in a K-major SWIZZLE_128B region of N rows
+        // byte offset of (row j, column d0) in a K-major SWIZZLE_128B region of N rows
+        auto swz = [&](int j, int d0) {
             const int half = d0 / 64, col = d0 % 64;
-            const uint32_t off = (uint32_t)half * (uint32_t)(N * 128) + (uint32_t)j * 128u +
-                                 (uint32_t)((((col / 8) ^ (j & 7)) << 4) + (col % 8) * 2);
+            return (uint32_t)half * (uint32_t)(N * 128) + (uint32_t)j * 128u +
+                   (uint32_t)((((col / 8) ^ (j & 7)) << 4) + (col % 8) * 2);
+        };
+        if constexpr (MINMAX) {
+            const __nv_bfloat16* hi0 = kmax + ((size_t)s_first * P.hkv + g) * D;
+            const __nv_bfloat16* lo0 = kmin + ((size_t)s_first * P.hkv + g) * D;
+            for (int e = threadIdx.x; e < N * (D / 8); e += kThreads) {
+                const int j = e / (D / 8), d0 = (e % (D / 8)) * 8;
+                uint4 h4 = make_uint4(0u, 0u, 0u, 0u), l4 = h4;
+                if (j < c) {
+                    h4 = __ldg(reinterpret_cast<const uint4*>(hi0 + (size_t)j * mstride + d0));
+                    l4 = __ldg(reinterpret_cast<const uint4*>(lo0 + (size_t)j * mstride + d0));
+                }
+                *reinterpret_cast<uint4*>(smem + C::kQBytes(nq) + swz(j, d0)) = h4;
+                *reinterpret_cast<uint4*>(smem + C::kQBytes(nq) + split_bytes + swz(j, d0)) = l4;
+            }
+        } else {
+            const float* mg = means + ((size_t)s_first * P.hkv + g) * D;
+            for (int e = threadIdx.x; e < N * (D / 4); e += kThreads) {
+                const int j = e / (D / 4), d0 = (e % (D / 4)) * 4;
+                float4 m4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (j < c) m4 = __ldg(reinterpret_cast<const float4*>(mg + (size_t)j * mstride + d0));
+                const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
+                uint32_t part[3][2];
 #pragma unroll
-            for (int k = 0; k < 3; ++k) {
-                uint8_t* dst = smem + L::kMeans + k * split_bytes + off;
-                *reinterpret_cast<uint2*>(dst) = make_uint2(part[k][0], part[k][1]);
+                for (int u = 0; u < 2; ++u) {
+                    float r0 = mv[2 * u], r1 = mv[2 * u + 1];
+#pragma unroll
+                    for (int k = 0; k < 3; ++k) {
+                        const __nv_bfloat16 h0 = __float2bfloat16_rn(r0), h1 = __float2bfloat16_rn(r1);
+                        r0 -= __bfloat162float(h0);
+                        r1 -= __bfloat162float(h1);
+                        __nv_bfloat162 pr;
+                        pr.x = h0;
+                        pr.y = h1;
+                        part[k][u] = *reinterpret_cast<uint32_t*>(&pr);
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < 3; ++k)
+                    *reinterpret_cast<uint2*>(smem + C::kQBytes(nq) + k * split_bytes + swz(j, d0)) =
+                        make_uint2(part[k][0], part[k][1]);
             }
         }
     }
     fence_proxy_async();  // the MMAs read these shared-memory writes through the async proxy
     if (threadIdx.x == 0) {
-        mbar_init(BAR(B_QFULL), 1);
-        mbar_init(BAR(B_QEMPTY), 1);
-        mbar_init(BAR(B_SFULL), 1);
-        mbar_init(BAR(B_SFULL + 1), 1);
-        mbar_init(BAR(B_SEMPTY), 128);
-        mbar_init(BAR(B_SEMPTY + 1), 128);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(BAR(B_QFULL + i), 1);
+            mbar_init(BAR(B_QEMPTY + i), 1);
+        }
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(BAR(B_SFULL + i), 1);
+            mbar_init(BAR(B_SEMPTY + i), 128 * plan.wpt);
+        }
         mbar_init(BAR(B_FINAL), 1);
+        for (int i = 0; i < 6; ++i) mbar_init(BAR(B_XFER + i), 128);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == kWarpMMA) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
-                         smem_u32(&s_tmem)));
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&s_tmem)), "r"(plan.cols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     tc_fence_before();
@@ -160,38 +240,60 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
     int* st = status ? status : &dummy_status;
 
     if (warp == kWarpMMA) {
+        // ---------------- Q tiles (TMA), q+ / q- split, MMA issue ----------------
         const uint32_t idesc = idesc_bf16(N, false);
         for (int ti = 0; ti < ntiles; ++ti) {
             const int h = g * P.group + ti % P.group, qt = ti / P.group;
-            if (ti > 0 && !wait_bar(BAR(B_QEMPTY), (uint32_t)(ti - 1) & 1u, abort_flag, st)) break;
+            const int qb = ti % nq;
+            const uint32_t uq = (uint32_t)(ti / nq);
+            if (ti >= nq && !wait_bar(BAR(B_QEMPTY + qb), (uq - 1u) & 1u, abort_flag, st)) break;
+            const uint32_t qbase = sm_base + (uint32_t)qb * C::kARegions * C::kTile;
             if (lane == 0) {
-                mbar_arrive_tx(BAR(B_QFULL), (uint32_t)(kTileM * D * 2));
+                mbar_arrive_tx(BAR(B_QFULL + qb), (uint32_t)C::kTile);
 #pragma unroll
                 for (int hh = 0; hh < D / 64; ++hh)
-                    tma_load_3d(sm_base + L::kQ + hh * kHalfBytesQ, &tmap_q, BAR(B_QFULL), hh * 64, h,
+                    tma_load_3d(qbase + hh * kHalfBytesQ, &tmap_q, BAR(B_QFULL + qb), hh * 64, h,
                                 start + qt * kTileM);
             }
             __syncwarp();
-            const int sb = ti & 1;
-            if (!wait_bar(BAR(B_QFULL), (uint32_t)ti & 1u, abort_flag, st)) break;
-            if (ti >= 2 && !wait_bar(BAR(B_SEMPTY + sb), (uint32_t)((ti >> 1) - 1) & 1u, abort_flag, st))
-                break;
+            if (!wait_bar(BAR(B_QFULL + qb), uq & 1u, abort_flag, st)) break;
+            if constexpr (MINMAX) {
+                uint4* qp = reinterpret_cast<uint4*>(smem + (size_t)qb * C::kARegions * C::kTile);
+                uint4* qm = qp + C::kTile / 16;
+                for (int i = lane; i < C::kTile / 16; i += 32) {
+                    const uint4 x = qp[i];
+                    uint4 p4, n4;
+                    split_sign(x.x, p4.x, n4.x);
+                    split_sign(x.y, p4.y, n4.y);
+                    split_sign(x.z, p4.z, n4.z);
+                    split_sign(x.w, p4.w, n4.w);
+                    qp[i] = p4;
+                    qm[i] = n4;
+                }
+                fence_proxy_async();
+                __syncwarp();
+            }
+            const int grp = ti % plan.ngrp, u = ti / plan.ngrp;
+            const int buf = grp * plan.nb + u % plan.nb;
+            const uint32_t ub = (uint32_t)(u / plan.nb);
+            if (ub >= 1 && !wait_bar(BAR(B_SEMPTY + buf), (ub - 1u) & 1u, abort_flag, st)) break;
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t s_tmem = tmem + (uint32_t)sb * kMaxPast;
+                const uint32_t s_tmem = tmem + (uint32_t)(buf * plan.nc);
 #pragma unroll
-                for (int k = 0; k < 3; ++k) {
+                for (int p = 0; p < C::kPairs; ++p) {
+                    const uint32_t abase = qbase + (uint32_t)(MINMAX ? p : 0) * C::kTile;
+                    const uint32_t bbase = b_base + (uint32_t)p * (uint32_t)split_bytes;
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t aoff = (uint32_t)(kk >> 2) * kHalfBytesQ + (uint32_t)(kk & 3) * 32u;
-                        const uint32_t boff = (uint32_t)k * split_bytes + (uint32_t)(kk >> 2) * (uint32_t)(N * 128) +
-                                              (uint32_t)(kk & 3) * 32u;
-                        mma_ss(s_tmem, smem_desc(sm_base + L::kQ + aoff, 16, 1024),
-                               smem_desc(m_base + boff, 16, 1024), idesc, (k > 0 || kk > 0) ? 1u : 0u);
+                        const uint32_t boff = (uint32_t)(kk >> 2) * (uint32_t)(N * 128) + (uint32_t)(kk & 3) * 32u;
+                        mma_ss(s_tmem, smem_desc(abase + aoff, 16, 1024), smem_desc(bbase + boff, 16, 1024),
+                               idesc, (p > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
-                mma_commit(BAR(B_SFULL + sb));
-                mma_commit(BAR(B_QEMPTY));
+                mma_commit(BAR(B_SFULL + buf));
+                mma_commit(BAR(B_QEMPTY + qb));
             }
             __syncwarp();
         }
@@ -199,17 +301,26 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
         __syncwarp();
         drain_bar(BAR(B_FINAL), 0);
     } else {
-        // warps 0-3: thread r owns row r of every tile
-        const int r = threadIdx.x;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        for (int ti = 0; ti < ntiles; ++ti) {
+        // ---------------- top-k: warpgroup wg, thread = row ----------------
+        const int wg = warp >> 2;
+        const int grp = wg / plan.wpt, part = wg % plan.wpt;
+        const int r = threadIdx.x & 127;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        // this warpgroup's slice of the score columns
+        const int col_lo = part * kSliceCols;
+        const int col_hi = min(c, plan.wpt == 1 ? plan.nc : col_lo + kSliceCols);
+        const int xfer0 = B_XFER + grp * 3;
+        bool ok = true;
+        for (int ti = grp; ok && ti < ntiles; ti += plan.ngrp) {
             const int h = g * P.group + ti % P.group, qt = ti / P.group;
-            const int sb = ti & 1;
-            if (!wait_bar(BAR(B_SFULL + sb), (uint32_t)(ti >> 1) & 1u, abort_flag, st)) break;
+            const int u = ti / plan.ngrp;
+            const int buf = grp * plan.nb + u % plan.nb;
+            const uint32_t ub = (uint32_t)(u / plan.nb);
+            if (!wait_bar(BAR(B_SFULL + buf), ub & 1u, abort_flag, st)) break;
             tc_fence_after();
-            // two independent descending lists (even / odd columns) for instruction-level
-            // parallelism, merged at the end; inside a list, columns arrive in increasing order
-            // and an equal score never displaces an earlier (lower-index) block
+            const uint32_t s_tmem = tmem + lane_off + (uint32_t)(buf * plan.nc);
+            // lists sorted by (score descending, index ascending); inside a list columns arrive
+            // in increasing order and an equal score never displaces an earlier (lower) block
             float val[KMAX], val2[KMAX];
             int idx[KMAX], idx2[KMAX];
 #pragma unroll
@@ -217,23 +328,75 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
                 val[i] = val2[i] = -INFINITY;
                 idx[i] = idx2[i] = INT_MAX;
             }
-            const uint32_t s_tmem = tmem + lane_off + (uint32_t)sb * kMaxPast;
-            for (int j0 = 0; j0 < c; j0 += 32) {
+            for (int j0 = col_lo; j0 < col_hi; j0 += 32) {
                 float v[32];
                 tmem_ld32(s_tmem + (uint32_t)j0, v);
+                if constexpr (kTwoLists) {
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    insert_desc<KMAX>(val, idx, v[e], j0 + e, j0 + e < c);
-                    insert_desc<KMAX>(val2, idx2, v[e + 1], j0 + e + 1, j0 + e + 1 < c);
+                    for (int e = 0; e < 32; e += 2) {
+                        insert_desc<KMAX>(val, idx, v[e], j0 + e, j0 + e < col_hi);
+                        insert_desc<KMAX>(val2, idx2, v[e + 1], j0 + e + 1, j0 + e + 1 < col_hi);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) insert_desc<KMAX>(val, idx, v[e], j0 + e, j0 + e < col_hi);
                 }
             }
-            // merge: scores from the odd list enter with the full (score, lower index) order
+            if constexpr (kTwoLists) {
 #pragma unroll
-            for (int i = 0; i < KMAX; ++i) insert_ordered<KMAX>(val, idx, val2[i], idx2[i]);
+                for (int i = 0; i < KMAX; ++i) insert_ordered<KMAX>(val, idx, val2[i], idx2[i]);
+            }
+            // merge the slices of the tile pairwise through TMEM: level 1 (parts 1 -> 0, 3 -> 2),
+            // level 2 (part 2 -> 0); a list goes over the columns its writer has read
+            bool holder = true;
+            for (int lvl = 1; lvl < plan.wpt; lvl <<= 1) {
+                if (part % (2 * lvl) == lvl) {
+                    uint32_t w[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) w[i] = 0u;
+#pragma unroll
+                    for (int i = 0; i < KMAX && i < 16; ++i) {
+                        w[2 * i] = __float_as_uint(val[i]);
+                        w[2 * i + 1] = (uint32_t)idx[i];
+                    }
+                    tmem_st32(s_tmem + (uint32_t)col_lo, w);
+                    if constexpr (KMAX > 16) {
+#pragma unroll
+                        for (int i = 16; i < KMAX; ++i) {
+                            w[2 * (i - 16)] = __float_as_uint(val[i]);
+                            w[2 * (i - 16) + 1] = (uint32_t)idx[i];
+                        }
+                        tmem_st32(s_tmem + (uint32_t)col_lo + 32u, w);
+                    }
+                    tmem_st_wait();
+                    tc_fence_before();
+                    mbar_arrive(BAR(xfer0 + (lvl == 1 ? part / 2 : 2)));
+                    holder = false;
+                    break;
+                } else if (part % (2 * lvl) == 0) {
+                    if (!wait_bar(BAR(xfer0 + (lvl == 1 ? part / 2 : 2)), (uint32_t)u & 1u, abort_flag, st)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    float o[32];
+                    tmem_ld32(s_tmem + (uint32_t)((part + lvl) * kSliceCols), o);
+#pragma unroll
+                    for (int i = 0; i < KMAX && i < 16; ++i)
+                        insert_ordered<KMAX>(val, idx, o[2 * i], (int)__float_as_uint(o[2 * i + 1]));
+                    if constexpr (KMAX > 16) {
+                        tmem_ld32(s_tmem + (uint32_t)((part + lvl) * kSliceCols) + 32u, o);
+#pragma unroll
+                        for (int i = 16; i < KMAX; ++i)
+                            insert_ordered<KMAX>(val, idx, o[2 * (i - 16)], (int)__float_as_uint(o[2 * (i - 16) + 1]));
+                    }
+                }
+            }
+            if (!ok) break;
             tc_fence_before();
-            mbar_arrive(BAR(B_SEMPTY + sb));
+            mbar_arrive(BAR(B_SEMPTY + buf));
             const int rr = qt * kTileM + r;
-            if (rr < len) {
+            if (holder && rr < len) {
                 int o[KMAX];
 #pragma unroll
                 for (int i = 0; i < KMAX; ++i) o[i] = (i < n_route) ? idx[i] : INT_MAX;
@@ -262,7 +425,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
     __syncthreads();
     tc_fence_after();
     if (warp == kWarpMMA) {
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(plan.cols));
     }
 }
 
@@ -284,8 +447,8 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-template <int D, int KMAX>
-cudaError_t launch_tc(const Problem& P, const __nv_bfloat16* q, const float* means, const int* cu,
+template <int D, int KMAX, bool MINMAX>
+cudaError_t launch_tc(const Problem& P, const __nv_bfloat16* q, const GateSummary& s, const int* cu,
                       int* sel, int* status, int n_max, cudaStream_t st) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
@@ -298,43 +461,57 @@ cudaError_t launch_tc(const Problem& P, const __nv_bfloat16* q, const float* mea
            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    const int smem = GateSmem<D>::kBytes(n_max);
-    cudaError_t e = cudaFuncSetAttribute(gate_tc_kernel<D, KMAX>,
+    using C = GateCfg<D, MINMAX>;
+    // two Q buffers when they fit next to the summaries, else one
+    const int limit = 227 * 1024;
+    const int nq = C::kBytes(2, n_max) <= limit ? 2 : 1;
+    const int smem = C::kBytes(nq, n_max);
+    cudaError_t e = cudaFuncSetAttribute(gate_tc_kernel<D, KMAX, MINMAX>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid(P.nb_cap, P.hkv);
-    gate_tc_kernel<D, KMAX><<<grid, kThreads, smem, st>>>(mq, means, cu, P, sel, status, n_max);
+    gate_tc_kernel<D, KMAX, MINMAX><<<grid, GateWarps<KMAX>::kThreads, smem, st>>>(mq, s.means, s.kmin, s.kmax, cu, P, sel,
+                                                                   status, n_max, nq);
     return cudaGetLastError();
 }
 
-template <int D>
-cudaError_t launch_tc_k(const Problem& P, const __nv_bfloat16* q, const float* means,
-                        const int* cu, int* sel, int* status, int n_max, cudaStream_t st) {
+template <int D, bool MINMAX>
+cudaError_t launch_tc_k(const Problem& P, const __nv_bfloat16* q, const GateSummary& s, const int* cu,
+                        int* sel, int* status, int n_max, cudaStream_t st) {
     const int need = P.topk - 1;
-    if (need <= 2) return launch_tc<D, 2>(P, q, means, cu, sel, status, n_max, st);
-    if (need <= 4) return launch_tc<D, 4>(P, q, means, cu, sel, status, n_max, st);
-    if (need <= 8) return launch_tc<D, 8>(P, q, means, cu, sel, status, n_max, st);
-    if (need <= 11) return launch_tc<D, 11>(P, q, means, cu, sel, status, n_max, st);
-    if (need <= 16) return launch_tc<D, 16>(P, q, means, cu, sel, status, n_max, st);
-    return launch_tc<D, 32>(P, q, means, cu, sel, status, n_max, st);
+    if (need <= 2) return launch_tc<D, 2, MINMAX>(P, q, s, cu, sel, status, n_max, st);
+    if (need <= 4) return launch_tc<D, 4, MINMAX>(P, q, s, cu, sel, status, n_max, st);
+    if (need <= 8) return launch_tc<D, 8, MINMAX>(P, q, s, cu, sel, status, n_max, st);
+    if (need <= 11) return launch_tc<D, 11, MINMAX>(P, q, s, cu, sel, status, n_max, st);
+    if (need <= 16) return launch_tc<D, 16, MINMAX>(P, q, s, cu, sel, status, n_max, st);
+    return launch_tc<D, 32, MINMAX>(P, q, s, cu, sel, status, n_max, st);
 }
 
 }  // namespace
 
 // Tensor-core gate when every sequence has at most kMaxPast + 1 blocks (P.max_blocks, from the
 // caller's max_seqlen, else the block-count bound of the whole call), else the fp32 CUDA-core
-// gate.  Shared memory and the MMA's N are sized for the longest sequence's past blocks.
-cudaError_t launch_gate_best(const Problem& P, const __nv_bfloat16* q, const float* means,
+// gate (mean gate only).  Shared memory, TMEM and the MMA's N are sized for the longest
+// sequence's past blocks.
+cudaError_t launch_gate_best(const Problem& P, const __nv_bfloat16* q, const GateSummary& s,
                              const int* cu_seqlens, int* sel, int* status, cudaStream_t st,
                              int* path) {
     if (P.nb_cap == 0) return cudaSuccess;
+    const bool minmax = s.kmin != nullptr;
     const bool cuda_cores = P.max_blocks > kMaxPast + 1;
     if (path) *path = cuda_cores ? 2 : 1;
-    if (cuda_cores) return launch_gate(P, q, means, cu_seqlens, sel, st);
+    if (cuda_cores) {
+        if (minmax) return cudaErrorNotSupported;
+        return launch_gate(P, q, s.means, cu_seqlens, sel, st);
+    }
     const int n_max = ((P.max_blocks - 1) + 15) & ~15;  // largest c is max_blocks - 1
     const int n_alloc = n_max < 16 ? 16 : n_max;
-    if (P.d == 64) return launch_tc_k<64>(P, q, means, cu_seqlens, sel, status, n_alloc, st);
-    return launch_tc_k<128>(P, q, means, cu_seqlens, sel, status, n_alloc, st);
+    if (minmax) {
+        if (P.d == 64) return launch_tc_k<64, true>(P, q, s, cu_seqlens, sel, status, n_alloc, st);
+        return launch_tc_k<128, true>(P, q, s, cu_seqlens, sel, status, n_alloc, st);
+    }
+    if (P.d == 64) return launch_tc_k<64, false>(P, q, s, cu_seqlens, sel, status, n_alloc, st);
+    return launch_tc_k<128, false>(P, q, s, cu_seqlens, sel, status, n_alloc, st);
 }
 
 }  // namespace moba

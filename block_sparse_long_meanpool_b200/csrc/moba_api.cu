@@ -64,6 +64,9 @@ moba_status check_params(const moba_params* p) {
         return fail(MOBA_ERR_INVALID_ARG, "chunk_size must be >= 1 (got %d)", p->chunk_size);
     if (p->head_dim < 1) return fail(MOBA_ERR_INVALID_ARG, "head_dim must be >= 1");
     if (p->wave_tokens < 0) return fail(MOBA_ERR_INVALID_ARG, "wave_tokens must be >= 0");
+    if (p->gate != MOBA_GATE_MEAN && p->gate != MOBA_GATE_MINMAX)
+        return fail(MOBA_ERR_INVALID_ARG, "gate must be MOBA_GATE_MEAN or MOBA_GATE_MINMAX (got %d)",
+                    p->gate);
     if (p->max_seqlen < 0)
         return fail(MOBA_ERR_INVALID_ARG, "max_seqlen must be >= 0 (got %d)", p->max_seqlen);
     if (p->max_seqlen > 0 &&
@@ -175,6 +178,15 @@ int device_sm_count() {
     return n;
 }
 
+// The min/max gate runs on the tensor cores only: every sequence must have <= 257 blocks.
+moba_status check_minmax_gate(const Problem& P) {
+    if (P.max_blocks > 257)
+        return fail(MOBA_ERR_UNSUPPORTED,
+                    "the min/max gate needs every sequence to have <= 257 blocks (%d possible; "
+                    "give max_seqlen)", P.max_blocks);
+    return MOBA_OK;
+}
+
 // Index-range limits of the 32-bit indices used on the device.
 moba_status check_ranges(const moba_params& p, const Layout& L) {
     const long long lim = 0x7fffffffLL;
@@ -249,8 +261,30 @@ moba_status moba_gate_topk(const moba_params* p, const void* q, const float* k_m
     if (!aligned16(q) || !aligned16(k_mean))
         return fail(MOBA_ERR_INVALID_ARG, "q and k_mean must be 16-byte aligned");
     const Problem P = make_problem(*p, blocks_bound(*p));
-    cudaError_t e = launch_gate_best(P, static_cast<const __nv_bfloat16*>(q), k_mean, cu_seqlens,
-                                     sel, nullptr, static_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_gate_best(P, static_cast<const __nv_bfloat16*>(q),
+                                     GateSummary{k_mean, nullptr, nullptr}, cu_seqlens, sel, nullptr,
+                                     static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "gate launch");
+    return MOBA_OK;
+}
+
+moba_status moba_gate_minmax_topk(const moba_params* p, const void* q, const void* k_min,
+                                  const void* k_max, const int* cu_seqlens, int* sel, void* stream) {
+    NvtxScope range("moba_gate_minmax_topk");
+    moba_status s = check_params(p);
+    if (s != MOBA_OK) return s;
+    if (p->total_tokens == 0) return MOBA_OK;
+    if (!q || !k_min || !k_max || !cu_seqlens || !sel)
+        return fail(MOBA_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned16(q) || !aligned16(k_min) || !aligned16(k_max))
+        return fail(MOBA_ERR_INVALID_ARG, "q, k_min and k_max must be 16-byte aligned");
+    const Problem P = make_problem(*p, blocks_bound(*p));
+    s = check_minmax_gate(P);
+    if (s != MOBA_OK) return s;
+    cudaError_t e = launch_gate_best(P, static_cast<const __nv_bfloat16*>(q),
+                                     GateSummary{nullptr, static_cast<const __nv_bfloat16*>(k_min),
+                                                 static_cast<const __nv_bfloat16*>(k_max)},
+                                     cu_seqlens, sel, nullptr, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "gate launch");
     return MOBA_OK;
 }
@@ -283,6 +317,10 @@ moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, co
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const Problem P = make_problem(*p, L.nb_cap);
+    if (!sel_in && p->gate == MOBA_GATE_MINMAX) {
+        s = check_minmax_gate(P);
+        if (s != MOBA_OK) return s;
+    }
     char* base = static_cast<char*>(workspace);
     Workspace ws;
     ws.hdr = reinterpret_cast<WsHeader*>(base + L.hdr);
@@ -318,11 +356,21 @@ moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, co
         if (e != cudaSuccess) return cuda_fail(e, what); \
     } while (0)
 
+    // the block summary of the gate: fp32 means, or the bf16 min/max pair in the same bytes
+    const bool minmax = p->gate == MOBA_GATE_MINMAX;
+    const size_t summ_elems = (size_t)L.nb_cap * P.hkv * P.d;
+    __nv_bfloat16* kmin_ws = reinterpret_cast<__nv_bfloat16*>(ws.means);
+    __nv_bfloat16* kmax_ws = kmin_ws + summ_elems;
+    const GateSummary summary = minmax ? GateSummary{nullptr, kmin_ws, kmax_ws}
+                                       : GateSummary{ws.means, nullptr, nullptr};
     MOBA_TRY(record(MOBA_EV_BEGIN), "event record");
     {
         NvtxScope stage("means");
         MOBA_TRY(launch_plan_blocks(P, cu_seqlens, ws, st), "block table launch");
-        MOBA_TRY(launch_meanpool(P, kb, cu_seqlens, ws.means, st), "meanpool launch");
+        if (minmax)
+            MOBA_TRY(launch_minmaxpool(P, kb, cu_seqlens, kmin_ws, kmax_ws, st), "minmaxpool launch");
+        else
+            MOBA_TRY(launch_meanpool(P, kb, cu_seqlens, ws.means, st), "meanpool launch");
     }
     launches += 2;
     MOBA_TRY(record(MOBA_EV_MEANS_DONE), "event record");
@@ -331,7 +379,7 @@ moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, co
         NvtxScope stage("gate");
         int* dst = sel_out ? sel_out : ws.sel;
         int path = MOBA_GATE_PATH_NONE;
-        MOBA_TRY(launch_gate_best(P, qb, ws.means, cu_seqlens, dst, &ws.hdr->status, st, &path),
+        MOBA_TRY(launch_gate_best(P, qb, summary, cu_seqlens, dst, &ws.hdr->status, st, &path),
                  "gate launch");
         if (info) info->gate_path = path;
         ++launches;
@@ -374,6 +422,140 @@ moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, co
         info->launches = launches;
         info->waves = w;
     }
+    return MOBA_OK;
+}
+
+// ---- backward -------------------------------------------------------------------------
+
+namespace {
+
+struct BwdLayout {
+    size_t hdr, cu_blocks, blk_start, blk_len, blk_seq, blk_local, counts, offsets, cursor,
+        entries, items, nslots, rs, dq_acc, total;
+    long long nb_cap, max_items;
+};
+
+// The backward routes every row at once (one wave from token 0) and keeps no partial outputs:
+// the block table, the routing lists and work items of all T tokens, per-row statistics and
+// an fp32 dq accumulator.
+BwdLayout make_bwd_layout(const moba_params& p) {
+    moba_params one = p;
+    one.wave_tokens = 0;
+    const Layout F = make_layout(one);  // work-item bound of a single wave over all tokens
+    BwdLayout L{};
+    const long long T = p.total_tokens;
+    L.nb_cap = F.nb_cap;
+    L.max_items = F.max_items;
+    const long long lists = (long long)p.num_kv_heads * L.nb_cap;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o = align_up(o + bytes);
+        return at;
+    };
+    L.hdr = take(sizeof(WsHeader));
+    L.cu_blocks = take(4ull * (p.batch + 1));
+    L.blk_start = take(4ull * L.nb_cap);
+    L.blk_len = take(4ull * L.nb_cap);
+    L.blk_seq = take(4ull * L.nb_cap);
+    L.blk_local = take(4ull * L.nb_cap);
+    L.counts = take(4ull * lists);
+    L.offsets = take(4ull * (lists + 1));
+    L.cursor = take(4ull * lists);
+    L.entries = take(4ull * T * p.num_q_heads * (p.topk - 1));
+    L.items = take(sizeof(WorkItem) * L.max_items);
+    L.nslots = take(1ull * T * p.num_q_heads);
+    L.rs = take(8ull * T * p.num_q_heads);
+    L.dq_acc = take(4ull * T * p.num_q_heads * p.head_dim);
+    L.total = o;
+    return L;
+}
+
+}  // namespace
+
+size_t moba_bwd_workspace_size(const moba_params* p) {
+    if (check_params(p) != MOBA_OK) return 0;
+    return make_bwd_layout(*p).total;
+}
+
+moba_status moba_attn_bwd(const moba_params* p, const void* q, const void* k, const void* v,
+                          const void* out, const float* lse, const void* d_out, const float* d_lse,
+                          const int* cu_seqlens, const int* sel, void* workspace,
+                          size_t workspace_bytes, void* dq, void* dk, void* dv, void* stream) {
+    NvtxScope range("moba_attn_bwd");
+    moba_status s = check_params(p);
+    if (s != MOBA_OK) return s;
+    if (p->total_tokens == 0) return MOBA_OK;
+    if (!q || !k || !v || !out || !lse || !d_out || !cu_seqlens || !sel || !dq || !dk || !dv)
+        return fail(MOBA_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(d_out) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return fail(MOBA_ERR_INVALID_ARG, "q, k, v, out, d_out, dq, dk and dv must be 16-byte aligned");
+    if ((long long)p->total_tokens * p->num_q_heads * p->topk > 0x7fffffffLL)
+        return fail(MOBA_ERR_UNSUPPORTED, "total_tokens * num_q_heads * topk exceeds 2^31");
+    const BwdLayout L = make_bwd_layout(*p);
+    if (L.max_items > 0x7fffffffLL || (long long)p->num_kv_heads * L.nb_cap > 0x7fffffffLL)
+        return fail(MOBA_ERR_UNSUPPORTED, "too many blocks for 32-bit work indices");
+    if ((long long)p->num_kv_heads * L.nb_cap * (p->chunk_size / kTileM) > 0x7fffffffLL)
+        return fail(MOBA_ERR_UNSUPPORTED, "too many key tiles for one launch");
+    if (!workspace || workspace_bytes < L.total)
+        return fail(MOBA_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", L.total,
+                    workspace ? workspace_bytes : (size_t)0);
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+        return fail(MOBA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const Problem P = make_problem(*p, L.nb_cap);
+    char* base = static_cast<char*>(workspace);
+    Workspace ws{};
+    ws.hdr = reinterpret_cast<WsHeader*>(base + L.hdr);
+    ws.cu_blocks = reinterpret_cast<int*>(base + L.cu_blocks);
+    ws.blk_start = reinterpret_cast<int*>(base + L.blk_start);
+    ws.blk_len = reinterpret_cast<int*>(base + L.blk_len);
+    ws.blk_seq = reinterpret_cast<int*>(base + L.blk_seq);
+    ws.blk_local = reinterpret_cast<int*>(base + L.blk_local);
+    ws.counts = reinterpret_cast<int*>(base + L.counts);
+    ws.offsets = reinterpret_cast<int*>(base + L.offsets);
+    ws.cursor = reinterpret_cast<int*>(base + L.cursor);
+    ws.entries = reinterpret_cast<int*>(base + L.entries);
+    ws.items = reinterpret_cast<WorkItem*>(base + L.items);
+    ws.nslots = reinterpret_cast<unsigned char*>(base + L.nslots);
+    BwdArgs a;
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.k = static_cast<const __nv_bfloat16*>(k);
+    a.v = static_cast<const __nv_bfloat16*>(v);
+    a.out = static_cast<const __nv_bfloat16*>(out);
+    a.dout = static_cast<const __nv_bfloat16*>(d_out);
+    a.lse = lse;
+    a.dlse = d_lse;
+    a.rs = reinterpret_cast<float2*>(base + L.rs);
+    a.dq_acc = reinterpret_cast<float*>(base + L.dq_acc);
+    a.dq = static_cast<__nv_bfloat16*>(dq);
+    a.dk = static_cast<__nv_bfloat16*>(dk);
+    a.dv = static_cast<__nv_bfloat16*>(dv);
+
+    const int T = p->total_tokens;
+    int launches = 0;
+    cudaError_t e;
+#define MOBA_TRY(expr, what)                             \
+    do {                                                 \
+        e = (expr);                                      \
+        if (e != cudaSuccess) return cuda_fail(e, what); \
+    } while (0)
+    {
+        NvtxScope stage("route");
+        MOBA_TRY(launch_plan_blocks(P, cu_seqlens, ws, st), "block table launch");
+        MOBA_TRY(cudaMemsetAsync(ws.counts, 0, 4ull * P.hkv * L.nb_cap, st), "memset");
+        MOBA_TRY(launch_route_count(P, cu_seqlens, sel, ws, 0, T, st), "route count launch");
+        MOBA_TRY(launch_route_plan(P, ws, 0, T, st), "route plan launch");
+        MOBA_TRY(launch_route_scatter(P, cu_seqlens, sel, ws, 0, T, st), "route scatter launch");
+        MOBA_TRY(cudaMemsetAsync(a.dq_acc, 0, 4ull * T * P.hq * P.d, st), "memset");
+    }
+    {
+        NvtxScope stage("attention");
+        MOBA_TRY(launch_backward(P, a, ws, device_sm_count(), st, &launches), "backward launch");
+    }
+#undef MOBA_TRY
     return MOBA_OK;
 }
 

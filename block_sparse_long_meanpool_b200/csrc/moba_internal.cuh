@@ -153,9 +153,11 @@ cudaError_t launch_minmaxpool(const Problem& P, const __nv_bfloat16* k, const in
                               __nv_bfloat16* kmin, __nv_bfloat16* kmax, cudaStream_t st);
 cudaError_t launch_gate(const Problem& P, const __nv_bfloat16* q, const float* means,
                         const int* cu_seqlens, int* sel, cudaStream_t st);
-// Runs the tensor-core gate when every sequence fits it, else the CUDA-core gate; *path (when
-// non-null) receives MOBA_GATE_PATH_TENSOR_CORES (1) or MOBA_GATE_PATH_CUDA_CORES (2).
-cudaError_t launch_gate_best(const Problem& P, const __nv_bfloat16* q, const float* means,
+struct GateSummary;
+// Runs the tensor-core gate (mean or min/max summary) when every sequence fits it, else the
+// CUDA-core gate (mean summary only; the min/max summary returns cudaErrorNotSupported); *path
+// (when non-null) receives MOBA_GATE_PATH_TENSOR_CORES (1) or MOBA_GATE_PATH_CUDA_CORES (2).
+cudaError_t launch_gate_best(const Problem& P, const __nv_bfloat16* q, const GateSummary& s,
                              const int* cu_seqlens, int* sel, int* status, cudaStream_t st,
                              int* path = nullptr);
 cudaError_t launch_route_count(const Problem& P, const int* cu_seqlens, const int* sel,
@@ -170,6 +172,20 @@ cudaError_t launch_attention(const Problem& P, const __nv_bfloat16* q, const __n
 cudaError_t launch_merge(const Problem& P, const int* cu_seqlens, const int* sel,
                          const Workspace& ws, int t0, int t1, __nv_bfloat16* out, float* lse,
                          cudaStream_t st);
+
+// Buffers of one backward call (moba_attn_bwd).
+struct BwdArgs {
+    const __nv_bfloat16 *q, *k, *v, *out, *dout;
+    const float* lse;   // [hq, T]
+    const float* dlse;  // [hq, T] or nullptr
+    float2* rs;         // [hq, T]: (lse * log2 e, <dO, out> - dlse)
+    float* dq_acc;      // [T, hq, d] fp32 accumulator, zeroed before the dQ kernel
+    __nv_bfloat16 *dq, *dk, *dv;
+};
+// Row statistics, dK/dV, dQ and the dq conversion, after the routing pass over all rows
+// (one wave from token 0).  *launches is incremented per kernel queued.
+cudaError_t launch_backward(const Problem& P, const BwdArgs& a, const Workspace& ws, int num_sms,
+                            cudaStream_t st, int* launches);
 
 // Views into the workspace of one decode step (P.batch sequences, one query row each).
 struct DecodeWorkspace {
@@ -187,13 +203,14 @@ inline int decode_splits(int batch, int hq, int topk, int chunk) {
     while ((long long)batch * hq * topk * s < 1184 && topk * s * 2 <= 64 && chunk / (s * 2) >= 128) s *= 2;
     return s;
 }
-// Block summary the decode gate scores against: the fp32 means (kmin == kmax == nullptr) or
-// the bf16 min/max pair (means == nullptr), each [NB, Hkv, d].
-struct DecodeGate {
+// Block summary a gate scores against: the fp32 means (kmin == kmax == nullptr) or the bf16
+// min/max pair (means == nullptr), each [NB, Hkv, d].
+struct GateSummary {
     const float* means;
     const __nv_bfloat16* kmin;
     const __nv_bfloat16* kmax;
 };
+using DecodeGate = GateSummary;
 cudaError_t launch_decode(const Problem& P, const __nv_bfloat16* q, const __nv_bfloat16* k,
                           const __nv_bfloat16* v, const int* cu_seqlens, const DecodeGate& gate,
                           const DecodeWorkspace& ws, __nv_bfloat16* out, float* lse,

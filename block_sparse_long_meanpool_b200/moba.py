@@ -22,8 +22,11 @@ EXPORTS = (
     "moba_meanpool",
     "moba_minmaxpool",
     "moba_gate_topk",
+    "moba_gate_minmax_topk",
     "moba_attn_fwd",
     "moba_attn_fwd_noalloc",
+    "moba_bwd_workspace_size",
+    "moba_attn_bwd",
     "moba_decode_workspace_size",
     "moba_decode_fwd",
     "moba_decode_minmax_fwd",
@@ -55,6 +58,7 @@ class MobaParams(ctypes.Structure):
         ("topk", ctypes.c_int),
         ("softmax_scale", ctypes.c_float),
         ("wave_tokens", ctypes.c_int),
+        ("gate", ctypes.c_int),
     ]
 
 
@@ -98,11 +102,17 @@ def load_library(path=LIB_PATH):
     lib.moba_minmaxpool.restype = ctypes.c_int
     lib.moba_gate_topk.argtypes = [P, vp, vp, vp, vp, vp]
     lib.moba_gate_topk.restype = ctypes.c_int
+    lib.moba_gate_minmax_topk.argtypes = [P, vp, vp, vp, vp, vp, vp]
+    lib.moba_gate_minmax_topk.restype = ctypes.c_int
     lib.moba_attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp,
                                   ctypes.POINTER(MobaRunInfo), vp]
     lib.moba_attn_fwd.restype = ctypes.c_int
     lib.moba_attn_fwd_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
     lib.moba_attn_fwd_noalloc.restype = ctypes.c_int
+    lib.moba_bwd_workspace_size.argtypes = [P]
+    lib.moba_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.moba_attn_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp, vp, vp]
+    lib.moba_attn_bwd.restype = ctypes.c_int
     lib.moba_decode_workspace_size.argtypes = [P]
     lib.moba_decode_workspace_size.restype = ctypes.c_size_t
     lib.moba_decode_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp, vp]
@@ -132,11 +142,15 @@ def _check(status):
         raise MobaError(status, f"{name}: {msg}")
 
 
+GATES = {"mean": 0, "minmax": 1}  # moba_params.gate (MOBA_GATE_MEAN, MOBA_GATE_MINMAX)
+
+
 def make_params(batch, total_tokens, num_q_heads, num_kv_heads, head_dim, chunk_size, topk,
-                softmax_scale=None, wave_tokens=0, max_seqlen=0):
+                softmax_scale=None, wave_tokens=0, max_seqlen=0, gate="mean"):
     return MobaParams(int(batch), int(total_tokens), int(max_seqlen or 0), int(num_q_heads),
                       int(num_kv_heads), int(head_dim), int(chunk_size), int(topk),
-                      float(softmax_scale) if softmax_scale else 0.0, int(wave_tokens))
+                      float(softmax_scale) if softmax_scale else 0.0, int(wave_tokens),
+                      GATES[gate] if isinstance(gate, str) else int(gate))
 
 
 def _ptr(t):
@@ -277,6 +291,23 @@ def gate_topk(q, k_mean, cu_seqlens, chunk_size, topk, num_kv_heads=None, max_se
     return sel
 
 
+def gate_minmax_topk(q, k_min, k_max, cu_seqlens, chunk_size, topk, max_seqlen=None):
+    """Selections int32 [Hq, T, topk] with the min/max block summary (moba_gate_minmax_topk):
+    k_min, k_max bf16 [NB, Hkv, d] from ``minmaxpool``."""
+    _check_qkv(q, None)
+    batch = cu_seqlens.numel() - 1
+    T, hq, d = q.shape
+    hkv = k_min.shape[1]
+    p = make_params(batch, T, hq, hkv, d, chunk_size, topk, max_seqlen=max_seqlen)
+    bound = num_blocks_bound(p)
+    _require_summary(k_min, "k_min", torch.bfloat16, bound, hkv, d, q.device)
+    _require_summary(k_max, "k_max", torch.bfloat16, bound, hkv, d, q.device)
+    sel = torch.empty((hq, T, topk), dtype=torch.int32, device=q.device)
+    _check(load_library().moba_gate_minmax_topk(ctypes.byref(p), _ptr(q), _ptr(k_min), _ptr(k_max),
+                                                _ptr(cu_seqlens), _ptr(sel), _stream(q.device)))
+    return sel
+
+
 def _decode(fn, summary, q, k, v, cu_seqlens, chunk_size, topk, softmax_scale, workspace, out, lse):
     _check_qkv(q, k, v)
     _require(cu_seqlens.is_cuda, "cu_seqlens must be a CUDA tensor")
@@ -378,12 +409,13 @@ def choose_wave_tokens(T, hq, hkv, d, chunk_size, topk, batch, budget_bytes):
 
 def attn_fwd(q, k, v, cu_seqlens, chunk_size, topk, softmax_scale=None, sel=None,
              return_sel=False, wave_tokens=None, workspace=None, events=None,
-             workspace_budget=None, out=None, lse=None, max_seqlen=None):
+             workspace_budget=None, out=None, lse=None, max_seqlen=None, gate="mean"):
     """MoBA causal prefill forward (moba_attn_fwd).
 
     q bf16 [T, Hq, d], k/v bf16 [T, Hkv, d], cu_seqlens int32 [batch + 1] on the device.
     sel: optional int32 [Hq, T, topk] selection to use instead of the gate.
     max_seqlen: the longest sequence's length when known on the host (0 / None: unknown).
+    gate: "mean" (the paper's mean-pooled block summary) or "minmax" (the min/max summary).
     Returns (out bf16 [T, Hq, d], lse fp32 [Hq, T]) and, with return_sel, the gate's
     selection.  ``events`` may be a list of torch.cuda.Event recorded at the library's stage
     boundaries; the call's moba_run_info is returned in ``attn_fwd.last_info``.
@@ -400,7 +432,7 @@ def attn_fwd(q, k, v, cu_seqlens, chunk_size, topk, softmax_scale=None, sel=None
             free, _ = torch.cuda.mem_get_info(dev)
             workspace_budget = min(int(free * 0.45), 48 << 30)
         wave_tokens = choose_wave_tokens(T, hq, hkv, d, chunk_size, topk, batch, workspace_budget)
-    p = make_params(batch, T, hq, hkv, d, chunk_size, topk, softmax_scale, wave_tokens, max_seqlen)
+    p = make_params(batch, T, hq, hkv, d, chunk_size, topk, softmax_scale, wave_tokens, max_seqlen, gate)
     need = workspace_size(p)
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
@@ -441,3 +473,56 @@ def attn_fwd(q, k, v, cu_seqlens, chunk_size, topk, softmax_scale=None, sel=None
 
 
 attn_fwd.last_info = None
+
+
+def attn_bwd(q, k, v, out, lse, d_out, cu_seqlens, chunk_size, topk, sel, d_lse=None,
+             softmax_scale=None, workspace=None, dq=None, dk=None, dv=None, max_seqlen=None):
+    """Backward of the MoBA forward (moba_attn_bwd): gradients of out and lse with respect to
+    q, k and v, with the forward's selection ``sel`` held fixed.
+
+    q bf16 [T, Hq, d], k/v bf16 [T, Hkv, d], out bf16 [T, Hq, d] and lse fp32 [Hq, T] (the
+    forward's outputs), d_out bf16 [T, Hq, d], d_lse fp32 [Hq, T] or None, sel int32
+    [Hq, T, topk].  Returns (dq bf16 [T, Hq, d], dk, dv bf16 [T, Hkv, d]); the call's
+    workspace size and launches are in ``attn_bwd.last_info``.
+    """
+    _check_qkv(q, k, v)
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    dev = q.device
+    _require(k.shape == v.shape and k.shape[0] == T and k.shape[2] == d, "k/v shape mismatch")
+    _require(cu_seqlens.dtype == torch.int32 and cu_seqlens.is_cuda, "cu_seqlens int32 CUDA")
+    _require_buffer(out, "out", (T, hq, d), torch.bfloat16, dev)
+    _require_buffer(lse, "lse", (hq, T), torch.float32, dev)
+    _require_buffer(d_out, "d_out", (T, hq, d), torch.bfloat16, dev)
+    if d_lse is not None:
+        _require_buffer(d_lse, "d_lse", (hq, T), torch.float32, dev)
+    _require_buffer(sel, "sel", (hq, T, topk), torch.int32, dev)
+    batch = cu_seqlens.numel() - 1
+    p = make_params(batch, T, hq, hkv, d, chunk_size, topk, softmax_scale, 0, max_seqlen)
+    lib = load_library()
+    need = lib.moba_bwd_workspace_size(ctypes.byref(p))
+    if need == 0 and T > 0:
+        raise MobaError(ERR_INVALID_ARG, lib.moba_last_error().decode())
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    if dq is None:
+        dq = torch.empty((T, hq, d), dtype=torch.bfloat16, device=dev)
+    else:
+        _require_buffer(dq, "dq", (T, hq, d), torch.bfloat16, dev)
+    if dk is None:
+        dk = torch.empty((T, hkv, d), dtype=torch.bfloat16, device=dev)
+    else:
+        _require_buffer(dk, "dk", (T, hkv, d), torch.bfloat16, dev)
+    if dv is None:
+        dv = torch.empty((T, hkv, d), dtype=torch.bfloat16, device=dev)
+    else:
+        _require_buffer(dv, "dv", (T, hkv, d), torch.bfloat16, dev)
+    _check(lib.moba_attn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                             _ptr(d_out), _ptr(d_lse), _ptr(cu_seqlens), _ptr(sel), _ptr(workspace),
+                             ctypes.c_size_t(workspace.numel()), _ptr(dq), _ptr(dk), _ptr(dv),
+                             _stream(dev)))
+    attn_bwd.last_info = {"workspace_bytes": need}
+    return dq, dk, dv
+
+
+attn_bwd.last_info = None

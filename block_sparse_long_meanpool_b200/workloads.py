@@ -91,7 +91,15 @@ LENGTH_SWEEP["prefill_10m"] = Workload(
     "prefill_10m", [10 << 20], 8, 2, 128, (10 << 20) // 256, 12, "k_offsets", 1210,
     "1 x 10485760 tokens, 8 q / 2 kv heads (a quarter of a 32/8-head layer), d=128, "
     "256 blocks of 40960, top-12")
-ALL_WORKLOADS = {**WORKLOADS, **GRANULARITY_32K, **LENGTH_SWEEP}
+# A packed training batch of many short sequences: 64 x 8192 tokens, 1024 blocks of 512 in all
+# but 16 per sequence (the gate is sized by the longest sequence, given as max_seqlen).
+PACKED = {
+    "packed_64x8k": Workload(
+        "packed_64x8k", [8192] * 64, 32, 8, 128, 512, 3, "k_offsets", 1400,
+        "64 packed sequences of 8192 tokens, 32 q / 8 kv heads, d=128, chunk 512 (16 blocks each, "
+        "1024 in all), top-3"),
+}
+ALL_WORKLOADS = {**WORKLOADS, **GRANULARITY_32K, **LENGTH_SWEEP, **PACKED}
 
 # Decode step: caches of these shapes, one new query per sequence (its last row).
 DECODE_WORKLOADS = {

@@ -78,7 +78,13 @@ typedef struct {
     int wave_tokens;      /* moba_attn_fwd only: query tokens per wave, 0 = all tokens in one
                              wave; otherwise a positive multiple of 128.  Bounds the workspace
                              (per-wave partial outputs), see moba_workspace_size. */
+    int gate;             /* moba_attn_fwd / moba_attn_fwd_noalloc only: the block summary the
+                             gate scores against, MOBA_GATE_MEAN (0, the paper's mean pooling)
+                             or MOBA_GATE_MINMAX (1, the min/max summary, see
+                             moba_gate_minmax_topk).  Other values: MOBA_ERR_INVALID_ARG. */
 } moba_params;
+
+enum { MOBA_GATE_MEAN = 0, MOBA_GATE_MINMAX = 1 };
 
 /* Optional instrumentation for moba_attn_fwd.  All fields may be left zero. */
 typedef struct {
@@ -148,6 +154,21 @@ moba_status moba_minmaxpool(const moba_params* p, const void* k, const int* cu_s
 moba_status moba_gate_topk(const moba_params* p, const void* q, const float* k_mean,
                            const int* cu_seqlens, int* sel, void* stream);
 
+/* Steps 3-4 with the min/max (Quest-style) block summary in place of the mean (the analysis
+ * names Quest as the MoBA variant that pools blocks by min and max, §1.3, the stronger summary,
+ * §5.1 item 6 and §6.3): an earlier block j is scored by
+ *   s_j = sum_i max(q_i k_min[j, g, i], q_i k_max[j, g, i])
+ * (the largest q . x over the block's bounding box), computed exactly as
+ * q+ . k_max_j + q- . k_min_j with q+ = max(q, 0), q- = min(q, 0) on the tensor cores (bf16
+ * products exact, fp32 sum).  Mask, forced own block, top-k and tie rule as moba_gate_topk.
+ *   q              bf16 [T, Hq, d] device
+ *   k_min, k_max   bf16 [NB, Hkv, d] device, as written by moba_minmaxpool
+ *   sel            int32 [Hq, T, topk] device, written in full (ascending, -1 padded)
+ * Every sequence must have at most 257 blocks (bounded by max_seqlen, else by the whole
+ * call's block count), else MOBA_ERR_UNSUPPORTED.  Uses no workspace. */
+moba_status moba_gate_minmax_topk(const moba_params* p, const void* q, const void* k_min,
+                                  const void* k_max, const int* cu_seqlens, int* sel, void* stream);
+
 /* The whole forward (steps 1-5): mean-pool, gate (unless sel_in is given), routing of rows
  * to (KV head, block) lists, block attention on the tensor cores, log-sum-exp merge.
  *   q, k, v     bf16 device, see conventions
@@ -162,14 +183,43 @@ moba_status moba_gate_topk(const moba_params* p, const void* q, const float* k_m
  *   out         bf16 [T, Hq, d] device (fp32 merge rounded to nearest even)
  *   lse         fp32 [Hq, T] device: natural-log log-sum-exp of the scaled logits
  *   info        optional instrumentation, may be NULL
+ * With p->gate = MOBA_GATE_MINMAX the gate scores with the min/max summary (computed in the
+ * workspace, in place of the means) as moba_gate_minmax_topk does, under its 257-block limit.
  * Workspace contents are undefined after the call. */
 moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, const void* v,
                           const int* cu_seqlens, const int* sel_in, int* sel_out,
                           void* workspace, size_t workspace_bytes, void* out, float* lse,
                           moba_run_info* info, void* stream);
 
-/* Reads (synchronously, on `stream`) the device status word a previous moba_attn_fwd left in
- * `workspace`: MOBA_OK, or MOBA_ERR_DEVICE_TIMEOUT when a bounded device-side wait gave up.
+/* ---- Backward pass --------------------------------------------------------------------
+ *
+ * Gradients of the forward's out and lse with respect to q, k and v.  The analysis page of the
+ * MoBA paper trains with MoBA (§3.3: continual pre-training up to 1M tokens) and makes it a
+ * parameter-equivalent replacement of full attention (§2.5): the gate has no parameters and
+ * routes by hard top-k (§2.2), so the selection is piecewise constant and the gradient flows
+ * only through the softmax attention over the selected blocks (§2.2-§2.3).  The backward
+ * therefore holds the forward's selection fixed and differentiates the attention:
+ *   p_u = exp(scale q.k_u - lse),  dv_u += p_u dO,  dz_u = p_u (dO.v_u - <dO, out> + d_lse),
+ *   dq = scale sum_u dz_u k_u,  dk_u += scale dz_u q  (summed over the query heads of a KV head).
+ *   q, k, v      bf16, as for moba_attn_fwd
+ *   out, lse     the forward's outputs (bf16 [T, Hq, d], fp32 [Hq, T])
+ *   d_out        bf16 [T, Hq, d]; d_lse fp32 [Hq, T] or NULL (zero)
+ *   sel          int32 [Hq, T, topk]: the selection the forward used (moba_attn_fwd's sel_out, or
+ *                the sel_in it was given), read with the same rule as sel_in
+ *   workspace    >= moba_bwd_workspace_size(p) bytes, 256-byte aligned (routing lists of all
+ *                rows and an fp32 dq accumulator [T, Hq, d]); p->wave_tokens is ignored
+ *   dq           bf16 [T, Hq, d]; dk, dv bf16 [T, Hkv, d]: written in full
+ * Runs on the tensor cores (tcgen05); asynchronous on `stream`; argument errors return before
+ * any launch; T * Hq * topk must stay below 2^31 (MOBA_ERR_UNSUPPORTED).  A bounded device wait
+ * that gives up is reported through moba_device_status on this workspace. */
+size_t moba_bwd_workspace_size(const moba_params* p);
+moba_status moba_attn_bwd(const moba_params* p, const void* q, const void* k, const void* v,
+                          const void* out, const float* lse, const void* d_out, const float* d_lse,
+                          const int* cu_seqlens, const int* sel, void* workspace,
+                          size_t workspace_bytes, void* dq, void* dk, void* dv, void* stream);
+
+/* Reads (synchronously, on `stream`) the device status word a previous moba_attn_fwd (or
+ * moba_attn_bwd) left in `workspace`: MOBA_OK, or MOBA_ERR_DEVICE_TIMEOUT when a bounded device-side wait gave up.
  * Waits for the stream. */
 moba_status moba_device_status(const moba_params* p, const void* workspace, void* stream);
 

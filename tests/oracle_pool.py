@@ -81,10 +81,12 @@ def _compare_head(gsel_h, osel_h, q16, means_g, cu, chunk, topk):
     return np.asarray(ties, dtype=np.int64), bad
 
 
-def _select_rows(q_rows16, ts, means_g, cu, chunk, topk):
-    """oracle.select_blocks_rows for sampled tokens of one query head."""
-    return oracle.select_blocks_rows(_RowsView(q_rows16, ts), means_g[:, None, :], cu, chunk, topk,
-                                     [(int(t), i) for i, t in enumerate(ts)])
+def _select_rows(q_rows16, ts, summary_g, cu, chunk, topk, minmax):
+    """oracle.select_blocks_rows for sampled tokens of one query head: the mean gate against
+    summary_g [NB, d], or the min/max gate against summary_g [NB, 2, d] (min, max)."""
+    score = oracle.minmax_scores_row if minmax else oracle.gate_scores_row
+    return oracle.select_blocks_rows(_RowsView(q_rows16, ts), summary_g[:, None], cu, chunk, topk,
+                                     [(int(t), i) for i, t in enumerate(ts)], score=score)
 
 
 def _attend(q_rows16, ts, k16, v16, cu, chunk, sel_rows, scale):
@@ -94,6 +96,14 @@ def _attend(q_rows16, ts, k16, v16, cu, chunk, sel_rows, scale):
     v = PT.from_bits(v16)[:, None, :]
     return oracle.attend_rows(_RowsView(q_rows16, ts), k, v, cu, chunk, sel_rows,
                               [(int(t), i) for i, t in enumerate(ts)], scale)
+
+
+def _backward_head(q_h, k_g, v_g, cu, chunk, sel_h, dout_h, dlse_h, scale):
+    """oracle.moba_backward for one query head against its KV head: returns that head's dq and
+    its contribution to the KV head's dk and dv."""
+    dq, dk, dv = oracle.moba_backward(q_h[:, None], k_g[:, None], v_g[:, None], cu, chunk, sel_h[None],
+                                      dout_h[:, None], None if dlse_h is None else dlse_h[None], scale)
+    return dq[:, 0], dk[:, 0], dv[:, 0]
 
 
 class _RowsView:
@@ -178,16 +188,40 @@ def attend_rows_par(ex, rows, q_row16, k16, v16, cu, chunk, sel_rows, group, sca
     return out, lse
 
 
-def select_rows_par(ex, rows, q_row16, means, cu, chunk, topk, group):
-    """oracle.select_blocks_rows for sampled (t, h) rows, one task per head."""
+def select_rows_par(ex, rows, q_row16, means, cu, chunk, topk, group, minmax=False):
+    """oracle.select_blocks_rows for sampled (t, h) rows, split by head into about one task
+    per worker.  ``means`` is [NB, Hkv, d], or [NB, Hkv, 2, d] (min, max) with minmax=True."""
     hs = np.array([h for _, h in rows])
     ts = np.array([t for t, _ in rows])
     res = np.zeros((len(rows), topk), dtype=np.int64)
     futs = []
+    per_task = max(64, math.ceil(len(rows) / n_workers()))
     for h in np.unique(hs):
-        idx = np.nonzero(hs == h)[0]
-        futs.append((idx, ex.submit(_select_rows, q_row16[idx], ts[idx],
-                                    np.ascontiguousarray(means[:, h // group]), cu, chunk, topk)))
+        idx_h = np.nonzero(hs == h)[0]
+        for idx in np.array_split(idx_h, max(1, math.ceil(len(idx_h) / per_task))):
+            futs.append((idx, ex.submit(_select_rows, q_row16[idx], ts[idx],
+                                        np.ascontiguousarray(means[:, h // group]), cu, chunk, topk, minmax)))
     for idx, f in futs:
         res[idx] = f.result()
     return res
+
+
+def backward_by_head(ex, q, k, v, cu, chunk, sel, d_out, d_lse=None, scale=None):
+    """oracle.moba_backward split by query head: dq of each head is that head's; dk and dv of a
+    KV head are the sums of its query heads' contributions (the oracle's GQA rule)."""
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    group = hq // hkv
+    futs = [ex.submit(_backward_head, np.ascontiguousarray(q[:, h]), np.ascontiguousarray(k[:, h // group]),
+                      np.ascontiguousarray(v[:, h // group]), cu, chunk, np.ascontiguousarray(sel[h]),
+                      np.ascontiguousarray(d_out[:, h]), None if d_lse is None else np.ascontiguousarray(d_lse[h]),
+                      scale) for h in range(hq)]
+    dq = np.zeros((T, hq, d))
+    dk = np.zeros((T, hkv, d))
+    dv = np.zeros((T, hkv, d))
+    for h, f in enumerate(futs):
+        a, b, c = f.result()
+        dq[:, h] = a
+        dk[:, h // group] += b
+        dv[:, h // group] += c
+    return dq, dk, dv

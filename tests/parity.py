@@ -75,11 +75,12 @@ def well_formed(sel_row, c, topk):
             and r[n] == c and all(x == -1 for x in r[n + 1:]))
 
 
-def near_tie_alternative(gpu_row, ref_row, scores, c, topk, tie_rel=TIE_REL):
+def near_tie_alternative(gpu_row, ref_row, scores, c, topk, tie_rel=TIE_REL, slack=None):
     """True when gpu_row is a well-formed selection that routes the oracle's blocks except for
     swaps at the top-k cut: every oracle block it drops and every block it routes instead have
-    oracle scores within tie_rel (relative) of each other.  ``scores`` are the oracle's gate
-    scores of blocks 0..c-1 of the row."""
+    oracle scores within tie_rel (relative) of each other, or, when ``slack`` (an absolute error
+    bound of the GPU's score per block) is given, within the sum of their two bounds.
+    ``scores`` are the oracle's gate scores of blocks 0..c-1 of the row."""
     if not well_formed(gpu_row, c, topk):
         return False
     n = min(topk - 1, c)
@@ -88,16 +89,32 @@ def near_tie_alternative(gpu_row, ref_row, scores, c, topk, tie_rel=TIE_REL):
     for i in o - g:
         for j in g - o:
             a, b = float(scores[i]), float(scores[j])
-            if a - b > tie_rel * max(abs(a), abs(b)):
+            band = tie_rel * max(abs(a), abs(b)) if slack is None else float(slack[i] + slack[j])
+            if a - b > band:
                 return False
     return True
 
 
+def minmax_slack(q_row, summary_rows):
+    """Absolute error bound of the GPU's min/max gate score of each block: the score is the fp32
+    sum of the 2d exact products q+_i kmax_i and q-_i kmin_i (q+ = max(q, 0), q- = min(q, 0)),
+    added in an order the tensor core chooses, so it is off by at most
+    (2d - 1) 2^-24 sum_i (|q+_i kmax_i| + |q-_i kmin_i|).  ``summary_rows`` is [n, 2, d]
+    (index 0 = min, 1 = max)."""
+    q = np.asarray(q_row, dtype=np.float64)
+    mm = np.asarray(summary_rows, dtype=np.float64)
+    qp, qn = np.maximum(q, 0.0), np.minimum(q, 0.0)
+    mag = np.abs(mm[:, 1, :] * qp).sum(axis=1) + np.abs(mm[:, 0, :] * qn).sum(axis=1)
+    return (2 * q.shape[0] - 1) * 2.0 ** -24 * mag
+
+
 def check_selection(gpu_sel, ref_sel, rows, q, summary, cu, chunk, topk, group,
-                    score=oracle.gate_scores_row, tie_rel=TIE_REL):
+                    score=oracle.gate_scores_row, tie_rel=TIE_REL, slack_fn=None):
     """gpu_sel / ref_sel: [n, topk] for the listed (t, h) rows.  Returns the set of row
     indices whose GPU selection differs from the oracle's as a valid near-tie alternative
-    (``near_tie_alternative``); any other difference, or a malformed row, fails."""
+    (``near_tie_alternative``; with ``slack_fn(q_row, summary_rows)`` the band is the GPU's
+    error bound per block instead of the relative band); any other difference, or a malformed
+    row, fails."""
     gpu_sel = np.asarray(gpu_sel)
     ref_sel = np.asarray(ref_sel)
     ties = set()
@@ -106,9 +123,11 @@ def check_selection(gpu_sel, ref_sel, rows, q, summary, cu, chunk, topk, group,
     for r in diff:
         t, h = rows[r]
         _, b0, c = row_block(cu, chunk, t)
-        sc = score(np.asarray(q[t, h], dtype=np.float64),
-                   np.asarray(summary[b0:b0 + c, h // group], dtype=np.float64))
-        if near_tie_alternative(gpu_sel[r], ref_sel[r], sc, c, topk, tie_rel):
+        q_row = np.asarray(q[t, h], dtype=np.float64)
+        summ = np.asarray(summary[b0:b0 + c, h // group], dtype=np.float64)
+        sc = score(q_row, summ)
+        slack = slack_fn(q_row, summ) if slack_fn is not None else None
+        if near_tie_alternative(gpu_sel[r], ref_sel[r], sc, c, topk, tie_rel, slack):
             ties.add(int(r))
         else:
             bad.append((t, h, list(gpu_sel[r]), list(ref_sel[r])))

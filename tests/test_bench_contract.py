@@ -44,6 +44,8 @@ def test_reference_arm_prints_one_contract_line(args, unit, workload):
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
     if "--gate" in args:
         assert d["config"]["gate"] == "minmax"
+    if "--decode" not in args:
+        assert cb["cpu_count"] >= 1 and cb["extrapolated"] is True
 
 
 def test_reference_arm_runs_on_rank_zero_only():
@@ -52,7 +54,7 @@ def test_reference_arm_runs_on_rank_zero_only():
     assert r.returncode == 0 and r.stdout.strip() == ""
 
 
-@pytest.mark.parametrize("args", [["--warmup", "2"], ["--gate", "minmax"]], ids=["warmup_below_3", "gate_without_decode"])
+@pytest.mark.parametrize("args", [["--warmup", "2"], ["--gate", "maxmin"]], ids=["warmup_below_3", "unknown_gate"])
 def test_invalid_command_lines_are_rejected(args):
     r = _run("--impl", "reference", "--steps", "1", *args, timeout=120)
     assert r.returncode != 0 and "error" in r.stderr

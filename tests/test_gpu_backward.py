@@ -1,0 +1,124 @@
+"""GPU parity of the backward pass (moba_attn_bwd, through the C ABI) against the float64
+oracle's ``moba_backward``.
+
+The backward takes the forward's selection as fixed (the gate has no parameters and routes by
+hard top-k, so no gradient flows through it); the GPU forward's own selection is passed to both
+sides.  d_out is seeded N(0, 1) bf16, d_lse seeded N(0, 1) fp32 (or absent).
+
+Tolerance, per gradient tensor G against the oracle's R (derived from the arithmetic: P and dS
+enter the tensor-core products rounded to bf16, relative error <= 2^-9 per term, which adds up
+like a random walk to about 1e-3 of the typical magnitude; the result is rounded once more to
+bf16, 2^-9 relative; everything else is fp32):
+    max |G - R| <= 2e-2 * rms(R)    and    mean |G - R| <= 3e-3 * rms(R).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import oracle_pool as OP
+import parity as PT
+from block_sparse_long_meanpool_b200 import build, moba
+from block_sparse_long_meanpool_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+GRAD_MAX = 2e-2
+GRAD_MEAN = 3e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def library():
+    build.build()
+    moba.load_library()
+
+
+def check_grad(name, g, r):
+    g = np.asarray(g, dtype=np.float64)
+    r = np.asarray(r, dtype=np.float64)
+    rms = float(np.sqrt((r ** 2).mean()))
+    err = np.abs(g - r)
+    stats = {"grad": name, "max_abs": float(err.max()), "mean_abs": float(err.mean()), "rms_ref": rms}
+    assert stats["max_abs"] <= GRAD_MAX * rms, stats
+    assert stats["mean_abs"] <= GRAD_MEAN * rms, stats
+    return stats
+
+
+def run_case(w, with_dlse, seed, ex=None):
+    x = W.make_inputs(w, device="cuda")
+    q, k, v, cu = x["q"], x["k"], x["v"], x["cu_seqlens"]
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    out, lse, sel = moba.attn_fwd(q, k, v, cu, w.chunk_size, w.topk, return_sel=True)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(seed)
+    d_out = torch.randn((T, hq, d), generator=gen, device="cuda").to(torch.bfloat16)
+    d_lse = torch.randn((hq, T), generator=gen, device="cuda") if with_dlse else None
+    dq, dk, dv = moba.attn_bwd(q, k, v, out, lse, d_out, cu, w.chunk_size, w.topk, sel, d_lse=d_lse)
+    torch.cuda.synchronize()
+    cu_np = np.asarray(w.cu_seqlens)
+    q_np, k_np, v_np = PT.host(q), PT.host(k), PT.host(v)
+    s_np = PT.host(sel, np.int64)
+    do_np = PT.host(d_out)
+    dl_np = PT.host(d_lse) if with_dlse else None
+    if ex is None:
+        rq, rk, rv = oracle.moba_backward(q_np, k_np, v_np, cu_np, w.chunk_size, s_np, do_np, dl_np)
+    else:
+        rq, rk, rv = OP.backward_by_head(ex, q_np, k_np, v_np, cu_np, w.chunk_size, s_np, do_np, dl_np)
+    return [check_grad("dq", PT.host(dq), rq), check_grad("dk", PT.host(dk), rk),
+            check_grad("dv", PT.host(dv), rv)]
+
+
+SMALL = [
+    (W.WORKLOADS["tiny_2k"], True),
+    # ragged varlen GQA: empty and 1-token sequences, partial blocks, several key tiles
+    (W.custom("bwd_ragged_gqa", [700, 1337, 128, 1, 0, 390], 8, 2, 128, 128, 3, "k_offsets", 81), True),
+    (W.custom("bwd_ragged_gqa_no_dlse", [700, 1337, 128, 1, 0, 390], 8, 2, 128, 128, 3, "k_offsets", 81), False),
+    # odd GQA group, blocks of 3 key tiles with a partial last block
+    (W.custom("bwd_odd_group", [1500, 900], 6, 2, 128, 384, 3, "k_offsets", 82), True),
+    # MHA, d = 64, partial blocks
+    (W.custom("bwd_mha_d64", [1000, 1700], 3, 3, 64, 384, 3, "qk_offsets", 83), True),
+    # many routed blocks per row, 128-token blocks
+    (W.custom("bwd_topk8", [3000], 4, 1, 64, 128, 8, "k_offsets", 84), True),
+    # every block selected: dense causal attention
+    (W.custom("bwd_dense", [1000, 600], 4, 4, 128, 256, 8, "k_offsets", 85), True),
+    # one block longer than the sequence
+    (W.custom("bwd_single_block", [300, 77], 2, 1, 128, 512, 3, "k_offsets", 86), True),
+]
+
+
+@pytest.mark.parametrize("w,with_dlse", SMALL, ids=[w.name for w, _ in SMALL])
+def test_backward_small(w, with_dlse):
+    run_case(w, with_dlse, seed=w.seed + 1)
+
+
+@pytest.fixture(scope="module")
+def ex():
+    with OP.pool() as e:
+        yield e
+
+
+@pytest.mark.parametrize("name", ["long_32k", "scaling_8k"])
+def test_backward_full_size(name, ex):
+    """All rows and all keys of a full-size workload (the oracle split by query head)."""
+    w = W.ALL_WORKLOADS[name]
+    run_case(w, True, seed=w.seed + 2, ex=ex)
+
+
+def test_backward_gqa_8k(ex):
+    """GQA at 8K tokens: 8 q / 2 kv heads, chunk 512, top-3, all rows and keys."""
+    w = W.custom("bwd_gqa_8k", [8192], 8, 2, 128, 512, 3, "k_offsets", 87)
+    run_case(w, True, seed=88, ex=ex)
+
+
+def test_backward_is_deterministic_in_dk_dv():
+    """dK and dV are written once per key tile (no reductions across CTAs): bitwise repeatable."""
+    w = SMALL[1][0]
+    x = W.make_inputs(w, device="cuda")
+    q, k, v, cu = x["q"], x["k"], x["v"], x["cu_seqlens"]
+    out, lse, sel = moba.attn_fwd(q, k, v, cu, w.chunk_size, w.topk, return_sel=True)
+    d_out = torch.randn(out.shape, device="cuda").to(torch.bfloat16)
+    a = moba.attn_bwd(q, k, v, out, lse, d_out, cu, w.chunk_size, w.topk, sel)
+    b = moba.attn_bwd(q, k, v, out, lse, d_out, cu, w.chunk_size, w.topk, sel)
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])

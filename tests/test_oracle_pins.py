@@ -582,6 +582,27 @@ def test_minmax_score_is_the_centre_radius_contraction():
             np.testing.assert_allclose(got, want[r], rtol=1e-13, atol=1e-12)
 
 
+def test_minmax_score_is_the_positive_negative_part_contraction():
+    """max(q_i lo_i, q_i hi_i) = max(q_i, 0) hi_i + min(q_i, 0) lo_i (lo_i <= hi_i), so the
+    min/max score is the length-2d product of [q+, q-] with [kmax; kmin], whose operands are
+    the bf16 inputs themselves (torch fp64 matmul over all blocks at once; zeros included)."""
+    rng = np.random.default_rng(14)
+    k = rng.standard_normal((600, 2, 16)) * 3 + rng.standard_normal((1, 2, 16))
+    cu = np.array([0, 100, 600])
+    kmin, kmax = oracle.block_minmax(k, cu, 48)
+    q = rng.standard_normal((6, 16))
+    q[:, :4] = 0.0
+    q[0] = np.abs(q[0])   # all non-negative
+    q[1] = -np.abs(q[1])  # all non-positive
+    for g in range(2):
+        lhs = torch.cat([torch.from_numpy(np.maximum(q, 0)), torch.from_numpy(np.minimum(q, 0))], dim=1)
+        rhs = torch.cat([torch.from_numpy(kmax[:, g]), torch.from_numpy(kmin[:, g])], dim=1)
+        want = (lhs @ rhs.T).numpy()
+        for r in range(q.shape[0]):
+            got = oracle.minmax_scores_row(q[r], np.stack([kmin[:, g], kmax[:, g]], axis=1))
+            np.testing.assert_allclose(got, want[r], rtol=1e-13, atol=1e-12)
+
+
 # ---- backward: moba_backward (dq, dk, dv for the forward's selection)
 
 def _bw_case(seqlens, hq, hkv, d, chunk, topk, seed):

@@ -48,3 +48,41 @@ def test_check_selection_counts_ties_and_fails_otherwise():
     assert ties == {0}
     with pytest.raises(AssertionError):
         PT.check_selection(np.array([[2, 3, -1]]), ref, rows, q, means, cu, 800, 2, 1)
+
+
+def test_oracle_pool_pieces_equal_the_whole_oracle():
+    """The parallel checker only splits the oracle's work: every driver of oracle_pool gives the
+    oracle's own result on a small ragged GQA problem (spawned workers, as on the GPU machine)."""
+    import oracle
+    import oracle_pool as OP
+
+    rng = np.random.default_rng(5)
+    T, hq, hkv, d, chunk, topk = 420, 4, 2, 16, 64, 3
+    cu = [0, 250, 250, 420]
+    to_bf16 = lambda a: PT.from_bits((a.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16))
+    q = to_bf16(rng.standard_normal((T, hq, d)))
+    k = to_bf16(rng.standard_normal((T, hkv, d)))
+    v = to_bf16(rng.standard_normal((T, hkv, d)))
+    bits = lambda a: (a.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    ref = oracle.moba_forward(q, k, v, cu, chunk, topk)
+    rows = [(t, h) for t in range(0, T, 7) for h in range(hq)]
+    ts = np.array([t for t, _ in rows])
+    hs = np.array([h for _, h in rows])
+    sel_rows = ref["sel"][hs, ts]
+    do = rng.standard_normal((T, hq, d))
+    dl = rng.standard_normal((hq, T))
+    with OP.pool() as ex:
+        o, l = OP.dense_all_heads(ex, bits(q), bits(k), bits(v), cu, chunk, ref["sel"])
+        assert np.abs(o - ref["out"]).max() < 1e-12 and np.abs(l - ref["lse"]).max() < 1e-12
+        o2, l2 = OP.attend_rows_par(ex, rows, bits(q)[ts, hs], bits(k), bits(v), cu, chunk, sel_rows, hq // hkv)
+        assert np.abs(o2 - ref["out"][ts, hs]).max() < 1e-12
+        assert np.abs(l2 - ref["lse"][hs, ts]).max() < 1e-12
+        s2 = OP.select_rows_par(ex, rows, bits(q)[ts, hs], ref["means"], cu, chunk, topk, hq // hkv)
+        assert (s2 == sel_rows).all()
+        full = OP.select_and_compare_heads(ex, lambda h: bits(q)[:, h], ref["means"],
+                                           lambda h: ref["sel"][h].astype(np.int16), cu, chunk, topk,
+                                           hq // hkv, range(hq))
+        assert all((full[h][0] == ref["sel"][h]).all() and len(full[h][1]) == 0 for h in range(hq))
+        g = OP.backward_by_head(ex, q, k, v, cu, chunk, ref["sel"], do, dl)
+    r = oracle.moba_backward(q, k, v, cu, chunk, ref["sel"], do, dl)
+    assert all(np.abs(a - b).max() < 1e-10 for a, b in zip(g, r))
