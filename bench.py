@@ -504,6 +504,53 @@ def _e2e_pipelined(moba, w, x, fwd, steps, world):
                           "overlap the neighbouring steps' compute"}
 
 
+def run_backward(args, w, world, rank, local):
+    """--backward: one moba_attn_bwd per step (the forward runs once, outside the timing, for
+    out, lse and its selection), weak scaling like the forward."""
+    import torch
+
+    from block_sparse_long_meanpool_b200 import build as _build
+    from block_sparse_long_meanpool_b200 import moba
+    from block_sparse_long_meanpool_b200 import workloads as W
+
+    if rank == 0:
+        _build.build()
+    barrier(world)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    x = W.make_inputs(w, device=dev, seed=rank_seed(w, rank))
+    peaks = read_peaks()
+    sampler = ClockSampler(_gpu_id(dev))
+    barrier(world)
+    sampler.start()
+    rec = _sub_backward(moba, W, w, x, dev, peaks, steps=args.steps, warmup=args.warmup)
+    clocks = sampler.stop()
+    ms = max_over_ranks(rec["ms_per_step"], world)
+    if rank == 0:
+        f_sel = W.selected_block_flops(w.seqlens, w.num_q_heads, w.head_dim, w.chunk_size, w.topk)
+        alg = 2.5 * f_sel / (ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained"] if ms > 200.0 else peaks["bf16_tflops"]
+        print(json.dumps({
+            "metric": "MoBA backward tokens/s (dq, dk, dv of one attention layer, all heads)",
+            "value": job_value(w.total_tokens, world, ms), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded, generated on device)",
+            "config": {"workload": w.name, "description": w.description, "parallelism": f"dp{world}",
+                       "l2": "inputs larger than L2 (no flush)"},
+            "roofline": {"bound": "tensor", "kernel": "backward (dK/dV and dQ kernels)",
+                         "achieved": alg, "peak": peak, "unit": "TFLOP/s", "frac": alg / peak,
+                         "peak_kind": ("bf16 sustained" if ms > 200.0 else "bf16 burst") + f" ({peaks['source']})",
+                         "traffic": None,
+                         "note": rec["note"]},
+            "executed_tflops": rec["executed_tflops"],
+            "clocks": clocks,
+            "gpu_launches": 8 * args.steps,  # block table, 3 routing passes, 4 backward kernels
+            "e2e": None,
+            "cpu_baseline": None,
+        }), flush=True)
+
+
 def run_ours(args, w, world, rank, local):
     import torch
 
@@ -865,6 +912,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (moba_attn_bwd) instead of the forward")
     ap.add_argument("--decode", action="store_true",
                     help="time the decode step (workloads.DECODE_WORKLOADS) instead of the prefill")
     ap.add_argument("--gate", choices=["mean", "minmax"], default="mean",
@@ -893,6 +942,17 @@ def main():
                 dist.destroy_process_group()
         return
     w = W.ALL_WORKLOADS[args.workload]
+    if args.backward:
+        if args.impl == "reference":
+            ap.error("--backward has no reference arm")
+        world, rank, local = dist_setup()
+        try:
+            run_backward(args, w, world, rank, local)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
+        return
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))

@@ -356,7 +356,10 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constan
         bool ok = true;
         for (int i = 0; i < n_tiles; ++i) {
             const uint32_t bb = (uint32_t)(i & 1);
-            if (!wait_bar(BAR(B_SFULL + (int)bb), (uint32_t)(i >> 1) & 1u, abort_flag, status)) {
+            // the row statistics of stage i % kStages come from the gather warp: acquire them
+            // from its FULL arrival (the slot cannot turn over before this tile's PREADY)
+            if (!wait_bar(BAR(B_FULL + i % kStages), (uint32_t)(i / kStages) & 1u, abort_flag, status) ||
+                !wait_bar(BAR(B_SFULL + (int)bb), (uint32_t)(i >> 1) & 1u, abort_flag, status)) {
                 ok = false;
                 break;
             }

@@ -63,7 +63,7 @@ __host__ __device__ constexpr int pow2_at_least(int x) {
 // >= the largest N), WPT warpgroups per tile (one per 64-column slice), NGRP = NWG / WPT tile
 // groups taking tiles in turn, NB buffers per group (two when one group takes every tile).
 struct GatePlan {
-    int nc, wpt, ngrp, nb, cols;
+    int nc, wpt, ngrp, nb, cols, slice;  // slice: score columns per warpgroup (nc / wpt)
 };
 __host__ __device__ inline GatePlan gate_plan(int n_alloc, int nwg) {
     GatePlan g;
@@ -74,6 +74,7 @@ __host__ __device__ inline GatePlan gate_plan(int n_alloc, int nwg) {
     g.ngrp = nwg / g.wpt;
     g.nb = g.ngrp == 1 ? 2 : 1;
     g.cols = g.ngrp * g.nb * g.nc;
+    g.slice = g.nc / g.wpt;
     return g;
 }
 
@@ -307,8 +308,8 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
         const int r = threadIdx.x & 127;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         // this warpgroup's slice of the score columns
-        const int col_lo = part * kSliceCols;
-        const int col_hi = min(c, plan.wpt == 1 ? plan.nc : col_lo + kSliceCols);
+        const int col_lo = part * plan.slice;
+        const int col_hi = min(c, col_lo + plan.slice);
         const int xfer0 = B_XFER + grp * 3;
         bool ok = true;
         for (int ti = grp; ok && ti < ntiles; ti += plan.ngrp) {
@@ -380,12 +381,12 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
                     }
                     tc_fence_after();
                     float o[32];
-                    tmem_ld32(s_tmem + (uint32_t)((part + lvl) * kSliceCols), o);
+                    tmem_ld32(s_tmem + (uint32_t)((part + lvl) * plan.slice), o);
 #pragma unroll
                     for (int i = 0; i < KMAX && i < 16; ++i)
                         insert_ordered<KMAX>(val, idx, o[2 * i], (int)__float_as_uint(o[2 * i + 1]));
                     if constexpr (KMAX > 16) {
-                        tmem_ld32(s_tmem + (uint32_t)((part + lvl) * kSliceCols) + 32u, o);
+                        tmem_ld32(s_tmem + (uint32_t)((part + lvl) * plan.slice) + 32u, o);
 #pragma unroll
                         for (int i = 16; i < KMAX; ++i)
                             insert_ordered<KMAX>(val, idx, o[2 * (i - 16)], (int)__float_as_uint(o[2 * (i - 16) + 1]));

@@ -84,6 +84,11 @@ LENGTH_SWEEP = {
         f"1 x {m << 20} tokens, 32 q / 8 kv heads, d=128, 256 blocks of {(m << 20) // 256}, top-12")
     for m in (2, 4)
 }
+# The 1M workload's block shape (4096-token blocks, top-12, 32 q / 8 kv heads) on 128K tokens:
+# small enough for a full profiler capture of one attention launch.
+LENGTH_SWEEP["prefill_128k"] = Workload(
+    "prefill_128k", [1 << 17], 32, 8, 128, 4096, 12, "k_offsets", 1230,
+    "1 x 131072 tokens, 32 q / 8 kv heads, d=128, 32 blocks of 4096, top-12")
 # 10M tokens with the same 256 blocks and top-12 (blocks of 40,960 tokens).  A 32 q / 8 kv-head
 # layer does not fit one GPU at this length (q and out alone are 168 GB), so this is one GPU's
 # share of it when the layer is split four ways by KV-head group: 8 q / 2 kv heads.
@@ -176,12 +181,14 @@ def make_inputs(w: Workload, device="cpu", seed: Optional[int] = None):
       query rows (t, h) gets the offset of a block chosen uniformly among the
       blocks of its sequence that start at or before t.
     * ``needles``: q, k, v ~ N(0,1); 8 distinct needle blocks per sequence
-      (uniform in 1..nb-2) each get a random unit direction u per kv head, and
-      2.0 u is added to each key row of the block.  A Bernoulli(0.05) subset of
+      (uniform in 1..nb-2) each get a random unit direction u per kv head; their
+      key noise is antithetic (the second half of the block's rows are the first
+      half's draws negated) and 2.0 u is added to each key row, so the block's
+      mean key is 2u up to the bf16 rounding.  A Bernoulli(0.05) subset of
       query rows that have a needle block strictly before their own block is
       replaced by |q| (0.8 u + 0.6 w), w a random unit vector orthogonal to
-      u, for one such needle chosen uniformly: cosine 0.8 with the planted
-      direction.
+      u, for one such needle chosen uniformly: cosine 0.8 with the block's
+      mean key.
     """
     device = torch.device(device)
     gen = torch.Generator(device=device)
@@ -234,6 +241,12 @@ def make_inputs(w: Workload, device="cpu", seed: Optional[int] = None):
             dirs = dirs / dirs.norm(dim=-1, keepdim=True)
             for a, j in enumerate(needles.tolist()):
                 r0, r1 = s + j * B, min(s + (j + 1) * B, s + n)
+                # antithetic noise: the block's second half repeats the first half's draws
+                # negated, so the noise sums to zero and the block mean is exactly 2u before
+                # the final bf16 rounding (needle blocks are never a sequence's partial last
+                # block, and B is even)
+                hb = (r1 - r0) // 2
+                kf[r0 + hb:r0 + 2 * hb] = -kf[r0:r0 + hb]
                 kf[r0:r1] += 2.0 * dirs[a][None]
             pick = torch.rand((n, hq), generator=gen, device=device) < 0.05
             u = torch.rand((n, hq), generator=gen, device=device)
