@@ -158,8 +158,11 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
     const uint32_t b_base = sm_base + C::kQBytes(nq);
     const uint32_t bar0 = sm_base + C::kBars(nq, N);
     auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-    // B_XFER + 3 grp + k: a partner's list is in TMEM (k = 0: part 1 -> 0, 1: part 3 -> 2,
-    // 2: part 2 -> 0)
+    // B_XFER + 3 buf + k: a partner's list is in TMEM buffer buf (k = 0: part 1 -> 0,
+    // 1: part 3 -> 2, 2: part 2 -> 0).  One set per buffer: a writer's next arrival on the same
+    // barrier needs that buffer refilled, which needs the merger's SEMPTY arrival first, so no
+    // arrival can complete a second phase before the merger has waited for the first.  (Merges
+    // happen only with two or more warpgroups per tile, hence at most two buffers.)
     const int B_QFULL = 0, B_QEMPTY = 2, B_SFULL = 4, B_SEMPTY = 8, B_FINAL = 12, B_XFER = 13;
 
     // stage the summaries of past blocks 0..c-1 as K-major SW128 rows (rows c..N-1 are zero)
@@ -310,7 +313,6 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
         // this warpgroup's slice of the score columns
         const int col_lo = part * plan.slice;
         const int col_hi = min(c, col_lo + plan.slice);
-        const int xfer0 = B_XFER + grp * 3;
         bool ok = true;
         for (int ti = grp; ok && ti < ntiles; ti += plan.ngrp) {
             const int h = g * P.group + ti % P.group, qt = ti / P.group;
@@ -320,6 +322,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
             if (!wait_bar(BAR(B_SFULL + buf), ub & 1u, abort_flag, st)) break;
             tc_fence_after();
             const uint32_t s_tmem = tmem + lane_off + (uint32_t)(buf * plan.nc);
+            const int xfer0 = B_XFER + buf * 3;
             // lists sorted by (score descending, index ascending); inside a list columns arrive
             // in increasing order and an equal score never displaces an earlier (lower) block
             float val[KMAX], val2[KMAX];
@@ -375,7 +378,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
                     holder = false;
                     break;
                 } else if (part % (2 * lvl) == 0) {
-                    if (!wait_bar(BAR(xfer0 + (lvl == 1 ? part / 2 : 2)), (uint32_t)u & 1u, abort_flag, st)) {
+                    if (!wait_bar(BAR(xfer0 + (lvl == 1 ? part / 2 : 2)), ub & 1u, abort_flag, st)) {
                         ok = false;
                         break;
                     }

@@ -409,13 +409,16 @@ def choose_wave_tokens(T, hq, hkv, d, chunk_size, topk, batch, budget_bytes):
 
 def attn_fwd(q, k, v, cu_seqlens, chunk_size, topk, softmax_scale=None, sel=None,
              return_sel=False, wave_tokens=None, workspace=None, events=None,
-             workspace_budget=None, out=None, lse=None, max_seqlen=None, gate="mean"):
+             workspace_budget=None, out=None, lse=None, max_seqlen=None, gate="mean",
+             check_status=False):
     """MoBA causal prefill forward (moba_attn_fwd).
 
     q bf16 [T, Hq, d], k/v bf16 [T, Hkv, d], cu_seqlens int32 [batch + 1] on the device.
     sel: optional int32 [Hq, T, topk] selection to use instead of the gate.
     max_seqlen: the longest sequence's length when known on the host (0 / None: unknown).
     gate: "mean" (the paper's mean-pooled block summary) or "minmax" (the min/max summary).
+    check_status: wait for the call and raise MobaError if its device status word is not OK (a
+    bounded device wait gave up, or max_seqlen was shorter than a sequence).
     Returns (out bf16 [T, Hq, d], lse fp32 [Hq, T]) and, with return_sel, the gate's
     selection.  ``events`` may be a list of torch.cuda.Event recorded at the library's stage
     boundaries; the call's moba_run_info is returned in ``attn_fwd.last_info``.
@@ -467,6 +470,8 @@ def attn_fwd(q, k, v, cu_seqlens, chunk_size, topk, softmax_scale=None, sel=None
     attn_fwd.last_info = {"launches": info.launches, "waves": info.waves,
                           "gate_path": info.gate_path, "wave_tokens": wave_tokens,
                           "workspace_bytes": need}
+    if check_status:
+        device_status(p, workspace)
     if return_sel and sel is None:
         return out, lse, sel_out
     return out, lse

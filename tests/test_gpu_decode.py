@@ -53,58 +53,67 @@ def gpu_decode(w, q_new, k, v, cu_t, return_sel=False, gate="mean"):
     return out, lse, sel.cpu().numpy()
 
 
-def near_tie_rows(w, q_new_np, k_np, ref, gate="mean"):
-    """(b, h) rows whose last routed and first excluded past scores are within the band."""
+def decode_slack(q_row, summary_rows):
+    """Error bound of the decode min/max gate's score of each block: every term
+    max(q_i kmin_i, q_i kmax_i) is exact (bf16 x bf16 in fp32), and the kernel sums them in 4
+    accumulators of d/8 pair sums and two more adds, so a score is off by at most
+    (d/4 + 2) 2^-24 sum_i |t_i|.  (The mean gate's 1e-3 relative band would cover every row
+    here: a box over thousands of N(0, 1) keys gives scores of a few hundred that differ by a
+    few units.)  ``summary_rows`` is [n, 2, d] (min, max)."""
+    q = np.asarray(q_row, dtype=np.float64)
+    mm = np.asarray(summary_rows, dtype=np.float64)
+    terms = np.maximum(q * mm[:, 0, :], q * mm[:, 1, :])
+    return (q.shape[0] / 4 + 2) * 2.0 ** -24 * np.abs(terms).sum(axis=1)
+
+
+class _NewQuery:
+    """q[t, h] for the decode step: the new query of the sequence whose last cache row is t."""
+
+    def __init__(self, q_new, cu):
+        self.q = q_new
+        self.row_of = {int(cu[b + 1]) - 1: b for b in range(len(cu) - 1) if cu[b + 1] > cu[b]}
+        self.shape = (int(cu[-1]),) + tuple(q_new.shape[1:])
+
+    def __getitem__(self, th):
+        return self.q[self.row_of[int(th[0])], int(th[1])]
+
+
+def check_decode(w, q_new_np, k_np, v_np, sel, out, lse, ref, gate):
+    """Every (sequence, head) row: the GPU's selection is the oracle's or a valid near-tie
+    alternative of it (the band of R9 for the mean gate, the kernel's error bound for the
+    min/max gate), and its output matches the oracle's attention over the GPU's selection."""
     cu = np.asarray(w.cu_seqlens)
-    if gate == "minmax":
-        return near_tie_rows_minmax(w, q_new_np, k_np)
-    means = oracle.block_means(k_np, cu, w.chunk_size)
-    tab = oracle.block_table(cu, w.chunk_size)
-    group = w.num_q_heads // w.num_kv_heads
-    ties = set()
+    chunk, topk, hq = w.chunk_size, w.topk, w.num_q_heads
+    group = hq // w.num_kv_heads
+    if gate == "mean":
+        summary, score, slack = oracle.block_means(k_np, cu, chunk), oracle.gate_scores_row, None
+    else:
+        kmin, kmax = oracle.block_minmax(k_np, cu, chunk)
+        summary, score, slack = np.stack([kmin, kmax], axis=2), oracle.minmax_scores_row, decode_slack
+    qv = _NewQuery(q_new_np, cu)
+    rows, g_rows, o_rows = [], [], []
     for b in range(len(w.seqlens)):
         n = w.seqlens[b]
         if n == 0:
             continue
-        c = (n - 1) // w.chunk_size
-        b0 = int(tab["cu_blocks"][b])
-        for h in range(w.num_q_heads):
-            if PT._near_tie(q_new_np[b, h], means[b0:b0 + c, h // group], min(w.topk - 1, c)):
-                ties.add((b, h))
-    return ties
-
-
-def near_tie_rows_minmax(w, q_new_np, k_np):
-    """Rows whose m-th and (m+1)-th best min/max scores could swap under the kernel's fp32
-    arithmetic.  Every term max(q_i kmin_i, q_i kmax_i) is exact (bf16 x bf16), so a score is
-    off only by its fp32 sum: 4 accumulators of d/8 pair sums, then two more adds, at most
-    (d/4 + 2) * 2^-24 * sum_i |t_i|.  Two scores may swap only when their gap is below the sum
-    of their bounds.  (The mean gate's 1e-3 relative band would cover every row here: a box
-    over thousands of N(0, 1) keys gives scores of a few hundred that differ by a few units.)"""
-    cu = np.asarray(w.cu_seqlens)
-    kmin, kmax = oracle.block_minmax(k_np, cu, w.chunk_size)
-    tab = oracle.block_table(cu, w.chunk_size)
-    group = w.num_q_heads // w.num_kv_heads
-    unit = (w.head_dim / 4 + 2) * 2.0 ** -24
-    ties = set()
-    for b in range(len(w.seqlens)):
-        n = w.seqlens[b]
-        if n == 0:
-            continue
-        c = (n - 1) // w.chunk_size
-        m = min(w.topk - 1, c)
-        if m == 0 or c <= m:
-            continue
-        b0 = int(tab["cu_blocks"][b])
-        for h in range(w.num_q_heads):
-            q = q_new_np[b, h]
-            lo, hi = kmin[b0:b0 + c, h // group], kmax[b0:b0 + c, h // group]
-            terms = np.maximum(q * lo, q * hi)
-            score, bound = terms.sum(axis=1), unit * np.abs(terms).sum(axis=1)
-            order = np.argsort(-score, kind="stable")
-            x, y = order[m - 1], order[m]
-            if score[x] - score[y] <= bound[x] + bound[y]:
-                ties.add((b, h))
+        t, c = int(cu[b + 1]) - 1, (n - 1) // chunk
+        for h in range(hq):
+            # the decode selection lists the own block first and the routed blocks best first;
+            # as a prefill row: routed blocks ascending, the own block, -1 padding
+            got = [int(x) for x in sel[b, h] if x >= 0]
+            assert got[0] == c and len(got) == len(set(got)), (b, h, got)
+            g_rows.append(sorted(got[1:]) + [c] + [-1] * (topk - len(got)))
+            o_rows.append([int(x) for x in ref["sel"][b, h]])
+            rows.append((t, h))
+    # the oracle's decode selection is already in that form (select_blocks_rows)
+    g_rows, o_rows = np.array(g_rows), np.array(o_rows)
+    ties = PT.check_selection(g_rows, o_rows, rows, qv, summary, cu, chunk, topk, group, score=score,
+                              slack_fn=slack)
+    ref_o, ref_l = oracle.attend_rows(qv, k_np, v_np, cu, chunk, g_rows, rows)
+    batch_of = {t: qv.row_of[t] for t, _ in rows}
+    og = np.stack([out[batch_of[t], h] for t, h in rows])
+    lg = np.array([lse[h, batch_of[t]] for t, h in rows])
+    PT.check_out(og, lg, ref_o, ref_l)
     return ties
 
 
@@ -125,26 +134,10 @@ def test_decode_small(w, gate):
     out, lse, sel = gpu_decode(w, q_new, k, v, cu_t, return_sel=True, gate=gate)
     qn, kn, vn = PT.host(q_new), PT.host(k), PT.host(v)
     ref = oracle.moba_decode(qn, kn, vn, np.asarray(w.cu_seqlens), w.chunk_size, w.topk, gate=gate)
-    ties = near_tie_rows(w, qn, kn, ref, gate)
-    B, hq = len(w.seqlens), w.num_q_heads
-    keep = np.ones((B, hq), dtype=bool)
-    for b in range(B):
-        for h in range(hq):
-            got = sorted(int(x) for x in sel[b, h] if x >= 0)
-            want = sorted(int(x) for x in ref["sel"][b, h] if x >= 0)
-            if got != want:
-                assert (b, h) in ties, (b, h, got, want)
-                keep[b, h] = False
     o, l = PT.host(out), PT.host(lse)
-    empty = [b for b in range(B) if w.seqlens[b] == 0]
-    for b in empty:
+    for b in [b for b in range(len(w.seqlens)) if w.seqlens[b] == 0]:
         assert np.all(o[b] == 0) and np.all(np.isneginf(l[:, b]))
-    rows = [(b, h) for b in range(B) for h in range(hq) if keep[b, h] and w.seqlens[b] > 0]
-    og = np.stack([o[b, h] for b, h in rows])
-    orf = np.stack([ref["out"][b, h] for b, h in rows])
-    lg = np.array([l[h, b] for b, h in rows])
-    lr = np.array([ref["lse"][h, b] for b, h in rows])
-    PT.check_out(og, lg, orf, lr)
+    check_decode(w, qn, kn, vn, sel, o, l, ref, gate)
 
 
 def test_decode_matches_prefill_last_rows_on_gpu():
@@ -167,14 +160,10 @@ def test_decode_long_cache(gate):
     """A 256K-token cache with the 1M workload's block size and top-k (64 blocks of 4096)."""
     w = W.custom("dec_256k", [1 << 18], 8, 2, 128, 4096, 12, "k_offsets", 68)
     q_new, _, k, v, cu_t = decode_inputs(w)
-    out, lse = gpu_decode(w, q_new, k, v, cu_t, gate=gate)
+    out, lse, sel = gpu_decode(w, q_new, k, v, cu_t, return_sel=True, gate=gate)
     qn, kn, vn = PT.host(q_new), PT.host(k), PT.host(v)
     ref = oracle.moba_decode(qn, kn, vn, np.asarray(w.cu_seqlens), w.chunk_size, w.topk, gate=gate)
-    ties = near_tie_rows(w, qn, kn, ref, gate)
-    rows = [(0, h) for h in range(w.num_q_heads) if (0, h) not in ties]
-    o, l = PT.host(out), PT.host(lse)
-    PT.check_out(np.stack([o[b, h] for b, h in rows]), np.array([l[h, b] for b, h in rows]),
-                 np.stack([ref["out"][b, h] for b, h in rows]), np.array([ref["lse"][h, b] for b, h in rows]))
+    check_decode(w, qn, kn, vn, sel, PT.host(out), PT.host(lse), ref, gate)
 
 
 @pytest.mark.parametrize("w", [SMALL[0], SMALL[1], W.custom("mm_long", [1 << 17, 5000], 8, 8, 128, 4096, 4,

@@ -97,7 +97,8 @@ def test_small_all_rows(w):
     nb = moba.num_blocks(w.seqlens, chunk)
     means = moba.meanpool(k, cu_t, chunk, num_blocks_out=nb)
     sel_gate = moba.gate_topk(q, means, cu_t, chunk, topk)
-    out, lse, sel = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True, max_seqlen=w.max_seqlen)
+    out, lse, sel = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True, max_seqlen=w.max_seqlen,
+                                  check_status=True)
     torch.cuda.synchronize()
     q_np, k_np, v_np = PT.host(q), PT.host(k), PT.host(v)
     ref = oracle.moba_forward(q_np, k_np, v_np, cu, chunk, topk)
@@ -114,6 +115,44 @@ def test_small_all_rows(w):
     fed = torch.from_numpy(ref["sel"].astype(np.int32)).cuda()
     out2, lse2 = moba.attn_fwd(q, k, v, cu_t, chunk, topk, sel=fed)
     check_all_rows(out2, lse2, ref["out"], ref["lse"])
+
+
+WIDE = [
+    # 256 blocks: 256 score columns, the four warpgroups of a tile merge their lists twice
+    W.custom("wide_256_top12", [32768], 4, 1, 128, 128, 12, "k_offsets", 31),
+    # topk - 1 > 11: two warpgroups per tile, 128-column slices
+    W.custom("wide_256_top17", [32768], 2, 1, 64, 128, 17, "k_offsets", 32),
+    W.custom("wide_256_top32", [32768], 2, 1, 128, 128, 32, "k_offsets", 33),
+    # 128 blocks: two tile groups of two warpgroups each
+    W.custom("wide_128_top8", [16384, 9000], 4, 2, 128, 128, 8, "k_offsets", 34),
+]
+
+
+@pytest.mark.parametrize("w", WIDE, ids=[w.name for w in WIDE])
+def test_gate_with_merged_warpgroup_lists(w):
+    """The tensor-core gate when several warpgroups rank slices of one tile's scores and merge
+    their lists: every selection against the oracle's, then sampled outputs."""
+    q, k, v, cu_t = gpu_inputs(w)
+    cu = np.asarray(w.cu_seqlens)
+    chunk, topk, hq = w.chunk_size, w.topk, w.num_q_heads
+    group = hq // w.num_kv_heads
+    p = moba.make_params(len(w.seqlens), w.total_tokens, hq, w.num_kv_heads, w.head_dim, chunk, topk,
+                         max_seqlen=w.max_seqlen)
+    ws = torch.empty(moba.workspace_size(p), dtype=torch.uint8, device="cuda")
+    out, lse, sel = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True, max_seqlen=w.max_seqlen,
+                                  workspace=ws, wave_tokens=0)
+    assert moba.attn_fwd.last_info["gate_path"] == moba.GATE_PATH_TENSOR_CORES
+    moba.device_status(p, ws)  # no bounded wait gave up
+    q_np, k_np, v_np = PT.host(q), PT.host(k), PT.host(v)
+    om = oracle.block_means(k_np, cu, chunk)
+    osel = oracle.select_blocks(q_np, om, cu, chunk, topk)
+    gsel = PT.host(sel, np.int64)
+    ties = full_sel_check(gsel, osel, q_np, om, cu, chunk, topk, group)
+    assert len(ties) < 1e-3 * gsel.shape[0] * gsel.shape[1]
+    rows = sorted(set(PT.sample_rows(cu, chunk, hq, topk, 192, 64, seed=35)) | set(ties))
+    ref_o, ref_l = oracle.attend_rows(q_np, k_np, v_np, cu, chunk, np.stack([gsel[h, t] for t, h in rows]), rows)
+    PT.check_out(np.stack([PT.host(out[t, h]) for t, h in rows]), np.array([float(lse[h, t]) for t, h in rows]),
+                 ref_o, ref_l)
 
 
 def test_waves_give_bitwise_identical_results():
@@ -198,7 +237,8 @@ def test_full_size_all_rows(name, ex):
     group = hq // w.num_kv_heads
     nb = moba.num_blocks(w.seqlens, chunk)
     means = moba.meanpool(k, cu_t, chunk, num_blocks_out=nb)
-    out, lse, sel = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True, max_seqlen=w.max_seqlen)
+    out, lse, sel = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True, max_seqlen=w.max_seqlen,
+                                  check_status=True)
     torch.cuda.synchronize()
     q16, k16, v16 = PT.bf16_bits(q), PT.bf16_bits(k), PT.bf16_bits(v)
     q_np, k_np, v_np = PT.from_bits(q16), PT.from_bits(k16), PT.from_bits(v16)
@@ -229,7 +269,8 @@ def test_granularity_sweep_sampled(name, ex):
     group = hq // w.num_kv_heads
     nb = moba.num_blocks(w.seqlens, chunk)
     means = moba.meanpool(k, cu_t, chunk, num_blocks_out=nb)
-    out, lse, sel = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True, max_seqlen=w.max_seqlen)
+    out, lse, sel = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True, max_seqlen=w.max_seqlen,
+                                  check_status=True)
     torch.cuda.synchronize()
     q16, k16, v16 = PT.bf16_bits(q), PT.bf16_bits(k), PT.bf16_bits(v)
     q_np, k_np = PT.from_bits(q16), PT.from_bits(k16)
@@ -289,7 +330,8 @@ def _long_prefill_check(ex, w, sel_heads, n_uniform, n_strat, seed):
     chunk, topk, hq, hkv = w.chunk_size, w.topk, w.num_q_heads, w.num_kv_heads
     group = hq // hkv
     T = w.total_tokens
-    out, lse, sel = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True, max_seqlen=w.max_seqlen)
+    out, lse, sel = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True, max_seqlen=w.max_seqlen,
+                                  check_status=True)
     nb = moba.num_blocks(w.seqlens, chunk)
     means = moba.meanpool(k, cu_t, chunk, num_blocks_out=nb)
     torch.cuda.synchronize()
@@ -386,7 +428,8 @@ def test_cuda_core_gate_above_257_blocks():
     chunk, topk, group = w.chunk_size, w.topk, w.num_q_heads // w.num_kv_heads
     means = moba.meanpool(k, cu_t, chunk)
     sel = moba.gate_topk(q, means, cu_t, chunk, topk, max_seqlen=w.max_seqlen)
-    _, _, sel2 = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True, max_seqlen=w.max_seqlen)
+    _, _, sel2 = moba.attn_fwd(q, k, v, cu_t, chunk, topk, return_sel=True, max_seqlen=w.max_seqlen,
+                                  check_status=True)
     assert moba.attn_fwd.last_info["gate_path"] == moba.GATE_PATH_CUDA_CORES
     torch.cuda.synchronize()
     assert torch.equal(sel, sel2)
