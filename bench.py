@@ -202,24 +202,29 @@ def cpu_oracle_baseline(w, budget_s, seed=0, inputs=None, dense=False):
                             for i in range(len(cu) - 1)])
     t_means = time.perf_counter() - t0
     rng = np.random.default_rng(seed)
-    with OP.pool() as ex:
-        # warm the workers up (process start, imports) outside the timed parts
+    with OP.pool() as ex, OP.Shared(k=k16.transpose(1, 0, 2), v=v16.transpose(1, 0, 2)) as sh:
+        # start the workers (process start, imports) outside the measured parts
         list(ex.map(int, range(workers)))
         h = int(rng.integers(0, hq))
-        a = time.perf_counter()
-        ex.submit(OP._select_head, np.ascontiguousarray(q16[:, h]),
-                  np.ascontiguousarray(means[:, h // group]), cu, chunk, topk).result()
-        t_gate_head = time.perf_counter() - a
+        _, t_gate_head = ex.submit(OP.timed, "_select_head", np.ascontiguousarray(q16[:, h]),
+                                   np.ascontiguousarray(means[:, h // group]), cu, chunk, topk).result()
         done, cpu_rows = 0, 0.0
         wall0 = time.perf_counter()
         while time.perf_counter() - wall0 < budget_s:
-            rows = sorted({(int(rng.integers(0, T)), int(rng.integers(0, hq))) for _ in range(4 * workers)})
+            rows = sorted({(int(rng.integers(0, T)), int(rng.integers(0, hq))) for _ in range(8 * workers)})
             ts = np.array([t for t, _ in rows])
             hs = np.array([hh for _, hh in rows])
-            a = time.perf_counter()
-            sel = OP.select_rows_par(ex, rows, q16[ts, hs], means, cu, chunk, topk, group)
-            OP.attend_rows_par(ex, rows, q16[ts, hs], k16, v16, cu, chunk, sel, group)
-            cpu_rows += (time.perf_counter() - a) * workers
+            q_rows = np.ascontiguousarray(q16[ts, hs])
+            sel_futs = [ex.submit(OP.timed, "_select_rows", q_rows[part], ts[part],
+                                  np.ascontiguousarray(means[:, int(hs[part[0]]) // group]), cu, chunk, topk, False)
+                        for part in [np.nonzero(hs == hh)[0] for hh in np.unique(hs)]]
+            sel = np.zeros((len(rows), topk), dtype=np.int64)
+            for part, f in zip([np.nonzero(hs == hh)[0] for hh in np.unique(hs)], sel_futs):
+                r, c = f.result()
+                sel[part] = r
+                cpu_rows += c
+            _, _, c = OP.submit_attend_shared(ex, rows, q_rows, sh, cu, chunk, sel, group).result()
+            cpu_rows += c
             done += len(rows)
         dense_s = None
         if dense:
@@ -230,10 +235,10 @@ def cpu_oracle_baseline(w, budget_s, seed=0, inputs=None, dense=False):
                 for t in range(cu[i], cu[i + 1]):
                     c = (t - cu[i]) // chunk
                     all_sel[0, t, :c + 1] = np.arange(c + 1)
-            a = time.perf_counter()
-            ex.submit(OP._dense_head, np.ascontiguousarray(q16[:, 0]), np.ascontiguousarray(k16[:, 0]),
-                      np.ascontiguousarray(v16[:, 0]), cu, chunk, all_sel[0], None).result()
-            dense_s = (time.perf_counter() - a) * hq
+            _, c = ex.submit(OP.timed, "_dense_head", np.ascontiguousarray(q16[:, 0]),
+                             np.ascontiguousarray(k16[:, 0]), np.ascontiguousarray(v16[:, 0]), cu, chunk,
+                             all_sel[0], None).result()
+            dense_s = c * hq
     rows_all = float(T * hq)
     cpu_total = t_gate_head * hq + cpu_rows * rows_all / max(done, 1)
     seconds = t_means + cpu_total / workers
@@ -243,9 +248,10 @@ def cpu_oracle_baseline(w, budget_s, seed=0, inputs=None, dense=False):
         "gate_seconds_per_head": t_gate_head,
         "extrapolated": True,
         "sample": (f"{w.name} ({T} tokens x {hq} heads) on {workers} host processes: block means of the "
-                   f"whole input ({t_means:.1f} s), the full gate selection of one head ({t_gate_head:.1f} s, "
-                   f"x {hq} heads), {done} uniformly sampled rows' gate + attention ({cpu_rows:.0f} "
-                   f"CPU-s), extrapolated to all rows as means + CPU-seconds / processes")})
+                   f"whole input ({t_means:.1f} s), the full gate selection of one head ({t_gate_head:.1f} "
+                   f"CPU-s, x {hq} heads), {done} uniformly sampled rows' gate + attention ({cpu_rows:.1f} "
+                   f"CPU-s, measured in the workers), extrapolated to all rows as means + CPU-seconds / "
+                   f"processes")})
     if dense_s is not None:
         detail["dense_causal_fp64_tokens_per_s"] = T / (dense_s / workers)
         detail["dense_causal_fp64_note"] = ("the oracle with every block selected (dense causal attention), "

@@ -21,15 +21,13 @@
 // One CTA per (query block b, KV head g): it stages the summaries of the c past blocks of b's
 // sequence in shared memory once (SWIZZLE_128B, K-major), then runs the 128-row tiles of block
 // b for the query heads of g.  The last warp loads each Q tile by TMA (and, for the min/max
-// gate, splits it into q+ and q-) and issues the MMAs (N = c rounded up to 16) into TMEM.  Four
-// warpgroups (two for long lists; thread = row, TMEM lane) select the top-(topk-1): the
-// 64-column slices of a tile's scores are split over 1, 2 or 4 warpgroups, each keeps
-// a sorted list of its slice in registers, and the lists are merged pairwise through TMEM
-// (the merging warpgroup reads its partner's list from the columns the partner has finished
-// with, after a bounded mbarrier handshake) under the (score descending, index ascending)
-// order.  Rows with at most topk-1 past
-// blocks take all of them without scoring.  Sequences longer than 257 blocks use the fp32
-// CUDA-core gate instead (gate.cu).
+// gate, splits it into q+ and q-) and issues the MMAs (N = c rounded up to 16) into TMEM.  The
+// top-(topk-1) is chosen by warpgroups that take whole tiles in turn, each with its own TMEM
+// score buffer (four warpgroups while four buffers fit TMEM, i.e. up to 128 past blocks, and the
+// lists are short; two otherwise): thread = row = TMEM lane, a sorted (score, index) list kept in
+// registers as two interleaved lists merged at the end under the (score descending, lower index)
+// order.  Rows with at most topk-1 past blocks take all of them without scoring.  Sequences
+// longer than 257 blocks use the fp32 CUDA-core gate instead (gate.cu).
 #include <climits>
 
 #include "moba_internal.cuh"
@@ -42,13 +40,13 @@ namespace {
 using namespace ptx;
 
 constexpr int kMaxPast = 256;   // past blocks scored in one MMA (N <= 256)
-constexpr int kSliceCols = 64;  // score columns per warpgroup slice
 
-// Top-k warpgroups: four, or two when the lists are long (topk - 1 > 11), so that each
-// thread keeps its list, a 32-score load and a partner's list in registers.
-template <int KMAX>
+// Top-k warpgroups, each ranking whole tiles in its own TMEM score buffer: four when the scores
+// of a tile take at most 128 columns, two when they take 256 (TMEM holds 512 columns) or when
+// the lists are long (topk - 1 > 11, for registers).
+template <int NWG>
 struct GateWarps {
-    static constexpr int kNumWG = KMAX > 11 ? 2 : 4;
+    static constexpr int kNumWG = NWG;
     static constexpr int kThreads = kNumWG * 128 + 32;  // + the TMA / MMA warp
     static constexpr int kWarpMMA = kNumWG * 4;
 };
@@ -59,24 +57,9 @@ __host__ __device__ constexpr int pow2_at_least(int x) {
     return p;
 }
 
-// TMEM plan of one launch (the same in every CTA): NC columns per score buffer (a power of two
-// >= the largest N), WPT warpgroups per tile (one per 64-column slice), NGRP = NWG / WPT tile
-// groups taking tiles in turn, NB buffers per group (two when one group takes every tile).
-struct GatePlan {
-    int nc, wpt, ngrp, nb, cols, slice;  // slice: score columns per warpgroup (nc / wpt)
-};
-__host__ __device__ inline GatePlan gate_plan(int n_alloc, int nwg) {
-    GatePlan g;
-    g.nc = pow2_at_least(n_alloc);
-    g.wpt = g.nc / kSliceCols;
-    if (g.wpt < 1) g.wpt = 1;
-    if (g.wpt > nwg) g.wpt = nwg;
-    g.ngrp = nwg / g.wpt;
-    g.nb = g.ngrp == 1 ? 2 : 1;
-    g.cols = g.ngrp * g.nb * g.nc;
-    g.slice = g.nc / g.wpt;
-    return g;
-}
+// TMEM plan of one launch (the same in every CTA): one buffer of NC columns (a power of two
+// >= the largest N) per warpgroup.
+__host__ __device__ inline int gate_cols(int n_alloc, int nwg) { return nwg * pow2_at_least(n_alloc); }
 
 template <int D, bool MINMAX>
 struct GateCfg {
@@ -97,15 +80,15 @@ __device__ __forceinline__ void split_sign(uint32_t x, uint32_t& pos, uint32_t& 
     neg = x & m;
 }
 
-template <int D, int KMAX, bool MINMAX>
-__global__ void __launch_bounds__(GateWarps<KMAX>::kThreads, 1)
+template <int D, int KMAX, bool MINMAX, int NWG>
+__global__ void __launch_bounds__(GateWarps<NWG>::kThreads, 1)
 gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restrict__ means,
                const __nv_bfloat16* __restrict__ kmin, const __nv_bfloat16* __restrict__ kmax,
                const int* __restrict__ cu, Problem P, int* __restrict__ sel, int* status, int n_cap,
                int nq) {
     using C = GateCfg<D, MINMAX>;
-    constexpr int kThreads = GateWarps<KMAX>::kThreads;
-    constexpr int kWarpMMA = GateWarps<KMAX>::kWarpMMA;
+    constexpr int kThreads = GateWarps<NWG>::kThreads;
+    constexpr int kWarpMMA = GateWarps<NWG>::kWarpMMA;
     constexpr int kHalfBytesQ = kTileM * 128;
     constexpr bool kTwoLists = KMAX <= 16;  // a second list for instruction-level parallelism
     extern __shared__ uint8_t smem_raw[];
@@ -153,17 +136,14 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
     }
     const int N = (c + 15) & ~15;  // MMA N: past blocks rounded up to 16 (c <= n_cap)
     const int split_bytes = N * D * 2;
-    const GatePlan plan = gate_plan(n_cap, GateWarps<KMAX>::kNumWG);
+    const int nc = pow2_at_least(n_cap);  // TMEM columns of one warpgroup's score buffer
+    const int tmem_cols = gate_cols(n_cap, NWG);
     const uint32_t sm_base = smem_u32(smem);
     const uint32_t b_base = sm_base + C::kQBytes(nq);
     const uint32_t bar0 = sm_base + C::kBars(nq, N);
     auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-    // B_XFER + 3 buf + k: a partner's list is in TMEM buffer buf (k = 0: part 1 -> 0,
-    // 1: part 3 -> 2, 2: part 2 -> 0).  One set per buffer: a writer's next arrival on the same
-    // barrier needs that buffer refilled, which needs the merger's SEMPTY arrival first, so no
-    // arrival can complete a second phase before the merger has waited for the first.  (Merges
-    // happen only with two or more warpgroups per tile, hence at most two buffers.)
-    const int B_QFULL = 0, B_QEMPTY = 2, B_SFULL = 4, B_SEMPTY = 8, B_FINAL = 12, B_XFER = 13;
+    // per warpgroup w: SFULL + w (its scores are in TMEM), SEMPTY + w (it has read them)
+    const int B_QFULL = 0, B_QEMPTY = 2, B_SFULL = 4, B_SEMPTY = 8, B_FINAL = 12;
 
     // stage the summaries of past blocks 0..c-1 as K-major SW128 rows (rows c..N-1 are zero)
     {
@@ -222,17 +202,16 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
             mbar_init(BAR(B_QFULL + i), 1);
             mbar_init(BAR(B_QEMPTY + i), 1);
         }
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < NWG; ++i) {
             mbar_init(BAR(B_SFULL + i), 1);
-            mbar_init(BAR(B_SEMPTY + i), 128 * plan.wpt);
+            mbar_init(BAR(B_SEMPTY + i), 128);
         }
         mbar_init(BAR(B_FINAL), 1);
-        for (int i = 0; i < 6; ++i) mbar_init(BAR(B_XFER + i), 128);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == kWarpMMA) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                         smem_u32(&s_tmem)), "r"(plan.cols));
+                         smem_u32(&s_tmem)), "r"(tmem_cols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     tc_fence_before();
@@ -277,13 +256,13 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
                 fence_proxy_async();
                 __syncwarp();
             }
-            const int grp = ti % plan.ngrp, u = ti / plan.ngrp;
-            const int buf = grp * plan.nb + u % plan.nb;
-            const uint32_t ub = (uint32_t)(u / plan.nb);
-            if (ub >= 1 && !wait_bar(BAR(B_SEMPTY + buf), (ub - 1u) & 1u, abort_flag, st)) break;
+            // tile ti goes to warpgroup ti % NWG (its u-th tile), into that warpgroup's buffer
+            const int buf = ti % NWG;
+            const uint32_t u = (uint32_t)(ti / NWG);
+            if (u >= 1 && !wait_bar(BAR(B_SEMPTY + buf), (u - 1u) & 1u, abort_flag, st)) break;
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t s_tmem = tmem + (uint32_t)(buf * plan.nc);
+                const uint32_t s_tmem = tmem + (uint32_t)(buf * nc);
 #pragma unroll
                 for (int p = 0; p < C::kPairs; ++p) {
                     const uint32_t abase = qbase + (uint32_t)(MINMAX ? p : 0) * C::kTile;
@@ -305,24 +284,16 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
         __syncwarp();
         drain_bar(BAR(B_FINAL), 0);
     } else {
-        // ---------------- top-k: warpgroup wg, thread = row ----------------
+        // ---------------- top-k: warpgroup wg takes tiles wg, wg + NWG, ...; thread = row ----------------
         const int wg = warp >> 2;
-        const int grp = wg / plan.wpt, part = wg % plan.wpt;
         const int r = threadIdx.x & 127;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        // this warpgroup's slice of the score columns
-        const int col_lo = part * plan.slice;
-        const int col_hi = min(c, col_lo + plan.slice);
-        bool ok = true;
-        for (int ti = grp; ok && ti < ntiles; ti += plan.ngrp) {
+        const uint32_t s_tmem = tmem + lane_off + (uint32_t)(wg * nc);
+        for (int ti = wg; ti < ntiles; ti += NWG) {
             const int h = g * P.group + ti % P.group, qt = ti / P.group;
-            const int u = ti / plan.ngrp;
-            const int buf = grp * plan.nb + u % plan.nb;
-            const uint32_t ub = (uint32_t)(u / plan.nb);
-            if (!wait_bar(BAR(B_SFULL + buf), ub & 1u, abort_flag, st)) break;
+            const uint32_t u = (uint32_t)(ti / NWG);
+            if (!wait_bar(BAR(B_SFULL + wg), u & 1u, abort_flag, st)) break;
             tc_fence_after();
-            const uint32_t s_tmem = tmem + lane_off + (uint32_t)(buf * plan.nc);
-            const int xfer0 = B_XFER + buf * 3;
             // lists sorted by (score descending, index ascending); inside a list columns arrive
             // in increasing order and an equal score never displaces an earlier (lower) block
             float val[KMAX], val2[KMAX];
@@ -332,75 +303,28 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
                 val[i] = val2[i] = -INFINITY;
                 idx[i] = idx2[i] = INT_MAX;
             }
-            for (int j0 = col_lo; j0 < col_hi; j0 += 32) {
+            for (int j0 = 0; j0 < c; j0 += 32) {
                 float v[32];
                 tmem_ld32(s_tmem + (uint32_t)j0, v);
                 if constexpr (kTwoLists) {
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
-                        insert_desc<KMAX>(val, idx, v[e], j0 + e, j0 + e < col_hi);
-                        insert_desc<KMAX>(val2, idx2, v[e + 1], j0 + e + 1, j0 + e + 1 < col_hi);
+                        insert_desc<KMAX>(val, idx, v[e], j0 + e, j0 + e < c);
+                        insert_desc<KMAX>(val2, idx2, v[e + 1], j0 + e + 1, j0 + e + 1 < c);
                     }
                 } else {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) insert_desc<KMAX>(val, idx, v[e], j0 + e, j0 + e < col_hi);
+                    for (int e = 0; e < 32; ++e) insert_desc<KMAX>(val, idx, v[e], j0 + e, j0 + e < c);
                 }
             }
             if constexpr (kTwoLists) {
 #pragma unroll
                 for (int i = 0; i < KMAX; ++i) insert_ordered<KMAX>(val, idx, val2[i], idx2[i]);
             }
-            // merge the slices of the tile pairwise through TMEM: level 1 (parts 1 -> 0, 3 -> 2),
-            // level 2 (part 2 -> 0); a list goes over the columns its writer has read
-            bool holder = true;
-            for (int lvl = 1; lvl < plan.wpt; lvl <<= 1) {
-                if (part % (2 * lvl) == lvl) {
-                    uint32_t w[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) w[i] = 0u;
-#pragma unroll
-                    for (int i = 0; i < KMAX && i < 16; ++i) {
-                        w[2 * i] = __float_as_uint(val[i]);
-                        w[2 * i + 1] = (uint32_t)idx[i];
-                    }
-                    tmem_st32(s_tmem + (uint32_t)col_lo, w);
-                    if constexpr (KMAX > 16) {
-#pragma unroll
-                        for (int i = 16; i < KMAX; ++i) {
-                            w[2 * (i - 16)] = __float_as_uint(val[i]);
-                            w[2 * (i - 16) + 1] = (uint32_t)idx[i];
-                        }
-                        tmem_st32(s_tmem + (uint32_t)col_lo + 32u, w);
-                    }
-                    tmem_st_wait();
-                    tc_fence_before();
-                    mbar_arrive(BAR(xfer0 + (lvl == 1 ? part / 2 : 2)));
-                    holder = false;
-                    break;
-                } else if (part % (2 * lvl) == 0) {
-                    if (!wait_bar(BAR(xfer0 + (lvl == 1 ? part / 2 : 2)), ub & 1u, abort_flag, st)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    float o[32];
-                    tmem_ld32(s_tmem + (uint32_t)((part + lvl) * plan.slice), o);
-#pragma unroll
-                    for (int i = 0; i < KMAX && i < 16; ++i)
-                        insert_ordered<KMAX>(val, idx, o[2 * i], (int)__float_as_uint(o[2 * i + 1]));
-                    if constexpr (KMAX > 16) {
-                        tmem_ld32(s_tmem + (uint32_t)((part + lvl) * plan.slice) + 32u, o);
-#pragma unroll
-                        for (int i = 16; i < KMAX; ++i)
-                            insert_ordered<KMAX>(val, idx, o[2 * (i - 16)], (int)__float_as_uint(o[2 * (i - 16) + 1]));
-                    }
-                }
-            }
-            if (!ok) break;
             tc_fence_before();
-            mbar_arrive(BAR(B_SEMPTY + buf));
+            mbar_arrive(BAR(B_SEMPTY + wg));
             const int rr = qt * kTileM + r;
-            if (holder && rr < len) {
+            if (rr < len) {
                 int o[KMAX];
 #pragma unroll
                 for (int i = 0; i < KMAX; ++i) o[i] = (i < n_route) ? idx[i] : INT_MAX;
@@ -429,7 +353,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
     __syncthreads();
     tc_fence_after();
     if (warp == kWarpMMA) {
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(plan.cols));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tmem_cols));
     }
 }
 
@@ -451,6 +375,23 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+template <int D, int KMAX, bool MINMAX, int NWG>
+cudaError_t launch_tc_w(const Problem& P, const CUtensorMap& mq, const GateSummary& s, const int* cu,
+                        int* sel, int* status, int n_max, cudaStream_t st) {
+    using C = GateCfg<D, MINMAX>;
+    // two Q buffers when they fit next to the summaries, else one
+    const int limit = 227 * 1024;
+    const int nq = C::kBytes(2, n_max) <= limit ? 2 : 1;
+    const int smem = C::kBytes(nq, n_max);
+    cudaError_t e = cudaFuncSetAttribute(gate_tc_kernel<D, KMAX, MINMAX, NWG>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(P.nb_cap, P.hkv);
+    gate_tc_kernel<D, KMAX, MINMAX, NWG><<<grid, GateWarps<NWG>::kThreads, smem, st>>>(
+        mq, s.means, s.kmin, s.kmax, cu, P, sel, status, n_max, nq);
+    return cudaGetLastError();
+}
+
 template <int D, int KMAX, bool MINMAX>
 cudaError_t launch_tc(const Problem& P, const __nv_bfloat16* q, const GateSummary& s, const int* cu,
                       int* sel, int* status, int n_max, cudaStream_t st) {
@@ -465,18 +406,12 @@ cudaError_t launch_tc(const Problem& P, const __nv_bfloat16* q, const GateSummar
            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    using C = GateCfg<D, MINMAX>;
-    // two Q buffers when they fit next to the summaries, else one
-    const int limit = 227 * 1024;
-    const int nq = C::kBytes(2, n_max) <= limit ? 2 : 1;
-    const int smem = C::kBytes(nq, n_max);
-    cudaError_t e = cudaFuncSetAttribute(gate_tc_kernel<D, KMAX, MINMAX>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    dim3 grid(P.nb_cap, P.hkv);
-    gate_tc_kernel<D, KMAX, MINMAX><<<grid, GateWarps<KMAX>::kThreads, smem, st>>>(mq, s.means, s.kmin, s.kmax, cu, P, sel,
-                                                                   status, n_max, nq);
-    return cudaGetLastError();
+    // four warpgroups while four score buffers fit TMEM and the lists are short, else two
+    if constexpr (KMAX <= 11) {
+        if (pow2_at_least(n_max) <= 128)
+            return launch_tc_w<D, KMAX, MINMAX, 4>(P, mq, s, cu, sel, status, n_max, st);
+    }
+    return launch_tc_w<D, KMAX, MINMAX, 2>(P, mq, s, cu, sel, status, n_max, st);
 }
 
 template <int D, bool MINMAX>

@@ -45,6 +45,45 @@ def pool():
                                initializer=_init_worker)
 
 
+class Shared:
+    """Large read-only inputs shared with the workers through .npy files in shared memory
+    (/dev/shm when it has room, else the temporary directory), which each worker memory-maps
+    once, instead of pickling them into every task.  Use as a context manager; ``ref(name)``
+    is what a task receives."""
+
+    def __init__(self, **arrays):
+        import shutil
+        import tempfile
+        need = sum(a.nbytes for a in arrays.values()) + (1 << 30)
+        base = "/dev/shm" if os.path.isdir("/dev/shm") and shutil.disk_usage("/dev/shm").free > need else None
+        self.dir = tempfile.mkdtemp(prefix="moba_oracle_", dir=base)
+        self.paths = {}
+        for name, a in arrays.items():
+            path = os.path.join(self.dir, name + ".npy")
+            np.save(path, np.ascontiguousarray(a))
+            self.paths[name] = path
+
+    def ref(self, name):
+        return self.paths[name]
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        import shutil
+        shutil.rmtree(self.dir, ignore_errors=True)
+
+
+_maps = {}
+
+
+def _mapped(path):
+    """The memory-mapped array at path (opened once per worker process)."""
+    if path not in _maps:
+        _maps[path] = np.load(path, mmap_mode="r")
+    return _maps[path]
+
+
 # ---- worker tasks (top level, so that they pickle) ------------------------------------------
 
 def _dense_head(q16, k16, v16, cu, chunk, sel_h, scale):
@@ -96,6 +135,43 @@ def _attend(q_rows16, ts, k16, v16, cu, chunk, sel_rows, scale):
     v = PT.from_bits(v16)[:, None, :]
     return oracle.attend_rows(_RowsView(q_rows16, ts), k, v, cu, chunk, sel_rows,
                               [(int(t), i) for i, t in enumerate(ts)], scale)
+
+
+def _attend_shared(q_rows16, ts, kpath, vpath, g, cu, chunk, sel_rows, scale):
+    """As _attend, with KV head g of the shared head-major keys and values, read row by row
+    from the memory map.  Returns (out, lse, CPU seconds of the task)."""
+    import time
+    c0 = time.process_time()
+    o, l = oracle.attend_rows(_RowsView(q_rows16, ts), _HeadRows(kpath, g), _HeadRows(vpath, g), cu, chunk,
+                              sel_rows, [(int(t), i) for i, t in enumerate(ts)], scale)
+    return o, l, time.process_time() - c0
+
+
+class _HeadRows:
+    """k[u, 0] stand-in for oracle.attend_rows over one head of a shared head-major bf16-bits
+    file: the rows u are read from the memory map and widened exactly when asked for."""
+
+    def __init__(self, path, g):
+        self.rows = _mapped(path)[g]
+        self.shape = (self.rows.shape[0], 1, self.rows.shape[1])
+
+    def __getitem__(self, idx):
+        u, g = idx
+        assert g == 0
+        return PT.from_bits(self.rows[np.asarray(u)])
+
+
+def _select_compare_shared(qpath, h, means_g, gsel_h, cu, chunk, topk):
+    """oracle.select_blocks for query head h of the shared head-major q, then the comparison
+    with the GPU's selection of that head (as _compare_head).  Returns (oracle selection int16,
+    near-tie tokens, other differing rows, CPU seconds)."""
+    import time
+    c0 = time.process_time()
+    q16 = np.asarray(_mapped(qpath)[h])
+    osel = _select_head(q16, means_g, cu, chunk, topk)
+    ties, bad = (np.zeros(0, dtype=np.int64), []) if gsel_h is None else \
+        _compare_head(gsel_h, osel, q16, means_g, cu, chunk, topk)
+    return osel, ties, bad, time.process_time() - c0
 
 
 def _backward_head(q_h, k_g, v_g, cu, chunk, sel_h, dout_h, dlse_h, scale):
@@ -225,3 +301,71 @@ def backward_by_head(ex, q, k, v, cu, chunk, sel, d_out, d_lse=None, scale=None)
         dk[:, h // group] += b
         dv[:, h // group] += c
     return dq, dk, dv
+
+
+class Pending:
+    """Futures submitted to the pool and the function that assembles their results."""
+
+    def __init__(self, futs, finish):
+        self.futs, self.finish = futs, finish
+
+    def result(self):
+        return self.finish([f.result() for f in self.futs])
+
+
+def submit_attend_shared(ex, rows, q_row16, shared, cu, chunk, sel_rows, group, scale=None):
+    """oracle.attend_rows over the (t, h) rows with the keys and values of ``shared`` ("k",
+    "v": head-major [Hkv, T, d] bf16 bits), in tasks of one KV head, about four per worker.
+    ``.result()`` gives (out [n, d], lse [n], CPU seconds of all tasks)."""
+    n = len(rows)
+    per_task = max(32, math.ceil(n / (4 * n_workers())))
+    g_of = np.array([h // group for _, h in rows], dtype=np.int64)
+    ts = np.array([t for t, _ in rows], dtype=np.int64)
+    parts, futs = [], []
+    for g in np.unique(g_of):
+        idx = np.nonzero(g_of == g)[0]
+        for part in np.array_split(idx, max(1, math.ceil(len(idx) / per_task))):
+            parts.append(part)
+            futs.append(ex.submit(_attend_shared, q_row16[part], ts[part], shared.ref("k"), shared.ref("v"),
+                                  int(g), cu, chunk, sel_rows[part], scale))
+
+    def finish(res):
+        out = np.zeros((n, q_row16.shape[1]))
+        lse = np.zeros(n)
+        cpu = 0.0
+        for part, (o, l, c) in zip(parts, res):
+            out[part], lse[part] = o, l
+            cpu += c
+        return out, lse, cpu
+
+    return Pending(futs, finish)
+
+
+def submit_select_compare_shared(ex, shared, means, gsel, cu, chunk, topk, group, heads):
+    """oracle.select_blocks for each listed query head of ``shared`` ("q": head-major
+    [Hq, T, d] bf16 bits) against its KV head's summary, compared with gsel(h) (the GPU's
+    selection of the head, or None to skip the comparison).  ``.result()`` gives
+    {h: (oracle selection int16 [T, topk], near-tie tokens)} and fails on any row that is not a
+    valid near-tie alternative."""
+    heads = list(heads)
+    futs = [ex.submit(_select_compare_shared, shared.ref("q"), int(h), np.ascontiguousarray(means[:, h // group]),
+                      gsel(h), cu, chunk, topk) for h in heads]
+
+    def finish(res):
+        out, bad = {}, []
+        for h, (osel, ties, b, _) in zip(heads, res):
+            bad += [(h,) + x for x in b]
+            out[h] = (osel, ties)
+        assert not bad, f"{len(bad)} selection mismatches outside the near-tie band: {bad[:5]}"
+        return out
+
+    return Pending(futs, finish)
+
+
+def timed(name, *args):
+    """Runs the task ``name`` of this module in the worker and returns (its result, the CPU
+    seconds it took)."""
+    import time
+    c0 = time.process_time()
+    r = globals()[name](*args)
+    return r, time.process_time() - c0

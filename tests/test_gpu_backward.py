@@ -51,7 +51,9 @@ def check_grad(name, g, r):
     return stats
 
 
-def run_case(w, with_dlse, seed, ex=None):
+def run_case(w, with_dlse, seed, ex=None, heads=None):
+    """heads: check only these query heads (MHA: their KV heads' gradients come from them
+    alone), with the oracle on those heads only."""
     x = W.make_inputs(w, device="cuda")
     q, k, v, cu = x["q"], x["k"], x["v"], x["cu_seqlens"]
     T, hq, d = q.shape
@@ -68,12 +70,19 @@ def run_case(w, with_dlse, seed, ex=None):
     s_np = PT.host(sel, np.int64)
     do_np = PT.host(d_out)
     dl_np = PT.host(d_lse) if with_dlse else None
+    gq, gk, gv = PT.host(dq), PT.host(dk), PT.host(dv)
+    if heads is not None:
+        assert hq == hkv  # MHA: head h's KV gradients are its own
+        q_np, k_np, v_np, do_np = q_np[:, heads], k_np[:, heads], v_np[:, heads], do_np[:, heads]
+        s_np = s_np[heads]
+        dl_np = dl_np[heads] if dl_np is not None else None
+        gq, gk, gv = gq[:, heads], gk[:, heads], gv[:, heads]
     if ex is None:
         rq, rk, rv = oracle.moba_backward(q_np, k_np, v_np, cu_np, w.chunk_size, s_np, do_np, dl_np)
     else:
         rq, rk, rv = OP.backward_by_head(ex, q_np, k_np, v_np, cu_np, w.chunk_size, s_np, do_np, dl_np)
     res, errs = [], []
-    for name, g, r in (("dv", PT.host(dv), rv), ("dk", PT.host(dk), rk), ("dq", PT.host(dq), rq)):
+    for name, g, r in (("dv", gv, rv), ("dk", gk, rk), ("dq", gq, rq)):
         try:
             res.append(check_grad(name, g, r))
         except AssertionError as e:
@@ -111,11 +120,18 @@ def ex():
         yield e
 
 
-@pytest.mark.parametrize("name", ["long_32k", "scaling_8k"])
-def test_backward_full_size(name, ex):
-    """All rows and all keys of a full-size workload (the oracle split by query head)."""
-    w = W.ALL_WORKLOADS[name]
+def test_backward_scaling_8k(ex):
+    """All rows and all keys of scaling_8k (2 x 8192 tokens, 16 heads; the oracle split by query
+    head)."""
+    w = W.ALL_WORKLOADS["scaling_8k"]
     run_case(w, True, seed=w.seed + 2, ex=ex)
+
+
+def test_backward_long_32k(ex):
+    """long_32k (32K tokens, 32 heads MHA, 64 blocks of 512, top-3, needles): every row and every
+    key of four heads (one per quarter of the heads); the GPU computes all 32."""
+    w = W.ALL_WORKLOADS["long_32k"]
+    run_case(w, True, seed=w.seed + 2, ex=ex, heads=[0, 11, 22, 31])
 
 
 def test_backward_gqa_8k(ex):
@@ -124,8 +140,10 @@ def test_backward_gqa_8k(ex):
     run_case(w, True, seed=88, ex=ex)
 
 
-def test_backward_is_deterministic_in_dk_dv():
-    """dK and dV are written once per key tile (no reductions across CTAs): bitwise repeatable."""
+def test_backward_repeats_up_to_summation_order():
+    """Two backward calls agree to within the order of their fp32 additions: dK and dV are
+    written once per key tile, but the routing lists (and so the order in which a tile's rows
+    are added) are filled by atomics, and dq is summed by reductions."""
     w = SMALL[1][0]
     x = W.make_inputs(w, device="cuda")
     q, k, v, cu = x["q"], x["k"], x["v"], x["cu_seqlens"]
@@ -133,4 +151,6 @@ def test_backward_is_deterministic_in_dk_dv():
     d_out = torch.randn(out.shape, device="cuda").to(torch.bfloat16)
     a = moba.attn_bwd(q, k, v, out, lse, d_out, cu, w.chunk_size, w.topk, sel)
     b = moba.attn_bwd(q, k, v, out, lse, d_out, cu, w.chunk_size, w.topk, sel)
-    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+    for x_, y_ in zip(a, b):
+        diff = (x_.float() - y_.float()).abs().max().item()
+        assert diff <= 2 ** -7 * x_.float().abs().max().item(), diff

@@ -86,3 +86,31 @@ def test_oracle_pool_pieces_equal_the_whole_oracle():
         g = OP.backward_by_head(ex, q, k, v, cu, chunk, ref["sel"], do, dl)
     r = oracle.moba_backward(q, k, v, cu, chunk, ref["sel"], do, dl)
     assert all(np.abs(a - b).max() < 1e-10 for a, b in zip(g, r))
+
+
+def test_shared_input_drivers_equal_the_whole_oracle():
+    """The drivers that read the inputs from shared-memory files give the oracle's result."""
+    import oracle
+    import oracle_pool as OP
+
+    rng = np.random.default_rng(6)
+    T, hq, hkv, d, chunk, topk = 300, 4, 2, 16, 32, 3
+    cu = [0, 300]
+    bits = lambda a: (a.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    q16 = bits(rng.standard_normal((T, hq, d)))
+    k16 = bits(rng.standard_normal((T, hkv, d)))
+    v16 = bits(rng.standard_normal((T, hkv, d)))
+    q, k, v = PT.from_bits(q16), PT.from_bits(k16), PT.from_bits(v16)
+    ref = oracle.moba_forward(q, k, v, cu, chunk, topk)
+    rows = [(t, h) for t in range(0, T, 5) for h in range(hq)]
+    ts = np.array([t for t, _ in rows])
+    hs = np.array([h for _, h in rows])
+    with OP.pool() as ex, OP.Shared(q=q16.transpose(1, 0, 2), k=k16.transpose(1, 0, 2),
+                                    v=v16.transpose(1, 0, 2)) as sh:
+        o, l, cpu = OP.submit_attend_shared(ex, rows, q16[ts, hs], sh, cu, chunk, ref["sel"][hs, ts],
+                                            hq // hkv).result()
+        assert np.abs(o - ref["out"][ts, hs]).max() < 1e-12 and np.abs(l - ref["lse"][hs, ts]).max() < 1e-12
+        assert cpu > 0
+        full = OP.submit_select_compare_shared(ex, sh, ref["means"], lambda h: ref["sel"][h].astype(np.int16),
+                                               cu, chunk, topk, hq // hkv, range(hq)).result()
+        assert all((full[h][0] == ref["sel"][h]).all() and len(full[h][1]) == 0 for h in range(hq))
