@@ -551,7 +551,7 @@ def run_backward(args, w, world, rank, local):
                          "note": rec["note"]},
             "executed_tflops": rec["executed_tflops"],
             "clocks": clocks,
-            "gpu_launches": 8 * args.steps,  # block table, 3 routing passes, 4 backward kernels
+            "gpu_launches": 9 * args.steps,  # block table, 4 routing kernels, 4 backward kernels
             "e2e": None,
             "cpu_baseline": None,
         }), flush=True)

@@ -24,10 +24,13 @@
 // gate, splits it into q+ and q-) and issues the MMAs (N = c rounded up to 16) into TMEM.  The
 // top-(topk-1) is chosen by warpgroups that take whole tiles in turn, each with its own TMEM
 // score buffer (four warpgroups while four buffers fit TMEM, i.e. up to 128 past blocks, and the
-// lists are short; two otherwise): thread = row = TMEM lane, a sorted (score, index) list kept in
-// registers as two interleaved lists merged at the end under the (score descending, lower index)
-// order.  Rows with at most topk-1 past blocks take all of them without scoring.  Sequences
-// longer than 257 blocks use the fp32 CUDA-core gate instead (gate.cu).
+// lists are short; two otherwise), thread = row = TMEM lane, in two passes over the row's
+// scores: the first keeps the topk-1 largest values (a min/max merge network, no indices), the
+// second marks the blocks scoring at least the smallest of them; when equal scores at the cut
+// mark too many, the highest such blocks are dropped, so ties keep the lower block index.  The
+// result is the exact top-k under the (score descending, lower index) order.  Rows with at
+// most topk-1 past blocks take all of them without scoring.  Sequences longer than 257 blocks
+// use the fp32 CUDA-core gate instead (gate.cu).
 #include <climits>
 
 #include "moba_internal.cuh"
@@ -40,10 +43,26 @@ namespace {
 using namespace ptx;
 
 constexpr int kMaxPast = 256;   // past blocks scored in one MMA (N <= 256)
+constexpr int kWords = kMaxPast / 32;  // a row's past blocks as a bit mask
+constexpr int kMaxQBuf = 4;            // Q tile buffers (loads run ahead of the MMAs)
+
+// The K largest values seen so far, descending (-inf until K were seen).  Adding a pair is a
+// merge with the sorted two-element list (a, b), a >= b: the i-th largest of the union is
+// max(val[i], min(val[i-1], a), min(val[i-2], b)) with val[-1] = val[-2] = +inf.  Each position
+// takes two mins and a three-input max of old values, so the K positions are independent and
+// an insertion has no compares, selects or branches.
+template <int K>
+__device__ __forceinline__ void top_values_pair(float (&val)[K], float x0, float x1) {
+    const float a = fmaxf(x0, x1), b = fminf(x0, x1);
+#pragma unroll
+    for (int i = K - 1; i >= 2; --i) val[i] = fmax3(val[i], fminf(val[i - 1], a), fminf(val[i - 2], b));
+    if constexpr (K >= 2) val[1] = fmax3(val[1], fminf(val[0], a), b);
+    val[0] = fmaxf(val[0], a);
+}
 
 // Top-k warpgroups, each ranking whole tiles in its own TMEM score buffer: four when the scores
 // of a tile take at most 128 columns, two when they take 256 (TMEM holds 512 columns) or when
-// the lists are long (topk - 1 > 11, for registers).
+// the lists are long (topk - 1 > 16, for registers).
 template <int NWG>
 struct GateWarps {
     static constexpr int kNumWG = NWG;
@@ -85,12 +104,11 @@ __global__ void __launch_bounds__(GateWarps<NWG>::kThreads, 1)
 gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restrict__ means,
                const __nv_bfloat16* __restrict__ kmin, const __nv_bfloat16* __restrict__ kmax,
                const int* __restrict__ cu, Problem P, int* __restrict__ sel, int* status, int n_cap,
-               int nq) {
+               int smem_bytes) {
     using C = GateCfg<D, MINMAX>;
     constexpr int kThreads = GateWarps<NWG>::kThreads;
     constexpr int kWarpMMA = GateWarps<NWG>::kWarpMMA;
     constexpr int kHalfBytesQ = kTileM * 128;
-    constexpr bool kTwoLists = KMAX <= 16;  // a second list for instruction-level parallelism
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
@@ -119,8 +137,9 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
     const int qtiles = (len + kTileM - 1) / kTileM;
     const int ntiles = qtiles * P.group;
 
-    if (n_route == c || c > n_cap) {
-        // nothing to choose: every past block is routed (c <= topk - 1).  c > n_cap means the
+    if (n_route == c || n_route == 0 || c > n_cap) {
+        // nothing to choose: every past block is routed (c <= topk - 1), or none (topk = 1).
+        // c > n_cap means the
         // sequence is longer than the caller's max_seqlen promised: its rows keep the own block
         // only and the call's status word (when there is one) records the broken promise.
         const bool broken = c > n_cap;
@@ -129,7 +148,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
             const int h = g * P.group + e / len;
             const int t = start + e % len;
             int* dst = sel + ((size_t)h * P.T + t) * P.topk;
-            const int nr = broken ? 0 : c;
+            const int nr = broken ? 0 : n_route;
             for (int i = 0; i < P.topk; ++i) dst[i] = (i < nr) ? i : (i == nr ? c : -1);
         }
         return;
@@ -138,12 +157,18 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
     const int split_bytes = N * D * 2;
     const int nc = pow2_at_least(n_cap);  // TMEM columns of one warpgroup's score buffer
     const int tmem_cols = gate_cols(n_cap, NWG);
+    // Q buffers: as many as the launch's shared memory holds next to this CTA's summaries (at
+    // most kMaxQBuf), so the Q loads run up to nq - 1 tiles ahead of the MMAs
+    int nq = kMaxQBuf;
+    while (nq > 1 && C::kBytes(nq, N) > smem_bytes) --nq;
     const uint32_t sm_base = smem_u32(smem);
     const uint32_t b_base = sm_base + C::kQBytes(nq);
     const uint32_t bar0 = sm_base + C::kBars(nq, N);
     auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-    // per warpgroup w: SFULL + w (its scores are in TMEM), SEMPTY + w (it has read them)
-    const int B_QFULL = 0, B_QEMPTY = 2, B_SFULL = 4, B_SEMPTY = 8, B_FINAL = 12;
+    // per Q buffer: QFULL (loaded), QEMPTY (its MMAs are done); per warpgroup w: SFULL + w (its
+    // scores are in TMEM), SEMPTY + w (it has read them)
+    const int B_QFULL = 0, B_QEMPTY = kMaxQBuf, B_SFULL = 2 * kMaxQBuf, B_SEMPTY = B_SFULL + 4,
+              B_FINAL = B_SEMPTY + 4;
 
     // stage the summaries of past blocks 0..c-1 as K-major SW128 rows (rows c..N-1 are zero)
     {
@@ -198,7 +223,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
     }
     fence_proxy_async();  // the MMAs read these shared-memory writes through the async proxy
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kMaxQBuf; ++i) {
             mbar_init(BAR(B_QFULL + i), 1);
             mbar_init(BAR(B_QEMPTY + i), 1);
         }
@@ -225,11 +250,10 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
     if (warp == kWarpMMA) {
         // ---------------- Q tiles (TMA), q+ / q- split, MMA issue ----------------
         const uint32_t idesc = idesc_bf16(N, false);
-        for (int ti = 0; ti < ntiles; ++ti) {
+        // tile ti is loaded into buffer ti % nq (its (ti / nq)-th use)
+        auto load_q = [&](int ti) {
             const int h = g * P.group + ti % P.group, qt = ti / P.group;
             const int qb = ti % nq;
-            const uint32_t uq = (uint32_t)(ti / nq);
-            if (ti >= nq && !wait_bar(BAR(B_QEMPTY + qb), (uq - 1u) & 1u, abort_flag, st)) break;
             const uint32_t qbase = sm_base + (uint32_t)qb * C::kARegions * C::kTile;
             if (lane == 0) {
                 mbar_arrive_tx(BAR(B_QFULL + qb), (uint32_t)C::kTile);
@@ -239,7 +263,15 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
                                 start + qt * kTileM);
             }
             __syncwarp();
+        };
+        int next_load = min(nq, ntiles), consumed = 0;
+        for (int ti = 0; ti < next_load; ++ti) load_q(ti);
+        for (int ti = 0; ti < ntiles; ++ti) {
+            const int qb = ti % nq;
+            const uint32_t uq = (uint32_t)(ti / nq);
+            const uint32_t qbase = sm_base + (uint32_t)qb * C::kARegions * C::kTile;
             if (!wait_bar(BAR(B_QFULL + qb), uq & 1u, abort_flag, st)) break;
+            consumed = ti + 1;
             if constexpr (MINMAX) {
                 uint4* qp = reinterpret_cast<uint4*>(smem + (size_t)qb * C::kARegions * C::kTile);
                 uint4* qm = qp + C::kTile / 16;
@@ -279,7 +311,18 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
                 mma_commit(BAR(B_QEMPTY + qb));
             }
             __syncwarp();
+            // refill: tile next_load goes where tile next_load - nq was, once that tile's MMAs
+            // are complete.  With several buffers that tile was issued before this one (so its
+            // MMAs are done or nearly), which keeps the tensor pipe fed; with one buffer it is
+            // this tile.
+            if (next_load < ntiles && (nq == 1 || next_load - nq < ti)) {
+                const int prev = next_load - nq;
+                if (!wait_bar(BAR(B_QEMPTY + prev % nq), (uint32_t)(prev / nq) & 1u, abort_flag, st)) break;
+                load_q(next_load++);
+            }
         }
+        // Q loads still in flight after an abort land before the CTA exits (bounded)
+        for (int ti = consumed; ti < next_load; ++ti) drain_bar(BAR(B_QFULL + ti % nq), (uint32_t)(ti / nq) & 1u);
         if (lane == 0) mma_commit(BAR(B_FINAL));
         __syncwarp();
         drain_bar(BAR(B_FINAL), 0);
@@ -294,58 +337,81 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
             const uint32_t u = (uint32_t)(ti / NWG);
             if (!wait_bar(BAR(B_SFULL + wg), u & 1u, abort_flag, st)) break;
             tc_fence_after();
-            // lists sorted by (score descending, index ascending); inside a list columns arrive
-            // in increasing order and an equal score never displaces an earlier (lower) block
-            float val[KMAX], val2[KMAX];
-            int idx[KMAX], idx2[KMAX];
+            // pass 1: the n_route largest scores of the row, values only
+            float val[KMAX];
 #pragma unroll
-            for (int i = 0; i < KMAX; ++i) {
-                val[i] = val2[i] = -INFINITY;
-                idx[i] = idx2[i] = INT_MAX;
-            }
+            for (int i = 0; i < KMAX; ++i) val[i] = -INFINITY;
             for (int j0 = 0; j0 < c; j0 += 32) {
                 float v[32];
                 tmem_ld32(s_tmem + (uint32_t)j0, v);
-                if constexpr (kTwoLists) {
+                if (j0 + 32 > c) {
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        insert_desc<KMAX>(val, idx, v[e], j0 + e, j0 + e < c);
-                        insert_desc<KMAX>(val2, idx2, v[e + 1], j0 + e + 1, j0 + e + 1 < c);
-                    }
-                } else {
+                    for (int e = 0; e < 32; ++e) v[e] = (j0 + e < c) ? v[e] : -INFINITY;
+                }
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) insert_desc<KMAX>(val, idx, v[e], j0 + e, j0 + e < c);
+                for (int e = 0; e < 32; e += 2) top_values_pair<KMAX>(val, v[e], v[e + 1]);
+            }
+            // vk = val[n_route - 1], the smallest of the first n_route (val is descending)
+            float vk = val[0];
+#pragma unroll
+            for (int i = 1; i < KMAX; ++i) vk = fminf(vk, (i < n_route) ? val[i] : INFINITY);
+            // pass 2: the blocks scoring at least vk, as a bit mask in block order
+            uint32_t m[kWords];
+            int cnt = 0;
+#pragma unroll
+            for (int w = 0; w < kWords; ++w) {
+                m[w] = 0u;
+                if (w * 32 < c) {
+                    float v[32];
+                    tmem_ld32(s_tmem + (uint32_t)(w * 32), v);
+                    uint32_t mw = 0u;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) mw |= (v[e] >= vk) ? (1u << e) : 0u;
+                    if (c - w * 32 < 32) mw &= (1u << (c - w * 32)) - 1u;
+                    m[w] = mw;
+                    cnt += __popc(mw);
                 }
             }
-            if constexpr (kTwoLists) {
+            // scores equal to vk beyond the n_route places: the higher blocks drop out (ties
+            // keep the lower block index)
+            int excess = cnt - n_route;
+            if (__any_sync(0xffffffffu, excess > 0)) {
 #pragma unroll
-                for (int i = 0; i < KMAX; ++i) insert_ordered<KMAX>(val, idx, val2[i], idx2[i]);
+                for (int w = kWords - 1; w >= 0; --w) {
+                    if (w * 32 < c) {
+                        float v[32];
+                        tmem_ld32(s_tmem + (uint32_t)(w * 32), v);
+                        uint32_t eq = 0u;
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) eq |= (v[e] == vk) ? (1u << e) : 0u;
+                        eq &= m[w];
+                        while (excess > 0 && eq != 0u) {
+                            const uint32_t top = 1u << (31 - __clz(eq));
+                            m[w] &= ~top;
+                            eq &= ~top;
+                            --excess;
+                        }
+                    }
+                }
             }
             tc_fence_before();
             mbar_arrive(BAR(B_SEMPTY + wg));
             const int rr = qt * kTileM + r;
             if (rr < len) {
-                int o[KMAX];
-#pragma unroll
-                for (int i = 0; i < KMAX; ++i) o[i] = (i < n_route) ? idx[i] : INT_MAX;
-#pragma unroll
-                for (int p = 0; p < KMAX; ++p) {
-#pragma unroll
-                    for (int i = (p & 1); i + 1 < KMAX; i += 2) {
-                        const int lo = min(o[i], o[i + 1]), hi = max(o[i], o[i + 1]);
-                        o[i] = lo;
-                        o[i + 1] = hi;
-                    }
-                }
+                // routed blocks ascending, then the own block (pos < n_route only when the
+                // scores were not finite)
                 int* dst = sel + ((size_t)h * P.T + (start + rr)) * P.topk;
+                int pos = 0;
 #pragma unroll
-                for (int i = 0; i <= KMAX; ++i) {
-                    if (i < P.topk) {
-                        const int vo = (i < n_route) ? o[i < KMAX ? i : KMAX - 1] : (i == n_route ? c : -1);
-                        dst[i] = vo;
+                for (int w = 0; w < kWords; ++w) {
+                    uint32_t mw = m[w];
+                    while (mw != 0u && pos < n_route) {
+                        dst[pos++] = w * 32 + __ffs(mw) - 1;
+                        mw &= mw - 1u;
                     }
                 }
-                for (int i = KMAX + 1; i < P.topk; ++i) dst[i] = -1;
+                dst[pos] = c;
+                for (int i = pos + 1; i < P.topk; ++i) dst[i] = -1;
             }
         }
     }
@@ -379,16 +445,18 @@ template <int D, int KMAX, bool MINMAX, int NWG>
 cudaError_t launch_tc_w(const Problem& P, const CUtensorMap& mq, const GateSummary& s, const int* cu,
                         int* sel, int* status, int n_max, cudaStream_t st) {
     using C = GateCfg<D, MINMAX>;
-    // two Q buffers when they fit next to the summaries, else one
+    // as many Q buffers (up to kMaxQBuf) as fit next to the longest sequence's summaries; a CTA
+    // with fewer past blocks fits more into the same allocation
     const int limit = 227 * 1024;
-    const int nq = C::kBytes(2, n_max) <= limit ? 2 : 1;
+    int nq = kMaxQBuf;
+    while (nq > 1 && C::kBytes(nq, n_max) > limit) --nq;
     const int smem = C::kBytes(nq, n_max);
     cudaError_t e = cudaFuncSetAttribute(gate_tc_kernel<D, KMAX, MINMAX, NWG>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid(P.nb_cap, P.hkv);
     gate_tc_kernel<D, KMAX, MINMAX, NWG><<<grid, GateWarps<NWG>::kThreads, smem, st>>>(
-        mq, s.means, s.kmin, s.kmax, cu, P, sel, status, n_max, nq);
+        mq, s.means, s.kmin, s.kmax, cu, P, sel, status, n_max, smem);
     return cudaGetLastError();
 }
 
@@ -406,8 +474,9 @@ cudaError_t launch_tc(const Problem& P, const __nv_bfloat16* q, const GateSummar
            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    // four warpgroups while four score buffers fit TMEM and the lists are short, else two
-    if constexpr (KMAX <= 11) {
+    // four warpgroups while four score buffers fit TMEM and the lists are short (a longer list
+    // needs more than the 120 registers a thread of 544 may have), else two
+    if constexpr (KMAX <= 16) {
         if (pow2_at_least(n_max) <= 128)
             return launch_tc_w<D, KMAX, MINMAX, 4>(P, mq, s, cu, sel, status, n_max, st);
     }

@@ -98,7 +98,7 @@ long long blocks_bound(const moba_params& p) {
 
 struct Layout {
     size_t hdr, cu_blocks, blk_start, blk_len, blk_seq, blk_local, means, sel, counts, offsets,
-        cursor, entries, items, part_o, part_lse, nslots, total;
+        cursor, item_off, entries, items, part_o, part_lse, nslots, total;
     int wave;
     long long nb_cap, max_items;
 };
@@ -140,6 +140,7 @@ Layout make_layout(const moba_params& p) {
     L.counts = take(4ull * lists);
     L.offsets = take(4ull * (lists + 1));
     L.cursor = take(4ull * lists);
+    L.item_off = take(4ull * (lists + 1));
     L.entries = take(4ull * routed);
     L.items = take(sizeof(WorkItem) * L.max_items);
     L.part_o = take(2ull * W * p.num_q_heads * p.topk * p.head_dim);  // bf16
@@ -334,6 +335,7 @@ moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, co
     ws.counts = reinterpret_cast<int*>(base + L.counts);
     ws.offsets = reinterpret_cast<int*>(base + L.offsets);
     ws.cursor = reinterpret_cast<int*>(base + L.cursor);
+    ws.item_off = reinterpret_cast<int*>(base + L.item_off);
     ws.entries = reinterpret_cast<int*>(base + L.entries);
     ws.items = reinterpret_cast<WorkItem*>(base + L.items);
     ws.part_o = reinterpret_cast<__nv_bfloat16*>(base + L.part_o);
@@ -415,7 +417,7 @@ moba_status moba_attn_fwd(const moba_params* p, const void* q, const void* k, co
                      "merge launch");
         }
         MOBA_TRY(record(ev + 3), "event record");
-        launches += 5;
+        launches += 6;  // route count, plan, items, scatter; attention; merge
     }
 #undef MOBA_TRY
     if (info) {
@@ -431,7 +433,7 @@ namespace {
 
 struct BwdLayout {
     size_t hdr, cu_blocks, blk_start, blk_len, blk_seq, blk_local, counts, offsets, cursor,
-        entries, items, nslots, rs, dq_acc, total;
+        item_off, entries, items, nslots, rs, dq_acc, total;
     long long nb_cap, max_items;
 };
 
@@ -462,6 +464,7 @@ BwdLayout make_bwd_layout(const moba_params& p) {
     L.counts = take(4ull * lists);
     L.offsets = take(4ull * (lists + 1));
     L.cursor = take(4ull * lists);
+    L.item_off = take(4ull * (lists + 1));
     L.entries = take(4ull * T * p.num_q_heads * (p.topk - 1));
     L.items = take(sizeof(WorkItem) * L.max_items);
     L.nslots = take(1ull * T * p.num_q_heads);
@@ -517,6 +520,7 @@ moba_status moba_attn_bwd(const moba_params* p, const void* q, const void* k, co
     ws.counts = reinterpret_cast<int*>(base + L.counts);
     ws.offsets = reinterpret_cast<int*>(base + L.offsets);
     ws.cursor = reinterpret_cast<int*>(base + L.cursor);
+    ws.item_off = reinterpret_cast<int*>(base + L.item_off);
     ws.entries = reinterpret_cast<int*>(base + L.entries);
     ws.items = reinterpret_cast<WorkItem*>(base + L.items);
     ws.nslots = reinterpret_cast<unsigned char*>(base + L.nslots);

@@ -56,6 +56,7 @@ struct Workspace {
     int* counts;      // [hkv * nb_cap]
     int* offsets;     // [hkv * nb_cap + 1]
     int* cursor;      // [hkv * nb_cap]
+    int* item_off;    // [hkv * nb_cap + 1]: index of each list's first history work item
     int* entries;     // [wave * hq * (topk - 1)]
     WorkItem* items;  // [max_items]
     __nv_bfloat16* part_o;  // [wave * hq * topk, d]: normalised partial outputs

@@ -5,9 +5,10 @@
 // current block separately with a causal mask.  Here, per wave of query tokens [t0, t1):
 //
 //   route_count    histogram of routed rows per (KV head g, global block b)
-//   route_plan     exclusive scan -> list offsets; work items: the history items (<= 256 rows
-//                  of one list each), then the current-block items (one 128-token query tile
-//                  for one head, or for two heads of the same KV head), largest first
+//   route_plan     exclusive scans -> list offsets and each list's first work item; the
+//                  current-block items (one 128-token query tile for one head, or for two heads
+//                  of the same KV head), largest first, after the history items
+//   route_items    the history items (<= 256 rows of one list each), one thread per item
 //   route_scatter  writes each routed row's partial-output index into its list
 //
 // A routed entry is the row's partial-output index ((t - t0) * Hq + h) * topk + slot, where
@@ -198,7 +199,8 @@ route_plan_kernel(Problem P, Workspace ws, int t0, int t1) {
         carry += tot;
     }
     if (threadIdx.x == 0) ws.offsets[n_lists] = carry;
-    // 2. history items (up to two tiles of routed rows), list by list
+    // 2. history items (up to two tiles of routed rows), list by list: only each list's first
+    //    item index here; route_items_kernel writes the items themselves on the whole GPU
     int tcarry = 0;
     for (int base = 0; base < n_lists; base += kPlanThreads) {
         const int L = base + threadIdx.x;
@@ -206,19 +208,10 @@ route_plan_kernel(Problem P, Workspace ws, int t0, int t1) {
         const int nt = (cnt + kItemRows - 1) / kItemRows;
         int tot;
         const int ex = block_exclusive_scan(nt, s_warp, &tot);
-        if (L < n_lists && nt > 0) {
-            const int off = ws.offsets[L];
-            for (int i = 0; i < nt; ++i) {
-                WorkItem it;
-                it.a = L;
-                it.b = off + i * kItemRows;
-                it.c = min(kItemRows, cnt - i * kItemRows);
-                it.kind = 0;
-                ws.items[tcarry + ex + i] = it;
-            }
-        }
+        if (L < n_lists) ws.item_off[L] = tcarry + ex;
         tcarry += tot;
     }
+    if (threadIdx.x == 0) ws.item_off[n_lists] = tcarry;
     const int n_past = tcarry;
     // 3. current-block items of the blocks overlapping [t0, t1), by decreasing tile index
     //    (tile q has q + 1 key tiles of work)
@@ -320,6 +313,29 @@ route_plan_kernel(Problem P, Workspace ws, int t0, int t1) {
     }
 }
 
+// History work items of the wave, one thread per item: item i belongs to the last list L with
+// item_off[L] <= i (empty lists share their successor's offset), as its (i - item_off[L])-th
+// tile of up to kItemRows routed rows.
+__global__ void __launch_bounds__(256)
+route_items_kernel(Problem P, Workspace ws) {
+    const int n_lists = P.hkv * P.nb_cap;
+    const int n_past = ws.item_off[n_lists];
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_past; i += gridDim.x * blockDim.x) {
+        int lo = 0, hi = n_lists;  // answer in [lo, hi): item_off[lo] <= i < item_off[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldg(ws.item_off + mid) <= i) lo = mid; else hi = mid;
+        }
+        const int k = i - __ldg(ws.item_off + lo);
+        WorkItem it;
+        it.a = lo;
+        it.b = __ldg(ws.offsets + lo) + k * kItemRows;
+        it.c = min(kItemRows, __ldg(ws.counts + lo) - k * kItemRows);
+        it.kind = 0;
+        ws.items[i] = it;
+    }
+}
+
 template <bool kScatter>
 void launch_rows(const Problem& P, const int* cu, const int* sel, const Workspace& ws, int t0,
                  int t1, int grid, cudaStream_t st) {
@@ -356,6 +372,9 @@ cudaError_t launch_route_count(const Problem& P, const int* cu_seqlens, const in
 cudaError_t launch_route_plan(const Problem& P, const Workspace& ws, int t0, int t1,
                               cudaStream_t st) {
     route_plan_kernel<<<1, kPlanThreads, 0, st>>>(P, ws, t0, t1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    route_items_kernel<<<4 * 148, 256, 0, st>>>(P, ws);
     return cudaGetLastError();
 }
 
