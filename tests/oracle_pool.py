@@ -158,7 +158,7 @@ class _HeadRows:
     def __getitem__(self, idx):
         u, g = idx
         assert g == 0
-        return PT.from_bits(self.rows[np.asarray(u)])
+        return PT.from_bits64(self.rows[np.asarray(u)])
 
 
 def _select_compare_shared(qpath, h, means_g, gsel_h, cu, chunk, topk):

@@ -40,6 +40,17 @@ def from_bits(u16):
     return (np.asarray(u16).astype(np.uint32) << 16).view(np.float32)
 
 
+# every bf16 bit pattern's value as float64 (exact): one table lookup widens bf16 bits to
+# float64 in a single pass over the data
+with np.errstate(invalid="ignore"):  # the NaN patterns widen to NaN, as they should
+    BF16_TO_F64 = (np.arange(1 << 16, dtype=np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def from_bits64(u16):
+    """uint16 bf16 bit patterns -> float64 (exact), through BF16_TO_F64."""
+    return BF16_TO_F64[np.asarray(u16)]
+
+
 def check_means(gpu_means, k_np, cu, chunk, oracle_means):
     """Means within the fp32 summation bound of the float64 oracle."""
     tab = oracle.block_table(cu, chunk)
