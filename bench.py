@@ -259,6 +259,42 @@ def cpu_oracle_baseline(w, budget_s, seed=0, inputs=None, dense=False):
     return T / seconds, detail
 
 
+def dense_reference_rates(names=("tiny_2k", "scaling_8k", "long_32k")):
+    """The dense causal fp64 reference (the oracle with every block selected) on the small
+    configurations, timed on the host cores: one query head per workload in a worker process,
+    extrapolated to all heads on all processes.  Returns {workload: tokens/s} and the note."""
+    import numpy as np
+    import torch
+
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import oracle_pool as OP
+    from block_sparse_long_meanpool_b200 import workloads as W
+
+    bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    rates = {}
+    workers = OP.n_workers()
+    with OP.pool() as ex:
+        list(ex.map(int, range(workers)))
+        for name in names:
+            w = W.ALL_WORKLOADS[name]
+            x = W.make_inputs(w, device="cpu")
+            q16, k16, v16 = bits(x["q"]), bits(x["k"]), bits(x["v"])
+            cu = np.asarray(w.cu_seqlens)
+            T, chunk = w.total_tokens, w.chunk_size
+            nb = max((int(cu[i + 1] - cu[i]) + chunk - 1) // chunk for i in range(len(cu) - 1))
+            all_sel = np.full((T, nb), -1, dtype=np.int64)
+            for i in range(len(cu) - 1):
+                c = (np.arange(cu[i], cu[i + 1]) - cu[i]) // chunk
+                all_sel[cu[i]:cu[i + 1]] = np.where(np.arange(nb)[None, :] <= c[:, None], np.arange(nb)[None, :], -1)
+            _, c = ex.submit(OP.timed, "_dense_head", np.ascontiguousarray(q16[:, 0]),
+                             np.ascontiguousarray(k16[:, 0]), np.ascontiguousarray(v16[:, 0]), cu, chunk,
+                             all_sel, None).result()
+            rates[name] = T / (c * w.num_q_heads / workers)
+    note = ("dense causal attention in float64 (the oracle with every block selected) on the small "
+            "configurations: one query head timed in a worker, x heads / processes")
+    return rates, note
+
+
 def run_reference(args, w, world, rank):
     """--impl reference: the float64 CPU oracle on a bounded sample, rank 0 only."""
     if rank != 0:
@@ -634,6 +670,10 @@ def run_ours(args, w, world, rank, local):
         if "dense_causal_fp64_tokens_per_s" in det:
             cpu["dense_causal_fp64_tokens_per_s"] = det["dense_causal_fp64_tokens_per_s"]
             cpu["dense_causal_fp64_note"] = det["dense_causal_fp64_note"]
+        else:
+            rates, note = dense_reference_rates()
+            cpu["dense_causal_fp64_small_configs_tokens_per_s"] = rates
+            cpu["dense_causal_fp64_note"] = note
 
     if rank == 0:
         line = {
