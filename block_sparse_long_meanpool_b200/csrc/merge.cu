@@ -7,11 +7,11 @@
 //   lse = m + log(sum_i w_i).
 // The partial outputs o_i are bf16 (the precision an attention call returns its output in),
 // the lse_i fp32; the combination is computed in fp32.
-// A half-warp per query row (two rows per warp): the first partial rows are loaded before the
-// weights are known, lane s reads slot s's lse (and s + 16), the maximum and the weights come
-// from half-warp reductions, and each lane accumulates d/16 consecutive channels with four
-// partial rows in flight (streaming loads).  The output is rounded once to bf16 (nearest
-// even).  HBM-bound.
+// A half-warp per query row (two rows per warp), the row's slot count loaded while the previous
+// row is merged: the first partial rows are loaded before the weights are known, lane s reads
+// slot s's lse (and s + 16), the maximum and the weights come from half-warp reductions, and
+// each lane accumulates d/16 consecutive channels with four partial rows in flight (streaming
+// loads).  The output is rounded once to bf16 (nearest even).  HBM-bound.
 #include "moba_internal.cuh"
 
 namespace moba {
@@ -53,10 +53,15 @@ merge_kernel(const int* __restrict__ cu, const int* __restrict__ sel, Problem P,
     const int hl = lane & 15, half = lane >> 4;
     const long long n = (long long)(t1 - t0) * P.hq;
     const long long stride = (long long)gridDim.x * kWarps * 2;
-    for (long long base = ((long long)blockIdx.x * kWarps + warp) * 2; base < n; base += stride) {
+    long long base = ((long long)blockIdx.x * kWarps + warp) * 2;
+    // slot count (own block + routed history blocks) of this half-warp's next row, loaded one
+    // row ahead so that the partial rows' loads do not wait for it
+    int ns_next = (base + half < n) ? (int)ws.nslots[base + half] : 0;
+    for (; base < n; base += stride) {
         const long long r = base + half;
         const bool valid = r < n;
-        const int ns = valid ? (int)ws.nslots[r] : 0;  // own block + routed history blocks
+        const int ns = ns_next;
+        ns_next = (r + stride < n) ? (int)ws.nslots[r + stride] : 0;
         const size_t pbase = (size_t)(valid ? r : 0) * P.topk;
         const __nv_bfloat16* obase = ws.part_o + pbase * D + hl * V;
         // first partial rows in flight before the weights are known
