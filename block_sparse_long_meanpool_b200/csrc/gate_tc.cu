@@ -45,6 +45,7 @@ using namespace ptx;
 constexpr int kMaxPast = 256;   // past blocks scored in one MMA (N <= 256)
 constexpr int kWords = kMaxPast / 32;  // a row's past blocks as a bit mask
 constexpr int kMaxQBuf = 4;            // Q tile buffers (loads run ahead of the MMAs)
+constexpr int kHalfSmLimit = 113 * 1024;  // dynamic shared memory of one of two CTAs per SM
 
 // The K largest values seen so far, descending (-inf until K were seen).  Adding a pair is a
 // merge with the sorted two-element list (a, b), a >= b: the i-th largest of the union is
@@ -99,8 +100,8 @@ __device__ __forceinline__ void split_sign(uint32_t x, uint32_t& pos, uint32_t& 
     neg = x & m;
 }
 
-template <int D, int KMAX, bool MINMAX, int NWG>
-__global__ void __launch_bounds__(GateWarps<NWG>::kThreads, 1)
+template <int D, int KMAX, bool MINMAX, int NWG, int MINB>
+__global__ void __launch_bounds__(GateWarps<NWG>::kThreads, MINB)
 gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restrict__ means,
                const __nv_bfloat16* __restrict__ kmin, const __nv_bfloat16* __restrict__ kmax,
                const int* __restrict__ cu, Problem P, int* __restrict__ sel, int* status, int n_cap,
@@ -441,21 +442,23 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-template <int D, int KMAX, bool MINMAX, int NWG>
+// MINB CTAs per SM: with MINB = 2 the launch keeps to half an SM's shared memory (and the
+// kernel to half its registers) so that a second CTA's loads overlap this one's compute.
+template <int D, int KMAX, bool MINMAX, int NWG, int MINB>
 cudaError_t launch_tc_w(const Problem& P, const CUtensorMap& mq, const GateSummary& s, const int* cu,
                         int* sel, int* status, int n_max, cudaStream_t st) {
     using C = GateCfg<D, MINMAX>;
     // as many Q buffers (up to kMaxQBuf) as fit next to the longest sequence's summaries; a CTA
     // with fewer past blocks fits more into the same allocation
-    const int limit = 227 * 1024;
-    int nq = kMaxQBuf;
+    const int limit = MINB == 1 ? 227 * 1024 : kHalfSmLimit;
+    int nq = MINB == 1 ? kMaxQBuf : 2;
     while (nq > 1 && C::kBytes(nq, n_max) > limit) --nq;
     const int smem = C::kBytes(nq, n_max);
-    cudaError_t e = cudaFuncSetAttribute(gate_tc_kernel<D, KMAX, MINMAX, NWG>,
+    cudaError_t e = cudaFuncSetAttribute(gate_tc_kernel<D, KMAX, MINMAX, NWG, MINB>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid(P.nb_cap, P.hkv);
-    gate_tc_kernel<D, KMAX, MINMAX, NWG><<<grid, GateWarps<NWG>::kThreads, smem, st>>>(
+    gate_tc_kernel<D, KMAX, MINMAX, NWG, MINB><<<grid, GateWarps<NWG>::kThreads, smem, st>>>(
         mq, s.means, s.kmin, s.kmax, cu, P, sel, status, n_max, smem);
     return cudaGetLastError();
 }
@@ -474,13 +477,20 @@ cudaError_t launch_tc(const Problem& P, const __nv_bfloat16* q, const GateSummar
            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    // four warpgroups while four score buffers fit TMEM and the lists are short (a longer list
-    // needs more than the 120 registers a thread of 544 may have), else two
+    using C = GateCfg<D, MINMAX>;
     if constexpr (KMAX <= 16) {
+        // few query tiles per CTA (short blocks, small groups): each CTA is short and mostly
+        // waits for its loads, so two CTAs of two warpgroups share an SM when half its shared
+        // memory holds one
+        const int tiles = (P.chunk + kTileM - 1) / kTileM * P.group;
+        if (tiles <= 16 && C::kBytes(1, n_max) <= kHalfSmLimit)
+            return launch_tc_w<D, KMAX, MINMAX, 2, 2>(P, mq, s, cu, sel, status, n_max, st);
+        // four warpgroups while four score buffers fit TMEM and the lists are short (a longer
+        // list needs more than the 120 registers a thread of 544 may have), else two
         if (pow2_at_least(n_max) <= 128)
-            return launch_tc_w<D, KMAX, MINMAX, 4>(P, mq, s, cu, sel, status, n_max, st);
+            return launch_tc_w<D, KMAX, MINMAX, 4, 1>(P, mq, s, cu, sel, status, n_max, st);
     }
-    return launch_tc_w<D, KMAX, MINMAX, 2>(P, mq, s, cu, sel, status, n_max, st);
+    return launch_tc_w<D, KMAX, MINMAX, 2, 1>(P, mq, s, cu, sel, status, n_max, st);
 }
 
 template <int D, bool MINMAX>
