@@ -14,8 +14,9 @@
 //   bwd_rowstats_kernel  per row: lse * log2(e) and Dp (reads dO and out; HBM stream)
 //   bwd_dkdv_kernel      one CTA per (KV head, block, 128-key tile).  It streams every query
 //                        row attending the tile in 64-row tiles (routed rows of the block's
-//                        list, then the block's own rows of the group's heads) and computes,
-//                        with the keys on the TMEM lanes:
+//                        list, then the block's own rows of the group's heads; two warps
+//                        gather alternate row tiles, Q and dO together, by cp.async into a
+//                        3-stage ring) and computes, with the keys on the TMEM lanes:
 //                          S^T = K Q^T, dP^T = V dO^T            (SS MMA, M = 128 keys, N = 64)
 //                          P^T, dS^T                             (8 warps, thread = key)
 //                          dV += P^T dO, dK += dS^T Q            (TS MMA, A from TMEM)
@@ -179,7 +180,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constan
     if (threadIdx.x == 0) {
         mbar_init(BAR(B_KV), 1);
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(BAR(B_FULL + i), 64);  // the Q and the dO gather warps
+            mbar_init(BAR(B_FULL + i), 32);  // the gather warp of the tile
             mbar_init(BAR(B_EMPTY + i), 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -220,35 +221,35 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constan
         tok = t;
         return true;
     };
-    // cp.async gather of the 64 rows of tile i into a [64 x D] K-major SW128 tile (one warp)
-    auto gather = [&](const __nv_bfloat16* src_base, uint32_t dst_tile, int i, bool stats) {
+    // cp.async gather of the 64 rows of tile i, Q and dO, into [64 x D] K-major SW128 tiles at
+    // q_tile and q_tile + kQT, with the rows' statistics (one warp; each row is resolved once)
+    auto gather = [&](uint32_t q_tile, int i) {
         constexpr int CK = D / 8;
 #pragma unroll 1
         for (int r = lane; r < kQRows; r += 32) {
             int t = 0, h = 0, tok = -1;
             const bool valid = row_of(i, r, t, h, tok);
-            const __nv_bfloat16* src = valid ? src_base + ((long long)t * P.hq + h) * D : src_base;
-            const uint32_t rbase = dst_tile + (uint32_t)r * 128u;
+            const long long ro = valid ? ((long long)t * P.hq + h) * D : 0;
+            const uint32_t rbase = q_tile + (uint32_t)r * 128u;
 #pragma unroll
             for (int cc = 0; cc < CK; ++cc) {
                 const uint32_t dst = rbase + (uint32_t)(cc >> 3) * kHalfQ + (uint32_t)(((cc & 7) ^ (r & 7)) << 4);
-                cp_async16(dst, src + (valid ? cc * 8 : 0), valid);
+                cp_async16(dst, q + ro + (valid ? cc * 8 : 0), valid);
+                cp_async16(dst + (uint32_t)L::kQT, dout + ro + (valid ? cc * 8 : 0), valid);
             }
-            if (stats) {
-                RowInfo ri;
-                if (valid) {
-                    const float2 st = rs[(size_t)h * P.T + t];
-                    ri.lse2 = st.x;
-                    ri.dp = st.y;
-                    ri.tok = tok;
-                } else {
-                    ri.lse2 = 0.f;
-                    ri.dp = 0.f;
-                    ri.tok = -1;
-                }
-                ri.pad = 0;
-                rinfo[(i % kStages) * kQRows + r] = ri;
+            RowInfo ri;
+            if (valid) {
+                const float2 st = rs[(size_t)h * P.T + t];
+                ri.lse2 = st.x;
+                ri.dp = st.y;
+                ri.tok = tok;
+            } else {
+                ri.lse2 = 0.f;
+                ri.dp = 0.f;
+                ri.tok = -1;
             }
+            ri.pad = 0;
+            rinfo[(i % kStages) * kQRows + r] = ri;
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
         asm volatile("cp.async.wait_group 0;" ::: "memory");
@@ -256,10 +257,9 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constan
     };
 
     if (warp >= 8) {
-        if (warp == 8 || warp == 10) {
-            // ---------------- K / V tile (warp 10, once) and the Q / dO row stream ----------------
-            const bool is_q = warp == 8;
-            if (!is_q && lane == 0) {
+        if (warp == 10) {
+            // ---------------- K / V tile (once) ----------------
+            if (lane == 0) {
                 mbar_arrive_tx(BAR(B_KV), 2u * L::kKV);
 #pragma unroll
                 for (int hh = 0; hh < D / 64; ++hh) {
@@ -268,16 +268,17 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constan
                 }
             }
             __syncwarp();
-            for (int i = 0; i < n_tiles; ++i) {
+            drain_bar(BAR(B_KV), 0);  // the K / V tile must land before the CTA exits
+        } else if (warp == 8 || warp == 11) {
+            // ---------------- the Q / dO row stream: warp 8 even tiles, warp 11 odd ones ----------------
+            for (int i = (warp == 8 ? 0 : 1); i < n_tiles; i += 2) {
                 const int s = i % kStages;
                 if (i >= kStages &&
                     !wait_bar(BAR(B_EMPTY + s), (uint32_t)((i / kStages) - 1) & 1u, abort_flag, status))
                     break;
-                const uint32_t tile = sm_base + L::kRing + (uint32_t)s * 2u * L::kQT + (is_q ? 0u : (uint32_t)L::kQT);
-                gather(is_q ? q : dout, tile, i, is_q);
+                gather(sm_base + L::kRing + (uint32_t)s * 2u * L::kQT, i);
                 mbar_arrive(BAR(B_FULL + s));
             }
-            if (!is_q) drain_bar(BAR(B_KV), 0);  // the K / V tile must land before the CTA exits
         } else if (warp == 9) {
             // ---------------- MMA issuer (one thread) ----------------
             if (lane == 0) {
@@ -345,7 +346,6 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constan
             }
             __syncwarp();
         }
-        // warp 11 has no role here
     } else {
         // ---------------- P^T, dS^T (thread = key), then the dK / dV epilogue ----------------
         const int wg = warp >> 2, quad = warp & 3;
