@@ -14,9 +14,9 @@
 //   bwd_rowstats_kernel  per row: lse * log2(e) and Dp (reads dO and out; HBM stream)
 //   bwd_dkdv_kernel      one CTA per (KV head, block, 128-key tile).  It streams every query
 //                        row attending the tile in 64-row tiles (routed rows of the block's
-//                        list, then the block's own rows of the group's heads; two warps
-//                        gather alternate row tiles, Q and dO together, by cp.async into a
-//                        3-stage ring) and computes, with the keys on the TMEM lanes:
+//                        list, then the block's own rows of the group's heads; three warps,
+//                        one per stage of a 3-stage ring, gather row tiles in turn, Q and dO
+//                        together, by cp.async) and computes, with the keys on the TMEM lanes:
 //                          S^T = K Q^T, dP^T = V dO^T            (SS MMA, M = 128 keys, N = 64)
 //                          P^T, dS^T                             (8 warps, thread = key)
 //                          dV += P^T dO, dK += dS^T Q            (TS MMA, A from TMEM)
@@ -108,6 +108,7 @@ bwd_rowstats_kernel(const __nv_bfloat16* __restrict__ out, const __nv_bfloat16* 
 
 constexpr int kQRows = 64;   // query rows per tile of the dK/dV stream (MMA N)
 constexpr int kStages = 3;   // ring of (Q, dO, row info) tiles
+static_assert(kStages == 3, "one dK/dV gather warp per ring stage (warps 8, 10 and 11)");
 
 struct RowInfo {
     float lse2;  // lse * log2 e
@@ -257,21 +258,23 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constan
     };
 
     if (warp >= 8) {
-        if (warp == 10) {
-            // ---------------- K / V tile (once) ----------------
-            if (lane == 0) {
-                mbar_arrive_tx(BAR(B_KV), 2u * L::kKV);
+        if (warp == 8 || warp == 10 || warp == 11) {
+            // ---------------- K / V tile (warp 10, once) and the Q / dO row stream ----------------
+            // three gather warps, one per ring stage: warp 8 takes tiles 0, 3, 6, ..., warp 10
+            // tiles 1, 4, ..., warp 11 tiles 2, 5, ...
+            if (warp == 10) {
+                if (lane == 0) {
+                    mbar_arrive_tx(BAR(B_KV), 2u * L::kKV);
 #pragma unroll
-                for (int hh = 0; hh < D / 64; ++hh) {
-                    tma_load_3d(sm_base + L::kK + hh * kHalfKV, &tmap_k, BAR(B_KV), hh * 64, g, ks);
-                    tma_load_3d(sm_base + L::kV + hh * kHalfKV, &tmap_v, BAR(B_KV), hh * 64, g, ks);
+                    for (int hh = 0; hh < D / 64; ++hh) {
+                        tma_load_3d(sm_base + L::kK + hh * kHalfKV, &tmap_k, BAR(B_KV), hh * 64, g, ks);
+                        tma_load_3d(sm_base + L::kV + hh * kHalfKV, &tmap_v, BAR(B_KV), hh * 64, g, ks);
+                    }
                 }
+                __syncwarp();
             }
-            __syncwarp();
-            drain_bar(BAR(B_KV), 0);  // the K / V tile must land before the CTA exits
-        } else if (warp == 8 || warp == 11) {
-            // ---------------- the Q / dO row stream: warp 8 even tiles, warp 11 odd ones ----------------
-            for (int i = (warp == 8 ? 0 : 1); i < n_tiles; i += 2) {
+            const int first = warp == 8 ? 0 : (warp == 10 ? 1 : 2);
+            for (int i = first; i < n_tiles; i += kStages) {
                 const int s = i % kStages;
                 if (i >= kStages &&
                     !wait_bar(BAR(B_EMPTY + s), (uint32_t)((i / kStages) - 1) & 1u, abort_flag, status))
@@ -279,6 +282,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constan
                 gather(sm_base + L::kRing + (uint32_t)s * 2u * L::kQT, i);
                 mbar_arrive(BAR(B_FULL + s));
             }
+            if (warp == 10) drain_bar(BAR(B_KV), 0);  // the K / V tile must land before the CTA exits
         } else if (warp == 9) {
             // ---------------- MMA issuer (one thread) ----------------
             if (lane == 0) {
