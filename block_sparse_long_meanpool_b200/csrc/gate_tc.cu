@@ -24,7 +24,8 @@
 // gate, splits it into q+ and q-) and issues the MMAs (N = c rounded up to 16) into TMEM.  The
 // top-(topk-1) is chosen by warpgroups that take whole tiles in turn, each with its own TMEM
 // score buffer (four warpgroups while four buffers fit TMEM, i.e. up to 128 past blocks, and the
-// lists are short; two otherwise), thread = row = TMEM lane, in two passes over the row's
+// lists are short; two otherwise, or two CTAs of two per SM when a CTA has few tiles and half an
+// SM's shared memory holds it), thread = row = TMEM lane, in two passes over the row's
 // scores: the first keeps the topk-1 largest values (a min/max merge network, no indices), the
 // second marks the blocks scoring at least the smallest of them; when equal scores at the cut
 // mark too many, the highest such blocks are dropped, so ties keep the lower block index.  The
@@ -140,9 +141,9 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const float* __restri
 
     if (n_route == c || n_route == 0 || c > n_cap) {
         // nothing to choose: every past block is routed (c <= topk - 1), or none (topk = 1).
-        // c > n_cap means the
-        // sequence is longer than the caller's max_seqlen promised: its rows keep the own block
-        // only and the call's status word (when there is one) records the broken promise.
+        // c > n_cap means the sequence is longer than the caller's max_seqlen promised: its rows
+        // keep the own block only and the call's status word (when there is one) records the
+        // broken promise.
         const bool broken = c > n_cap;
         if (broken && threadIdx.x == 0 && status) atomicExch(status, 1 /* INVALID_ARG */);
         for (int e = threadIdx.x; e < len * P.group; e += kThreads) {
