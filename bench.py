@@ -425,6 +425,56 @@ def _sub_forward(moba, W, w, dev, steps, warmup, peaks, gate="mean", max_seqlen=
     return rec
 
 
+def _sub_decode(moba, W, w, dev, peaks, gate="mean", steps=50, warmup=5):
+    """A decode-step sub-record on decode workload w (caches larger than L2): one moba_decode_fwd
+    (or moba_decode_minmax_fwd) per step, the cache summary built outside the timing, as
+    `bench.py --decode` times it; sequences/s and the HBM rate of the attended K/V bytes."""
+    import torch
+
+    x = W.make_inputs(w, device=dev)
+    k, v, cu = x["k"], x["v"], x["cu_seqlens"]
+    B, hq, hkv, d = len(w.seqlens), w.num_q_heads, w.num_kv_heads, w.head_dim
+    chunk, topk = w.chunk_size, w.topk
+    last = torch.tensor([c - 1 for c in w.cu_seqlens[1:]], device=dev)
+    q_new = x["q"][last].contiguous()
+    del x
+    if gate == "minmax":
+        k_min, k_max = moba.minmaxpool(k, cu, chunk)
+    else:
+        means = moba.meanpool(k, cu, chunk)
+    p = moba.make_params(B, w.total_tokens, hq, hkv, d, chunk, topk)
+    ws = torch.empty(moba.load_library().moba_decode_workspace_size(p), dtype=torch.uint8, device=dev)
+    out = torch.empty((B, hq, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((hq, B), dtype=torch.float32, device=dev)
+
+    def step():
+        if gate == "minmax":
+            moba.decode_minmax_fwd(q_new, k, v, cu, k_min, k_max, chunk, topk, workspace=ws, out=out, lse=lse)
+        else:
+            moba.decode_fwd(q_new, k, v, cu, means, chunk, topk, workspace=ws, out=out, lse=lse)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    keys = W.decode_attended_keys(w.seqlens, chunk, topk)
+    algo_bytes = keys * hq * d * 2 * 2 + B * hq * d * 2 + B * hq * (d * 2 + 4)
+    gbs = algo_bytes / (ms * 1e-3) / 1e9
+    rec = {"workload": w.name, "gate": gate, "steps": steps, "ms_per_step": ms,
+           "sequences_per_s": B / (ms * 1e-3), "algorithmic_bytes": algo_bytes, "GB/s": gbs,
+           "hbm_frac": gbs / peaks["hbm_gbs"]}
+    del k, v, ws, out, lse
+    torch.cuda.empty_cache()
+    return rec
+
+
 def _sub_backward(moba, W, w, x, dev, peaks, steps=3, warmup=3):
     """A backward sub-record on workload w: the forward runs once (outside the timing) for
     out, lse and its selection; then moba_attn_bwd is timed.  TF/s counts the algorithmic
@@ -658,6 +708,9 @@ def run_ours(args, w, world, rank, local):
             subs["minmax_gate"] = _sub_forward(moba, W, w, dev, 3, 3, peaks, gate="minmax",
                                                max_seqlen=max_seqlen, seed=rank_seed(w, rank))
         subs["backward"] = _sub_backward(moba, W, w, x, dev, peaks)
+        dw = W.DECODE_WORKLOADS["decode_32k_b64"]
+        subs["decode_32k_b64"] = _sub_decode(moba, W, dw, dev, peaks)
+        subs["decode_32k_b64_minmax"] = _sub_decode(moba, W, dw, dev, peaks, gate="minmax")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
