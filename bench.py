@@ -708,6 +708,14 @@ def run_ours(args, w, world, rank, local):
             subs["minmax_gate"] = _sub_forward(moba, W, w, dev, 3, 3, peaks, gate="minmax",
                                                max_seqlen=max_seqlen, seed=rank_seed(w, rank))
         subs["backward"] = _sub_backward(moba, W, w, x, dev, peaks)
+        # the paper's block-granularity sweep at 32K (fixed sparsity, blocks of 4096 down to 256)
+        sweep = {}
+        for gw in W.GRANULARITY_32K.values():
+            r = _sub_forward(moba, W, gw, dev, 10, 3, peaks, max_seqlen=gw.max_seqlen)
+            sweep[gw.name] = {"tokens_per_s": r["tokens_per_s"], "ms_per_step": r["ms_per_step"],
+                              "attention_tflops": r["attention_tflops"],
+                              "attention_frac": r["attention_frac"], "stage_ms": r["stage_ms"]}
+        subs["granularity_32k"] = sweep
         dw = W.DECODE_WORKLOADS["decode_32k_b64"]
         subs["decode_32k_b64"] = _sub_decode(moba, W, dw, dev, peaks)
         subs["decode_32k_b64_minmax"] = _sub_decode(moba, W, dw, dev, peaks, gate="minmax")
